@@ -1,0 +1,187 @@
+"""CPU oracle for block-sparse causal attention forward (test infrastructure).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its binding) never touches it, and the two share no code.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64, OpenMP); this module only
+builds it with gcc and marshals numpy arrays.  What each function computes, and
+the passage of the pages it follows, is stated in ``oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+
+class OraclePattern(ctypes.Structure):
+    _fields_ = [
+        ("causal", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("sinks", ctypes.c_int32),
+        ("stride", ctypes.c_int32),
+        ("n_global", ctypes.c_int32),
+        ("global_rows_see_all", ctypes.c_int32),
+    ]
+
+
+@dataclass(frozen=True)
+class Pattern:
+    """A fixed sparsity pattern: causal band of width ``window`` (inclusive,
+    -1 for none), ``sinks`` leading key tokens, every ``stride``-th prior token
+    (0 for none) and ``n_global`` global tokens."""
+
+    window: int = -1
+    sinks: int = 0
+    stride: int = 0
+    n_global: int = 0
+    causal: int = 1
+    global_rows_see_all: int = 0
+
+    def c(self) -> OraclePattern:
+        return OraclePattern(self.causal, self.window, self.sinks, self.stride,
+                             self.n_global, self.global_rows_see_all)
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class Oracle:
+    """The compiled oracle at ``path`` (the default build, or a test's mutant)."""
+
+    def __init__(self, path: str):
+        L = ctypes.CDLL(path)
+        P = ctypes.POINTER(OraclePattern)
+        L.oracle_allowed.argtypes = [P, ctypes.c_int64, ctypes.c_int64]
+        L.oracle_allowed.restype = ctypes.c_int
+        L.oracle_count_pairs.argtypes = [P, ctypes.c_int64]
+        L.oracle_count_pairs.restype = ctypes.c_int64
+        L.oracle_block_mask.argtypes = [P, ctypes.c_int64, ctypes.c_int32,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        L.oracle_block_mask.restype = ctypes.c_int64
+        L.oracle_attention.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.c_int64, ctypes.c_int64, P, ctypes.c_double,
+                                       ctypes.c_void_p, ctypes.c_int64,
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
+        L.oracle_attention.restype = ctypes.c_int
+        L.oracle_max_threads.argtypes = []
+        L.oracle_max_threads.restype = ctypes.c_int
+        self.L = L
+
+    def allowed(self, p: Pattern, q: int, kv: int) -> bool:
+        r = self.L.oracle_allowed(ctypes.byref(p.c()), q, kv)
+        if r < 0:
+            raise ValueError("pattern not defined by the oracle")
+        return bool(r)
+
+    def count_pairs(self, p: Pattern, N: int) -> int:
+        return int(self.L.oracle_count_pairs(ctypes.byref(p.c()), N))
+
+    def block_mask(self, p: Pattern, N: int, block: int):
+        """Brute-force tile classification -> (counts[T], index[T, T], full[T, T])."""
+        T = (N + block - 1) // block
+        counts = np.zeros(T, dtype=np.int32)
+        index = np.zeros((T, T), dtype=np.int32)
+        full = np.zeros((T, T), dtype=np.uint8)
+        live = self.L.oracle_block_mask(ctypes.byref(p.c()), N, block, counts.ctypes.data,
+                                        index.ctypes.data, full.ctypes.data)
+        if live < 0:
+            raise ValueError("bad block-mask arguments")
+        return counts, index, full
+
+    def attention(self, q: np.ndarray, k: np.ndarray, v: np.ndarray, p: Pattern, scale: float,
+                  rows: np.ndarray | None = None, n_threads: int = 0):
+        """fp64 attention by definition.
+
+        q: uint16 bf16 bits [B, Hq, N, D]; k, v: [B, Hkv, N, D].
+        rows: optional int64 query positions.  Returns (O [B, Hq, R, D] float64,
+        LSE [B, Hq, R] float64) with R = len(rows) or N.
+        """
+        for t in (q, k, v):
+            if t.dtype != np.uint16 or not t.flags.c_contiguous:
+                raise TypeError("inputs must be contiguous uint16 (bf16 bit patterns)")
+        B, Hq, N, D = q.shape
+        Hkv = k.shape[1]
+        if k.shape != (B, Hkv, N, D) or v.shape != k.shape:
+            raise ValueError("shape mismatch")
+        if rows is None:
+            R = N
+            rows_ptr = None
+        else:
+            rows = np.ascontiguousarray(rows, dtype=np.int64)
+            R = rows.shape[0]
+            if R and (rows.min() < 0 or rows.max() >= N):
+                raise ValueError("row out of range")
+            rows_ptr = rows.ctypes.data
+        O = np.empty((B, Hq, R, D), dtype=np.float64)
+        LSE = np.empty((B, Hq, R), dtype=np.float64)
+        rc = self.L.oracle_attention(q.ctypes.data, k.ctypes.data, v.ctypes.data, B, Hq, Hkv, N, D,
+                                     ctypes.byref(p.c()), float(scale), rows_ptr, R,
+                                     O.ctypes.data, LSE.ctypes.data, int(n_threads))
+        if rc != 0:
+            raise ValueError("bad attention arguments")
+        return O, LSE
+
+    def max_threads(self) -> int:
+        return int(self.L.oracle_max_threads())
+
+
+_default = None
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle(build())
+    return _default
+
+
+def allowed(p: Pattern, q: int, kv: int) -> bool:
+    return default().allowed(p, q, kv)
+
+
+def count_pairs(p: Pattern, N: int) -> int:
+    return default().count_pairs(p, N)
+
+
+def block_mask(p: Pattern, N: int, block: int):
+    return default().block_mask(p, N, block)
+
+
+def attention(q, k, v, p: Pattern, scale: float, rows=None, n_threads: int = 0):
+    return default().attention(q, k, v, p, scale, rows=rows, n_threads=n_threads)
+
+
+def max_threads() -> int:
+    return default().max_threads()
+
+
+def compile_source(src_text: str, out_path: str) -> str:
+    """Compile oracle source text (a test's mutant of oracle.c) to ``out_path``."""
+    c_path = out_path + ".c"
+    with open(c_path, "w") as f:
+        f.write(src_text)
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                           "-o", out_path, c_path, "-lm"])
+    return out_path
+
+
+def source() -> str:
+    with open(_SRC) as f:
+        return f.read()

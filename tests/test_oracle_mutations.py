@@ -1,0 +1,87 @@
+"""Plant plausible mistakes in copies of the oracle (on the CPU) and check that
+the pins catch each one: a wrong window bound, sink bound, stride reading, LSE
+base, head mapping, missing scale, or tile-fullness test.  A pin set that let
+one of these through would not be pinning the oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from oracle import Pattern
+
+from test_oracle import (closed_live_window_sinks, closed_pairs_window_sinks,
+                         closed_row_count_strided, rule_sets)
+
+MUTANTS = {
+    "window_exclusive": ("delta <= p->window", "delta < p->window"),
+    "sinks_inclusive": ("if (kv < p->sinks)", "if (kv <= p->sinks)"),
+    "stride_absolute": ("delta % p->stride == 0", "kv % p->stride == 0"),
+    "lse_base2": ("*lse = m + log(l);", "*lse = m + log2(l);"),
+    "head_map_modulo": ("int64_t hkv = hq / group;", "int64_t hkv = hq % Hkv;"),
+    "scale_dropped": ("s[t] = scale * dot;", "s[t] = dot;"),
+    "full_ignores_ragged": ("full[i * T + c] = allowed == (q1 - q0) * (k1 - k0);",
+                            "full[i * T + c] = allowed == (int64_t)block * block;"),
+}
+
+
+def pins_hold(o: oracle.Oracle) -> bool:
+    """A compact run of the pins; False as soon as one fails."""
+    # printed figure
+    counts, _, _ = o.block_mask(Pattern(window=1024, sinks=4), 8192, 128)
+    if counts.sum() != 595:
+        return False
+    # closed forms
+    if o.count_pairs(Pattern(window=50, sinks=4), 600) != closed_pairs_window_sinks(600, 50, 4):
+        return False
+    if o.count_pairs(Pattern(window=10, stride=7, n_global=3), 300) != sum(
+            closed_row_count_strided(q, 10, 7, 3) for q in range(300)):
+        return False
+    counts, _, _ = o.block_mask(Pattern(window=100, sinks=3), 1000, 64)
+    if counts.sum() != closed_live_window_sinks(16, 100, 64, 3):
+        return False
+    # brute force on ragged tiny cases (the second has full ragged tiles)
+    for p, N, b in [(Pattern(window=3, sinks=2), 37, 8), (Pattern(window=30, sinks=2), 37, 8)]:
+        sets = [rule_sets(N, q, p) for q in range(N)]
+        counts, index, full = o.block_mask(p, N, b)
+        for i in range(-(-N // b)):
+            for c in range(counts[i]):
+                j = index[i, c]
+                qs = range(i * b, min(N, (i + 1) * b))
+                ks = range(j * b, min(N, (j + 1) * b))
+                n = sum(1 for q in qs for kv in ks if kv in sets[q])
+                if full[i, c] != int(n == len(qs) * len(ks)):
+                    return False
+    # Q = 0 gives ln |A(q)|
+    N, D, w, s = 200, 8, 20, 4
+    q = np.zeros((1, 1, N, D), dtype=np.uint16)
+    _, k, v = synth.qkv(1, 1, 1, N, D, seed=9)
+    _, LSE = o.attention(q, k, v, Pattern(window=w, sinks=s), 0.5)
+    cnt = np.array([min(r, w) + 1 + min(s, max(0, r - w)) for r in range(N)])
+    if np.abs(LSE[0, 0] - np.log(cnt)).max() > 1e-12:
+        return False
+    # dense causal with GQA equals the library routine
+    B, Hq, Hkv, N, D = 1, 4, 2, 64, 16
+    q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=11)
+    O, _ = o.attention(q, k, v, Pattern(window=N), 1 / math.sqrt(D))
+    f = lambda a: torch.from_numpy(synth.bf16_bits_to_float(a)).double()
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        f(q), f(k).repeat_interleave(2, 1), f(v).repeat_interleave(2, 1), is_causal=True, scale=1 / math.sqrt(D))
+    if np.abs(O - ref.numpy()).max() > 1e-12:
+        return False
+    return True
+
+
+def test_unmutated_oracle_passes():
+    assert pins_hold(oracle.default())
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = oracle.source()
+    assert src.count(old) == 1, f"mutation site for {name} not found"
+    path = oracle.compile_source(src.replace(old, new), str(tmp_path / f"lib_{name}.so"))
+    assert not pins_hold(oracle.Oracle(path))
