@@ -1,0 +1,159 @@
+// Pattern compiler: classify every (q-tile, kv-tile) of the causal score
+// matrix as empty, partial or full from interval arithmetic on the pattern,
+// and count allowed pairs in closed form per query row.
+//
+// "Sparse Attention" glossary page, section "Ein Muster in Einsparungen
+// verwandeln": a mask is split into 128 x 128 blocks so that kernels can skip
+// the blocks without an allowed pair.  Here the classification is analytic:
+// over a rectangle of queries [q0, q1] x keys [k0, k1] the distance q - kv
+// takes every integer in [q0 - k1, q1 - k0], so each rule of the pattern
+// (band, sink/global columns, global rows, stride) decides emptiness and
+// fullness with a few comparisons instead of a loop over the pairs.
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/sparse_attn.h"
+
+namespace sa {
+
+namespace {
+
+int64_t floor_div(int64_t a, int64_t b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
+
+// Is there a multiple of s in [a, b]?
+bool has_multiple(int64_t a, int64_t b, int64_t s) { return a <= b && floor_div(b, s) * s >= a; }
+
+struct Rect {
+    int64_t q0, q1, k0, k1;  // inclusive
+};
+
+// At least one allowed pair in the rectangle.
+bool any_allowed(const sa_pattern& p, const Rect& r)
+{
+    if (r.q1 < r.k0) return false;                          // entirely above the diagonal
+    const int64_t dmin = std::max<int64_t>(0, r.q0 - r.k1);  // causal distances present: [dmin, q1 - k0]
+    const int64_t dmax = r.q1 - r.k0;
+    if (p.window >= 0 && dmin <= p.window) return true;      // band
+    const int64_t cols = std::max(p.sinks, p.n_global);
+    if (r.k0 < cols) return true;                            // sink / global column at kv = k0, q = q1
+    if (p.n_global > 0 && r.q0 < p.n_global && r.k0 <= std::min<int64_t>(r.q1, p.n_global - 1))
+        return true;                                         // global row
+    if (p.stride > 0 && has_multiple(dmin, dmax, p.stride)) return true;
+    return false;
+}
+
+// Every pair of the rectangle allowed.
+bool all_allowed(const sa_pattern& p, const Rect& r)
+{
+    if (r.q0 < r.k1) return false;  // some pair above the diagonal
+    // Pairs outside the sink/global columns and the global rows:
+    const int64_t cols = std::max(p.sinks, p.n_global);
+    const int64_t qa = std::max<int64_t>(r.q0, p.n_global), ka = std::max<int64_t>(r.k0, cols);
+    if (qa > r.q1 || ka > r.k1) return true;
+    int64_t lo = qa - r.k1;
+    const int64_t hi = r.q1 - ka;
+    if (p.window >= 0) lo = std::max<int64_t>(lo, int64_t(p.window) + 1);  // band covers distances <= window
+    if (lo > hi) return true;
+    // distances [lo, hi] remain; each must be a multiple of the stride
+    if (p.stride <= 0) return false;
+    if (p.stride == 1) return true;
+    return lo == hi && lo % p.stride == 0;
+}
+
+bool pattern_ok(const sa_pattern* p)
+{
+    return p && p->causal == 1 && p->window >= -1 && p->sinks >= 0 && p->stride >= 0 && p->n_global >= 0;
+}
+
+}  // namespace
+
+// Allowed keys of query q (0 <= q < N): |band U columns U stride-hits|, or
+// all of [0, q] for a global row.
+int64_t row_pairs(const sa_pattern& p, int64_t q)
+{
+    if (q < p.n_global) return q + 1;
+    const int64_t cols = std::min<int64_t>(std::max(p.sinks, p.n_global), q + 1);  // kv in [0, cols)
+    int64_t n = cols;
+    int64_t lo;  // smallest distance the band does not cover
+    if (p.window >= 0) {
+        const int64_t wq = std::min<int64_t>(q, p.window);  // band kv in [q - wq, q]
+        const int64_t band_lo = q - wq;
+        n += (wq + 1) - std::max<int64_t>(0, cols - band_lo);  // band minus its overlap with the columns
+        lo = wq + 1;
+    } else {
+        lo = 0;
+    }
+    if (p.stride > 0) {
+        const int64_t hi = q - cols;  // distances whose key lies right of the columns
+        if (hi >= lo) n += floor_div(hi, p.stride) - floor_div(lo - 1, p.stride);
+    }
+    return n;
+}
+
+}  // namespace sa
+
+extern "C" int32_t sparse_attn_num_tiles(int64_t N, int32_t block)
+{
+    if (N < 0 || block <= 0) return SA_ERR_INVALID_ARG;
+    const int64_t T = (N + block - 1) / block;
+    if (T > INT32_MAX) return SA_ERR_UNSUPPORTED;
+    return static_cast<int32_t>(T);
+}
+
+extern "C" int sparse_attn_build_block_mask(const sa_pattern* pattern, int64_t N, int32_t block, sa_block_mask* out)
+{
+    if (!out || N < 0) return SA_ERR_INVALID_ARG;
+    if (!pattern) return SA_ERR_INVALID_ARG;
+    if (!sa::pattern_ok(pattern)) return pattern->causal != 1 ? SA_ERR_UNSUPPORTED : SA_ERR_INVALID_ARG;
+    if (block != 64 && block != 128) return SA_ERR_UNSUPPORTED;
+    const int64_t T64 = (N + block - 1) / block;
+    if (T64 > (1 << 20)) return SA_ERR_UNSUPPORTED;
+    const int32_t T = static_cast<int32_t>(T64);
+    if (out->n_q_tiles < T || out->n_kv_tiles < T) return SA_ERR_BUFFER_TOO_SMALL;
+    if (T > 0 && (!out->kv_count || !out->kv_index || !out->kv_full)) return SA_ERR_INVALID_ARG;
+
+    int32_t max_row = 0;
+    int64_t live = 0, nfull = 0;
+    for (int32_t i = 0; i < T; i++) {
+        sa::Rect r;
+        r.q0 = int64_t(i) * block;
+        r.q1 = std::min<int64_t>(N, r.q0 + block) - 1;
+        int32_t* idx = out->kv_index + int64_t(i) * T;
+        uint8_t* full = out->kv_full + int64_t(i) * T;
+        int32_t c = 0;
+        for (int32_t j = 0; j <= i; j++) {  // tiles right of the diagonal hold no causal pair
+            r.k0 = int64_t(j) * block;
+            r.k1 = std::min<int64_t>(N, r.k0 + block) - 1;
+            if (!sa::any_allowed(*pattern, r)) continue;
+            idx[c] = j;
+            full[c] = sa::all_allowed(*pattern, r) ? 1 : 0;
+            nfull += full[c];
+            c++;
+        }
+        for (int32_t t = c; t < T; t++) {
+            idx[t] = -1;
+            full[t] = 0;
+        }
+        out->kv_count[i] = c;
+        live += c;
+        max_row = std::max(max_row, c);
+    }
+    out->n_q_tiles = T;
+    out->n_kv_tiles = T;
+    out->block = block;
+    out->max_per_row = max_row;
+    out->n_live = live;
+    out->n_full = nfull;
+    return SA_OK;
+}
+
+extern "C" int sparse_attn_count_pairs(const sa_pattern* pattern, int64_t N, int64_t* pairs)
+{
+    if (!pattern || !pairs || N < 0) return SA_ERR_INVALID_ARG;
+    if (!sa::pattern_ok(pattern)) return pattern->causal != 1 ? SA_ERR_UNSUPPORTED : SA_ERR_INVALID_ARG;
+    int64_t total = 0;
+    for (int64_t q = 0; q < N; q++) total += sa::row_pairs(*pattern, q);
+    *pairs = total;
+    return SA_OK;
+}

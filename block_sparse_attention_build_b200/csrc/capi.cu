@@ -1,0 +1,218 @@
+// C ABI of the forward pass: argument checks, TMA descriptors, kernel choice
+// and launch, the host-buffer variant, and the device status word.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/sparse_attn.h"
+#include "fwd_sm100.cuh"
+#include "tma_host.h"
+
+namespace sa {
+namespace {
+
+constexpr long long kDefaultTimeout = 2000000000LL;  // SM cycles, about one second
+constexpr int kMaxDevices = 64;
+
+std::mutex g_mu;
+int32_t* g_status[kMaxDevices] = {};  // one status word per device, allocated on first use
+int32_t g_debug_flags = 0;
+long long g_timeout = kDefaultTimeout;
+
+// The device status word of the current device, allocated once.
+int status_word(int32_t** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status[dev]) {
+        int32_t* p = nullptr;
+        if (cudaMalloc(&p, sizeof(int32_t)) != cudaSuccess) return SA_ERR_CUDA;
+        if (cudaMemset(p, 0, sizeof(int32_t)) != cudaSuccess) return SA_ERR_CUDA;
+        g_status[dev] = p;
+    }
+    *out = g_status[dev];
+    return SA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int D, int BN>
+int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p, int grid,
+           cudaStream_t stream)
+{
+    using C = FwdCfg<D, BN>;
+    auto kern = fwd_kernel<D, BN>;
+    static bool attr_set[kMaxDevices] = {};  // per instantiation and device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SA_ERR_CUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+            return SA_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace sa
+
+extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, const sa_block_mask* mask,
+                               const sa_pattern* pattern, const sa_shape* shape, float scale, void* O, float* LSE,
+                               void* stream)
+{
+    using namespace sa;
+    if (!mask || !pattern || !shape) return SA_ERR_INVALID_ARG;
+    const sa_shape s = *shape;
+    if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
+    if (pattern->causal != 1) return SA_ERR_UNSUPPORTED;
+    if (pattern->window < -1 || pattern->sinks < 0 || pattern->stride < 0 || pattern->n_global < 0)
+        return SA_ERR_INVALID_ARG;
+    if (s.D != 64 && s.D != 128) return SA_ERR_UNSUPPORTED;
+    if (mask->block != 64 && mask->block != 128) return SA_ERR_UNSUPPORTED;
+    if (s.B == 0 || s.Hq == 0 || s.N == 0) return SA_OK;  // nothing to compute
+    if (s.Hkv <= 0 || s.Hq % s.Hkv != 0) return SA_ERR_UNSUPPORTED;
+    const int64_t T = (int64_t(s.N) + mask->block - 1) / mask->block;
+    if (mask->n_q_tiles != T || mask->n_kv_tiles != T) return SA_ERR_MASK_MISMATCH;
+    if (!Q || !K || !V || !O || !LSE || !mask->kv_count || !mask->kv_index || !mask->kv_full)
+        return SA_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+        return SA_ERR_MISALIGNED;
+    const int64_t n_qtiles = (int64_t(s.N) + kBM - 1) / kBM;
+    const int64_t grid = n_qtiles * s.B * s.Hq;
+    if (grid > INT32_MAX || int64_t(s.B) * s.Hq > INT32_MAX) return SA_ERR_UNSUPPORTED;
+
+    int32_t* status = nullptr;
+    if (int rc = status_word(&status)) return rc;
+
+    CUtensorMap mq, mk, mv;
+    const uint32_t bn = static_cast<uint32_t>(mask->block);
+    if (!make_map_bf16_3d(&mq, Q, s.D, s.N, uint64_t(s.B) * s.Hq, kBM) ||
+        !make_map_bf16_3d(&mk, K, s.D, s.N, uint64_t(s.B) * s.Hkv, bn) ||
+        !make_map_bf16_3d(&mv, V, s.D, s.N, uint64_t(s.B) * s.Hkv, bn))
+        return SA_ERR_CUDA;
+
+    FwdParams p;
+    p.kv_count = mask->kv_count;
+    p.kv_index = mask->kv_index;
+    p.kv_full = mask->kv_full;
+    p.T = static_cast<int32_t>(T);
+    p.N = s.N;
+    p.B = s.B;
+    p.Hq = s.Hq;
+    p.Hkv = s.Hkv;
+    p.group = s.Hq / s.Hkv;
+    p.n_qtiles = static_cast<int32_t>(n_qtiles);
+    p.window = pattern->window;
+    p.sinks = pattern->sinks;
+    p.stride = pattern->stride;
+    p.n_global = pattern->n_global;
+    p.scale_log2 = scale * 1.44269504088896340736f;
+    p.O = static_cast<__nv_bfloat16*>(O);
+    p.LSE = LSE;
+    p.status = status;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        p.timeout = g_timeout;
+        p.debug_flags = g_debug_flags;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int g = static_cast<int>(grid);
+    if (s.D == 128 && mask->block == 128) return launch<128, 128>(mq, mk, mv, p, g, st);
+    if (s.D == 64 && mask->block == 128) return launch<64, 128>(mq, mk, mv, p, g, st);
+    if (s.D == 128 && mask->block == 64) return launch<128, 64>(mq, mk, mv, p, g, st);
+    return launch<64, 64>(mq, mk, mv, p, g, st);
+}
+
+extern "C" int sparse_attn_fwd_host_workspace(const sa_shape* shape, size_t* bytes)
+{
+    if (!shape || !bytes) return SA_ERR_INVALID_ARG;
+    const sa_shape s = *shape;
+    if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t q = size_t(s.B) * s.Hq * s.N * s.D * 2;
+    const size_t kv = size_t(s.B) * s.Hkv * s.N * s.D * 2;
+    const size_t lse = size_t(s.B) * s.Hq * s.N * 4;
+    *bytes = up(q) + 2 * up(kv) + up(q) + up(lse);
+    return SA_OK;
+}
+
+extern "C" int sparse_attn_fwd_host(const void* Q_host, const void* K_host, const void* V_host,
+                                    const sa_block_mask* mask, const sa_pattern* pattern, const sa_shape* shape,
+                                    float scale, void* O_host, float* LSE_host, void* workspace,
+                                    size_t workspace_bytes, void* stream)
+{
+    if (!shape || !mask || !pattern) return SA_ERR_INVALID_ARG;
+    size_t need = 0;
+    if (int rc = sparse_attn_fwd_host_workspace(shape, &need)) return rc;
+    const sa_shape s = *shape;
+    if (s.B == 0 || s.Hq == 0 || s.N == 0) return SA_OK;
+    if (!Q_host || !K_host || !V_host || !O_host || !LSE_host || !workspace) return SA_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return SA_ERR_BUFFER_TOO_SMALL;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SA_ERR_MISALIGNED;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t qb = size_t(s.B) * s.Hq * s.N * s.D * 2;
+    const size_t kvb = size_t(s.B) * s.Hkv * s.N * s.D * 2;
+    const size_t lseb = size_t(s.B) * s.Hq * s.N * 4;
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    void* dQ = w;
+    void* dK = w + up(qb);
+    void* dV = w + up(qb) + up(kvb);
+    void* dO = w + up(qb) + 2 * up(kvb);
+    float* dL = reinterpret_cast<float*>(w + 2 * up(qb) + 2 * up(kvb));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(dQ, Q_host, qb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dK, K_host, kvb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dV, V_host, kvb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return SA_ERR_CUDA;
+    if (int rc = sparse_attn_fwd(dQ, dK, dV, mask, pattern, shape, scale, dO, dL, stream)) return rc;
+    if (cudaMemcpyAsync(O_host, dO, qb, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(LSE_host, dL, lseb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return SA_ERR_CUDA;
+    return sparse_attn_check_device(stream);
+}
+
+extern "C" int sparse_attn_check_device(void* stream)
+{
+    int32_t* status = nullptr;
+    if (int rc = sa::status_word(&status)) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t word = 0;
+    if (cudaMemcpyAsync(&word, status, sizeof word, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_CUDA;
+    if (word != 0) {
+        if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return SA_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_CUDA;
+        return SA_ERR_DEVICE_TIMEOUT;
+    }
+    return SA_OK;
+}
+
+extern "C" int sparse_attn_set_debug(int32_t flags, int64_t timeout_cycles)
+{
+    std::lock_guard<std::mutex> lk(sa::g_mu);
+    sa::g_debug_flags = flags;
+    sa::g_timeout = timeout_cycles > 0 ? timeout_cycles : sa::kDefaultTimeout;
+    return SA_OK;
+}
+
+extern "C" const char* sparse_attn_status_string(int status)
+{
+    switch (status) {
+    case SA_OK: return "ok";
+    case SA_ERR_INVALID_ARG: return "invalid argument";
+    case SA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case SA_ERR_BUFFER_TOO_SMALL: return "buffer too small";
+    case SA_ERR_CUDA: return "CUDA error";
+    case SA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case SA_ERR_MASK_MISMATCH: return "block mask does not match N and block";
+    default: return "unknown status";
+    }
+}
+
+extern "C" int32_t sparse_attn_version(void) { return 100; }

@@ -1,0 +1,167 @@
+/*
+ * sparse_attn — block-sparse causal attention forward for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Plain pointers and sizes only; no C++ or framework types cross it.
+ * Every call returns an int status (SA_OK or a negative SA_ERR_* code); no
+ * exception or abort crosses the boundary.  The caller owns every buffer.
+ *
+ * The computation.  Scaled dot-product attention in which query q may attend
+ * only to keys kv allowed by a fixed pattern, with the softmax taken over the
+ * allowed keys alone.  The pattern and the masked-softmax definition follow:
+ *   - "Sparse Attention" glossary page (ultralytics.com/de/glossary/sparse-attention),
+ *     section "Gängige Sparsity-Muster": sliding window, every s-th prior token,
+ *     global tokens, attention sinks;
+ *   - the same page, section "Ein Muster in Einsparungen verwandeln": the
+ *     local_plus_sinks predicate (causal, q - kv <= window, or kv < sinks), its
+ *     compilation into 128 x 128 blocks, and kernels that skip the empty ones;
+ *   - "Sparse-трансформеры: как урезать O(n²) внимания" (1gpt.online), section
+ *     "Как это выглядит в коде": scores q.k / sqrt(d), -inf outside the mask,
+ *     softmax, times V.
+ *
+ * Tensor layouts (all contiguous, row-major):
+ *   Q, O  [B, Hq,  N, D] bf16        K, V  [B, Hkv, N, D] bf16
+ *   LSE   [B, Hq,  N]    fp32        natural log of the softmax denominator,
+ *                                    sum over allowed kv of exp(scale * q.k)
+ * Query head hq reads key/value head hq / (Hq / Hkv).
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------- */
+#define SA_OK 0
+#define SA_ERR_INVALID_ARG (-1)      /* null pointer, negative size, bad scale */
+#define SA_ERR_UNSUPPORTED (-2)      /* D not in {64, 128}, block not in {64, 128}, causal != 1, Hq % Hkv != 0 */
+#define SA_ERR_MISALIGNED (-3)       /* a tensor pointer is not 16-byte aligned */
+#define SA_ERR_BUFFER_TOO_SMALL (-4) /* output arrays smaller than the tile count */
+#define SA_ERR_CUDA (-5)             /* a CUDA runtime call or kernel launch failed */
+#define SA_ERR_DEVICE_TIMEOUT (-6)   /* a bounded wait inside the kernel expired */
+#define SA_ERR_MASK_MISMATCH (-7)    /* block mask built for another N or block */
+
+/*
+ * A fixed sparsity pattern.  A pair (q, kv) is allowed when
+ *     q >= kv  and  ( (window >= 0 and q - kv <= window)
+ *                     or kv < sinks
+ *                     or (stride > 0 and (q - kv) mod stride == 0)
+ *                     or kv < n_global or q < n_global ).
+ * Pages: "Sparse Attention", sections "Gängige Sparsity-Muster" and "Ein
+ * Muster in Einsparungen verwandeln" (window inclusive, as in local_plus_sinks).
+ * The stride counts back from the query (every s-th prior token); the global
+ * rows and columns stay causal.  causal must be 1.
+ */
+typedef struct {
+    int32_t causal;
+    int32_t window;
+    int32_t sinks;
+    int32_t stride;
+    int32_t n_global;
+} sa_pattern;
+
+/*
+ * The compiled pattern: for every query tile i (block rows) the ascending list
+ * of kv tiles that hold at least one allowed pair, and for each a flag that is
+ * 1 when every in-range pair of the tile is allowed (the kernel then skips the
+ * per-element mask).  Arrays are row-major with row stride n_kv_tiles:
+ *   kv_count[i]                number of listed tiles of row i
+ *   kv_index[i*n_kv_tiles + c] c-th listed kv tile, ascending; -1 after the last
+ *   kv_full [i*n_kv_tiles + c] 1 full, 0 partial; 0 after the last
+ * The last tile of each side is ragged when block does not divide N; only its
+ * in-range pairs count.  Pages: "Sparse Attention", section "Ein Muster in
+ * Einsparungen verwandeln" (create_block_mask and its 128 x 128 blocks).
+ */
+typedef struct {
+    int32_t n_q_tiles;   /* builder: in = capacity of rows, out = T */
+    int32_t n_kv_tiles;  /* builder: in = capacity of a row, out = T (the row stride) */
+    int32_t block;       /* out: tile edge */
+    int32_t max_per_row; /* out: largest kv_count */
+    int64_t n_live;      /* out: sum of kv_count */
+    int64_t n_full;      /* out: number of full tiles */
+    int32_t* kv_count;
+    int32_t* kv_index;
+    uint8_t* kv_full;
+} sa_block_mask;
+
+typedef struct {
+    int32_t B, Hq, Hkv, N, D;
+} sa_shape;
+
+/* T = ceil(N / block), the number of tiles per side; negative status on a bad argument. */
+int32_t sparse_attn_num_tiles(int64_t N, int32_t block);
+
+/*
+ * Classify every (q-tile, kv-tile) pair of an N x N causal score matrix as
+ * empty, partial or full, analytically from the pattern (no per-pair loop),
+ * and write the lists described at sa_block_mask.  Host-only; `out` holds
+ * caller-owned host arrays with capacity out->n_q_tiles rows of
+ * out->n_kv_tiles entries, both at least T (else SA_ERR_BUFFER_TOO_SMALL).
+ * block is 64 or 128; N >= 0 (N = 0 gives T = 0).
+ */
+int sparse_attn_build_block_mask(const sa_pattern* pattern, int64_t N, int32_t block, sa_block_mask* out);
+
+/*
+ * Number of allowed (q, kv) pairs of one head, 0 <= q, kv < N, in closed form
+ * per query row.  4 * D * pairs is the useful work of one (batch, head).
+ */
+int sparse_attn_count_pairs(const sa_pattern* pattern, int64_t N, int64_t* pairs);
+
+/*
+ * Forward pass on the GPU.  Q, K, V, O, LSE are device pointers (16-byte
+ * aligned) in the layouts above; `mask` holds DEVICE copies of the arrays
+ * built by sparse_attn_build_block_mask for this pattern, N and block (its
+ * scalar fields as the builder returned them).  scale > 0 multiplies q.k
+ * (1/sqrt(D) in the pages' prototype).  `stream` is a cudaStream_t (NULL: the
+ * legacy default stream).  Asynchronous: returns once the kernel is queued;
+ * launch errors come back as SA_ERR_CUDA, a device-side timeout through
+ * sparse_attn_check_device.  Rows with no allowed key get O = 0, LSE = -inf.
+ * Supported: D in {64, 128}, mask block in {64, 128}, Hq % Hkv == 0, causal.
+ */
+int sparse_attn_fwd(const void* Q, const void* K, const void* V, const sa_block_mask* mask,
+                    const sa_pattern* pattern, const sa_shape* shape, float scale, void* O, float* LSE,
+                    void* stream);
+
+/*
+ * The same forward pass from HOST buffers: copies Q, K, V from host memory
+ * into `workspace` (device memory, at least sparse_attn_fwd_host_workspace
+ * bytes, 256-byte aligned), runs sparse_attn_fwd on `stream`, copies O and LSE
+ * back to host memory and waits for the stream.  Pinned host memory makes the
+ * copies asynchronous DMA.  `mask` is the device-resident block mask.
+ * Returns the first error, including a device timeout.
+ */
+int sparse_attn_fwd_host(const void* Q_host, const void* K_host, const void* V_host, const sa_block_mask* mask,
+                         const sa_pattern* pattern, const sa_shape* shape, float scale, void* O_host,
+                         float* LSE_host, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Device bytes sparse_attn_fwd_host needs for `shape`. */
+int sparse_attn_fwd_host_workspace(const sa_shape* shape, size_t* bytes);
+
+/*
+ * Wait for `stream`, then read and clear this device's kernel status word:
+ * SA_ERR_DEVICE_TIMEOUT if a bounded wait inside a forward kernel gave up
+ * since the last check, else SA_OK (or SA_ERR_CUDA if the wait failed).
+ */
+int sparse_attn_check_device(void* stream);
+
+/*
+ * Test hook.  flags: bit 0 makes the next forward launches skip the Q tile
+ * load, so the kernel's bounded waits expire and it reports
+ * SA_ERR_DEVICE_TIMEOUT instead of computing.  timeout_cycles bounds every
+ * wait in SM clock cycles (<= 0 restores the default, about one second).
+ */
+int sparse_attn_set_debug(int32_t flags, int64_t timeout_cycles);
+
+const char* sparse_attn_status_string(int status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int32_t sparse_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */

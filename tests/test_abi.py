@@ -1,0 +1,127 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+symbol the header declares, the pattern compiler agrees bit for bit with the
+oracle's brute-force classifier, the pair counter with the oracle's count,
+and argument errors come back as status codes."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import block_sparse_attention_build_b200 as sa
+import oracle
+from synth.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f)).read()
+            names |= set(re.findall(r"\b(sparse_attn_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert "sparse_attn_fwd" in names and "sparse_attn_build_block_mask" in names
+    for n in names:
+        assert hasattr(sa.lib, n), n
+    assert set(sa.EXPORTED) <= set(names)
+
+
+def test_version_and_status_strings():
+    assert sa.version() >= 100
+    assert sa.status_string(0) == "ok"
+    assert "timed out" in sa.status_string(sa.SA_ERR_DEVICE_TIMEOUT)
+
+
+def opattern(p: sa.Pattern):
+    return oracle.Pattern(window=p.window, sinks=p.sinks, stride=p.stride, n_global=p.n_global)
+
+
+SWEEP = [
+    (sa.Pattern(window=w, sinks=s, stride=st, n_global=g), N, b)
+    for (w, s, st, g) in [(1024, 4, 0, 0), (128, 4, 0, 0), (0, 0, 0, 0), (-1, 3, 0, 0), (63, 1, 0, 0),
+                          (64, 0, 0, 0), (127, 128, 0, 0), (200, 130, 0, 0), (128, 0, 128, 16),
+                          (10, 0, 7, 3), (-1, 0, 64, 0), (-1, 0, 1, 0), (5, 0, 200, 70), (300, 2, 3, 0),
+                          (-1, 0, 0, 0), (100000, 0, 0, 0)]
+    for N in (1, 63, 64, 65, 500, 1000, 1024)
+    for b in (64, 128)
+]
+
+
+@pytest.mark.parametrize("p,N,b", SWEEP)
+def test_block_mask_matches_oracle(p, N, b):
+    m = sa.build_block_mask(p, N, b)
+    c, i, f = oracle.block_mask(opattern(p), N, b)
+    assert np.array_equal(m.counts, c) and np.array_equal(m.index, i) and np.array_equal(m.full, f)
+    assert m.n_live == c.sum() and m.max_per_row == (c.max() if len(c) else 0)
+    assert m.n_full == sum(int(f[r, : c[r]].sum()) for r in range(len(c)))
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_block_mask_workloads_match_oracle(name):
+    w = WORKLOADS[name]
+    p = sa.Pattern(**w.pattern_args())
+    m = sa.build_block_mask(p, w.N, w.block)
+    c, i, f = oracle.block_mask(opattern(p), w.N, w.block)
+    assert np.array_equal(m.counts, c) and np.array_equal(m.index, i) and np.array_equal(m.full, f)
+    assert sa.count_pairs(p, w.N) == oracle.count_pairs(opattern(p), w.N)
+
+
+@pytest.mark.parametrize("p,N", [(p, N) for (p, N, b) in SWEEP if b == 64])
+def test_pair_count_matches_oracle(p, N):
+    assert sa.count_pairs(p, N) == oracle.count_pairs(opattern(p), N)
+
+
+def test_empty_sequence():
+    m = sa.build_block_mask(sa.Pattern(window=4), 0, 128)
+    assert m.T == 0 and m.n_live == 0
+    assert sa.count_pairs(sa.Pattern(window=4), 0) == 0
+
+
+def test_builder_errors():
+    with pytest.raises(sa.SparseAttnError) as e:
+        sa.build_block_mask(sa.Pattern(window=4), 100, 32)
+    assert e.value.status == sa.SA_ERR_UNSUPPORTED
+    with pytest.raises(sa.SparseAttnError) as e:
+        sa.build_block_mask(sa.Pattern(window=4, causal=0), 100, 64)
+    assert e.value.status == sa.SA_ERR_UNSUPPORTED
+    with pytest.raises(sa.SparseAttnError) as e:
+        sa.build_block_mask(sa.Pattern(window=-2), 100, 64)
+    assert e.value.status == sa.SA_ERR_INVALID_ARG
+    # capacity too small
+    m = sa._BlockMask(1, 1, 0, 0, 0, 0, None, None, None)
+    rc = sa.lib.sparse_attn_build_block_mask(ctypes.byref(sa.Pattern(window=4)._c()), 1000, 128, ctypes.byref(m))
+    assert rc == sa.SA_ERR_BUFFER_TOO_SMALL
+
+
+def test_fwd_argument_errors_without_gpu():
+    """Checks that return before any CUDA call."""
+    p = sa.Pattern(window=8)._c()
+    m = sa._BlockMask(1, 1, 128, 1, 1, 0, 16, 16, 16)
+    fake = 1 << 20  # never dereferenced: every case below fails validation first
+
+    def call(shape, scale=0.125, mask=m, pat=p, ptr=fake):
+        return sa.lib.sparse_attn_fwd(ptr, ptr, ptr, ctypes.byref(mask), ctypes.byref(pat),
+                                      ctypes.byref(sa._Shape(*shape)), scale, ptr, ptr, None)
+
+    assert call((1, 2, 2, 100, 96)) == sa.SA_ERR_UNSUPPORTED          # D
+    assert call((1, 2, 2, 100, 128), scale=0.0) == sa.SA_ERR_INVALID_ARG
+    assert call((1, 2, 2, 100, 128), scale=float("nan")) == sa.SA_ERR_INVALID_ARG
+    assert call((1, 3, 2, 100, 128)) == sa.SA_ERR_UNSUPPORTED         # Hq % Hkv
+    assert call((1, 2, 2, 1000, 128)) == sa.SA_ERR_MASK_MISMATCH      # T != ceil(N / block)
+    assert call((-1, 2, 2, 100, 128)) == sa.SA_ERR_INVALID_ARG
+    assert call((1, 2, 2, 100, 128), ptr=fake + 8) == sa.SA_ERR_MISALIGNED
+    assert call((0, 2, 2, 100, 128)) == sa.SA_OK                      # nothing to compute
+    assert call((1, 2, 2, 0, 128)) == sa.SA_OK
+    bad = sa.Pattern(window=8, causal=0)._c()
+    assert call((1, 2, 2, 100, 128), pat=bad) == sa.SA_ERR_UNSUPPORTED
+    ws = ctypes.c_size_t(0)
+    assert sa.lib.sparse_attn_fwd_host_workspace(ctypes.byref(sa._Shape(1, 2, 1, 100, 64)), ctypes.byref(ws)) == 0
+    assert ws.value >= 2 * (2 * 100 * 64 * 2) + 2 * (100 * 64 * 2) + 2 * 100 * 4
