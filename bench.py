@@ -1,0 +1,409 @@
+"""Throughput of the block-sparse causal attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one forward pass (one kernel launch) over the workload's whole
+batch.  Prints one JSON line on rank 0.
+
+value      useful TFLOP/s = 4 * D * (allowed pairs per head) * B * Hq per step,
+           divided by the device time of K steps (CUDA events, barrier and
+           synchronize on both sides, max over ranks); inputs resident in HBM.
+           Inputs rotate over several sets whose footprint exceeds L2.
+roofline   the forward kernel against the measured dense bf16 tensor peak:
+           executed-tile FLOP per launch (4 * D * block^2 per live tile) over
+           the mean per-launch duration (CUDA events on the launching stream).
+e2e        the same metric through the host-buffer C ABI call (pinned host
+           Q/K/V in, O/LSE out, copies inside the timed region).
+cpu_baseline  the fp64 CPU oracle on a bounded row sample, host cores.
+
+With --impl reference the oracle is the timed program (rank 0 only).
+Multi-GPU (torchrun): every rank runs its own batch of the workload (the
+problems are independent; no collective on the data path); value is the sum
+over ranks of the work divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from synth.workloads import HEADLINE, WORKLOADS  # noqa: E402
+
+METRIC = "block-sparse attn fwd useful TFLOP/s (bf16, 1 B200) and % of tensor peak"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+KERNEL_SOURCES = ["block_sparse_attention_build_b200/csrc/fwd_sm100.cuh",
+                  "block_sparse_attention_build_b200/csrc/sm100.cuh"]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"fwd_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, _, v = line.strip()[2:].partition(":")
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha") != kernel_sha():
+        return None
+    try:
+        return int(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def workload_counts(w):
+    import block_sparse_attention_build_b200 as sa
+    p = sa.Pattern(**w.pattern_args())
+    pairs = sa.count_pairs(p, w.N)
+    mask = sa.build_block_mask(p, w.N, w.block)
+    useful = 4.0 * w.D * pairs * w.B * w.Hq
+    executed = 4.0 * w.D * w.block * w.block * mask.n_live * w.B * w.Hq
+    qo = w.B * w.Hq * w.N * w.D * 2
+    kv = w.B * w.Hkv * w.N * w.D * 2
+    min_bytes = 2 * qo + 2 * kv + w.B * w.Hq * w.N * 4
+    return p, mask, pairs, useful, executed, min_bytes
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _sample_rows(w, n):
+    return np.unique(np.linspace(0, w.N - 1, n).round().astype(np.int64))
+
+
+def _sample_flops(w, rows):
+    """Useful FLOP of the sampled rows: 4 * D * (allowed keys of each row) * B * Hq."""
+    import block_sparse_attention_build_b200 as sa
+    p = sa.Pattern(**w.pattern_args())
+    keys = sum(sa.count_pairs(p, int(r) + 1) - sa.count_pairs(p, int(r)) for r in rows)
+    return 4.0 * w.D * keys * w.B * w.Hq
+
+
+class OracleSample:
+    """The fp64 CPU oracle on an evenly spaced row sample of the workload (all
+    batches and heads), sized once to about target_s seconds per call."""
+
+    def __init__(self, w, target_s: float):
+        import oracle
+        self.oracle = oracle
+        self.w = w
+        self.q, self.k, self.v = synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=w.seed)
+        self.op = oracle.Pattern(**w.pattern_args())
+        n = 8
+        while True:
+            rows = _sample_rows(w, n)
+            dt = self._time(rows)
+            if dt >= target_s or n >= w.N:
+                break
+            n = min(w.N, max(n * 2, int(n * target_s / max(dt, 1e-4) * 1.05)))
+        self.rows = rows
+        self.flops = _sample_flops(w, rows)
+        self.threads = oracle.max_threads()
+
+    def _time(self, rows):
+        t0 = time.perf_counter()
+        self.oracle.attention(self.q, self.k, self.v, self.op, self.w.scale, rows=rows)
+        return time.perf_counter() - t0
+
+    def run(self):
+        """One timed call: (useful TFLOP/s, seconds)."""
+        dt = self._time(self.rows)
+        return self.flops / dt / 1e12, dt
+
+    def describe(self, dt):
+        return (f"{len(self.rows)} evenly spaced query rows of {self.w.N} x all {self.w.B * self.w.Hq} "
+                f"(batch, head) pairs, fp64, {dt:.2f} s per call")
+
+
+def run_reference(args, w):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    per_step = min(2.0, max(0.01, 120.0 / (args.steps + args.warmup)))
+    sample = OracleSample(w, per_step)
+    for _ in range(args.warmup):
+        sample.run()
+    secs = [sample.run()[1] for _ in range(args.steps)]
+    total = float(np.sum(secs))
+    value = sample.flops * args.steps / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": sample.threads, "kind": "oracle",
+                         "sample": sample.describe(total / args.steps)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def config_of(w, n_gpus, extra=None):
+    c = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "D": w.D,
+         "pattern": {"causal": 1, **w.pattern_args()}, "block": w.block, "seed": w.seed,
+         "inputs": "iid N(0,1) -> bf16, scale 1/sqrt(D)",
+         "parallelism": "single GPU" if n_gpus == 1 else f"{n_gpus} independent batches, one per GPU"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_build_b200 as sa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    p, mask_h, pairs, useful, executed, min_bytes = workload_counts(w)
+    mask = mask_h.to_device(dev)
+
+    # inputs: every rank its own batch (seed offset by rank); rotate sets past L2
+    q, k, v = synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=w.seed + rank)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    set_bytes = min_bytes
+    n_sets = args.sets if args.sets > 0 else max(1, min(8, math.ceil(3 * L2_BYTES / set_bytes)))
+    Q0, K0, V0 = to_dev(q), to_dev(k), to_dev(v)
+    sets = []
+    for i in range(n_sets):
+        Qi, Ki, Vi = (Q0, K0, V0) if i == 0 else (Q0.clone(), K0.clone(), V0.clone())
+        Oi = torch.empty_like(Qi)
+        Li = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+        sets.append((Qi, Ki, Vi, Oi, Li))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        Qi, Ki, Vi, Oi, Li = sets[i % n_sets]
+        sa.fwd(Qi, Ki, Vi, mask, p, scale=w.scale, out=Oi, lse=Li, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if sa.check_device(stream) != sa.SA_OK:
+        raise SystemExit("device status not ok after warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step(i)
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    status = sa.check_device(stream)
+    if status != sa.SA_OK:
+        raise SystemExit(f"device status {sa.status_string(status)}")
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    mean_launch_ms = float(np.mean(launch_ms))
+    median_launch_ms = float(np.median(launch_ms))
+
+    # end to end through the host-buffer entry point (pinned memory)
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+        Qh, Kh, Vh = pin(q), pin(k), pin(v)
+        Oh = torch.empty((w.B, w.Hq, w.N, w.D), dtype=torch.bfloat16).pin_memory()
+        Lh = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32).pin_memory()
+        ws = torch.empty(sa.fwd_host_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.D), dtype=torch.uint8,
+                         device=dev)
+        e2e_steps = max(3, min(args.steps, 20))
+        for _ in range(2):
+            sa.fwd_host(Qh, Kh, Vh, mask, p, Oh, Lh, ws, scale=w.scale, stream=stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            sa.fwd_host(Qh, Kh, Vh, mask, p, Oh, Lh, ws, scale=w.scale, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh))
+        d2h = Oh.numel() * Oh.element_size() + Lh.numel() * Lh.element_size()
+        e2e = {"value": world * useful * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "ms_per_step": e2e_ms / e2e_steps}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    value = world * useful * args.steps / (elapsed_ms * 1e-3) / 1e12
+    achieved = executed / (mean_launch_ms * 1e-3) / 1e12
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        sample = OracleSample(w, args.cpu_seconds)
+        rate, dt = sample.run()
+        cpu = {"value": rate, "unit": UNIT, "cores": sample.threads, "kind": "oracle",
+               "sample": sample.describe(dt)}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(w, world, {
+            "l2": f"{n_sets} rotating input sets of {set_bytes / 1e6:.1f} MB "
+                  f"({n_sets * set_bytes / 1e6:.0f} MB > {L2_BYTES / 1e6:.0f} MB L2)",
+            "live_tiles": int(mask_h.n_live), "full_tiles": int(mask_h.n_full),
+            "allowed_pairs_per_head": int(pairs)}),
+        "useful_frac_of_peak": value / world / peak,
+        "executed_tflops": world * executed * args.steps / (elapsed_ms * 1e-3) / 1e12,
+        "executed_frac_of_peak": executed / (elapsed_ms / args.steps * 1e-3) / 1e12 / peak,
+        "peak_kind": f"bf16 dense, {peak_kind} ({peak} TFLOP/s burst)",
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(w.name),
+                     "kernel": "fwd_kernel<D,BN>", "mean_launch_us": mean_launch_ms * 1e3,
+                     "median_launch_us": median_launch_ms * 1e3,
+                     "algorithmic_flop_per_launch": executed,
+                     "hbm_gbs_min_bytes": min_bytes / (mean_launch_ms * 1e-3) / 1e9},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling runs)")
+    ap.add_argument("--sets", type=int, default=0, help="rotating input sets (0: enough to exceed L2)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

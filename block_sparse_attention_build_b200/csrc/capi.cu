@@ -39,6 +39,20 @@ int status_word(int32_t** out)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Number of SMs of the current device (cached).
+int sm_count()
+{
+    static int counts[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    if (!counts[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
 template <int D, int BN>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p, int grid,
            cudaStream_t stream)
@@ -83,8 +97,14 @@ extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, cons
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
         return SA_ERR_MISALIGNED;
     const int64_t n_qtiles = (int64_t(s.N) + kBM - 1) / kBM;
-    const int64_t grid = n_qtiles * s.B * s.Hq;
-    if (grid > INT32_MAX || int64_t(s.B) * s.Hq > INT32_MAX) return SA_ERR_UNSUPPORTED;
+    const int64_t group = s.Hq / s.Hkv;
+    // work units: two 128-row query tiles that share a key/value head
+    const int64_t pairs = group >= 2 ? (group + 1) / 2 : (n_qtiles + 1) / 2;
+    const int64_t n_units = group >= 2 ? n_qtiles * s.B * s.Hkv * pairs : pairs * s.B * s.Hq;
+    if (n_units > INT32_MAX || int64_t(s.B) * s.Hq > INT32_MAX) return SA_ERR_UNSUPPORTED;
+    const int n_sm = sm_count();
+    if (n_sm <= 0) return SA_ERR_CUDA;
+    const int64_t grid = n_units < n_sm ? n_units : n_sm;
 
     int32_t* status = nullptr;
     if (int rc = status_word(&status)) return rc;
@@ -107,6 +127,8 @@ extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, cons
     p.Hkv = s.Hkv;
     p.group = s.Hq / s.Hkv;
     p.n_qtiles = static_cast<int32_t>(n_qtiles);
+    p.n_units = static_cast<int32_t>(n_units);
+    p.pairs = static_cast<int32_t>(pairs);
     p.window = pattern->window;
     p.sinks = pattern->sinks;
     p.stride = pattern->stride;

@@ -1,31 +1,44 @@
 // Block-sparse causal attention forward for sm_100a.
 //
-// One CTA computes one 128-row query tile of one (batch, query head).  It
-// walks the tile's list of live kv tiles (the compiled pattern) and never
-// touches an empty tile ("Sparse Attention" glossary page, section "Ein Muster
-// in Einsparungen verwandeln": speed comes from kernels that skip empty tiles).
-// Per kv tile the work is the tiled exact attention of Flash-attention (the
-// same page, related terms): S = Q K^T on the tensor cores, an online softmax,
-// O += P V on the tensor cores.
+// Persistent kernel: one CTA per SM walks a strided share of the work units.
+// A work unit is two 128-row query tiles ("slots" A and B) that read the same
+// key/value head: two query heads of one group at the same query tile when
+// heads are grouped, else two consecutive query tiles of one head.  The unit
+// walks the union of the slots' lists of live kv tiles (the compiled pattern)
+// and never touches a tile outside it ("Sparse Attention" glossary page,
+// section "Ein Muster in Einsparungen verwandeln": speed comes from kernels
+// that skip empty tiles).  Per kv tile the work is the tiled exact attention
+// of Flash-attention (same page, related terms): S = Q K^T on the tensor
+// cores, an online softmax, O += P V on the tensor cores.
 //
-// Warp roles (192 threads):
-//   warp 0     TMA producer: Q once, then K and V tiles of each listed kv tile
-//              into two rings of shared-memory stages
+// Warp roles (384 threads, three warpgroups):
+//   warp 0     TMA producer: Q of both slots per unit, then K and V of each
+//              kv tile of the union into two rings of shared-memory stages
 //   warp 1     allocates tensor memory; one lane issues every tcgen05.mma
-//   warps 2-5  softmax: thread t owns query row t (its tensor-memory lane),
-//              masks partial tiles, keeps the running max and sum, writes P
-//              (bf16) into tensor memory, rescales O when the max moves far,
-//              and stores O and LSE at the end
+//   warps 2-3  idle
+//   warps 4-7  softmax of slot A, warps 8-11 softmax of slot B: thread t of a
+//              group owns query row t (its tensor-memory lane), masks partial
+//              tiles, keeps the running max and sum, writes P (bf16) over its
+//              S in tensor memory, rescales O when the max moves far, and
+//              writes O and LSE at the end of the unit
+// The first warpgroup gives registers up (56 per thread) so that the softmax
+// warpgroups can hold a whole row of S (224 per thread): 128 x 56 + 256 x 224
+// equals the 384 x 168 the block is launched with.
 //
-// Tensor memory (512 columns): S double buffer [2 x BN], O [D], P double
-// buffer [2 x BN/2] (bf16 pairs).  S(j+1) = Q K(j+1)^T runs on the tensor
-// cores while the softmax of tile j runs; O += P(j) V(j) follows as soon as
-// P(j) is written.
+// Ping-pong: the MMA warp issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the
+// tensor cores work on one slot while the other slot's softmax runs.
 //
-// Every wait is bounded (`timeout` SM cycles).  On expiry the waiting role
-// sets a bit in the device status word and an abort flag, everyone leaves
-// their loops, in-flight copies and MMAs are waited for (again bounded), the
-// tensor memory is freed and the CTA exits.
+// Tensor memory (512 columns): S_A, S_B [BN each], O_A, O_B [D each].  P_X
+// (bf16 pairs, BN/2 columns) is written over the first columns of S_X once S_X
+// has been read; the next S_X MMA is issued after PV_X, and tcgen05.mma
+// operations issued by one thread execute in issue order.  A commit after
+// S_X(j) also covers PV_X(j-1), so when the softmax sees S_X(j), O_X holds
+// every product up to tile j-1.
+//
+// Every wait is bounded (`timeout` SM cycles).  On expiry the waiting role sets
+// a bit in the device status word and an abort flag, everyone leaves their
+// loops, in-flight copies and MMAs are waited for (again bounded), the tensor
+// memory is freed and the CTA exits.
 #pragma once
 
 #include <cuda.h>
@@ -45,13 +58,15 @@ struct FwdParams {
     int32_t T;                // mask tiles per side
     int32_t N, B, Hq, Hkv, group;
     int32_t n_qtiles;         // ceil(N / 128): query tiles of 128 rows
+    int32_t n_units;          // work units
+    int32_t pairs;            // grouped: ceil(group / 2); else ceil(n_qtiles / 2)
     int32_t window, sinks, stride, n_global;
     float scale_log2;         // scale * log2(e)
     __nv_bfloat16* O;
     float* LSE;
     int32_t* status;          // device status word (bits: which wait expired)
     long long timeout;        // SM cycles per wait
-    int32_t debug_flags;      // bit 0: skip the Q load (test hook)
+    int32_t debug_flags;      // bit 0: skip the first Q load (test hook)
 };
 
 enum : int32_t {
@@ -62,8 +77,10 @@ enum : int32_t {
     ST_DRAIN_WAIT = 16,
 };
 
-constexpr int kThreads = 192;
-constexpr int kBM = 128;  // query rows per CTA tile
+constexpr int kThreads = 384;
+constexpr int kRegsControl = 56;
+constexpr int kRegsSoftmax = 224;
+constexpr int kBM = 128;  // query rows per slot
 
 template <int D, int BN>
 struct FwdCfg {
@@ -73,106 +90,165 @@ struct FwdCfg {
     static constexpr int kKVBytes = BN * D * 2;
     static constexpr int kQPanel = kBM * 128;  // 64 columns x 128 rows
     static constexpr int kKVPanel = BN * 128;  // 64 columns x BN rows
-    // shared memory offsets (1024-byte aligned base)
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffQ = 0;            // two slots
+    static constexpr int kOffK = kOffQ + 2 * kQBytes;
     static constexpr int kOffV = kOffK + kStagesK * kKVBytes;
     static constexpr int kOffBar = kOffV + kStagesV * kKVBytes;
-    static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 6 + 1;
+    static constexpr int kNumBars = 2 * kStagesK + 2 * kStagesV + 2 * 6 + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemUsed = kOffMisc + 16;
-    // request at least this much so that one CTA owns the SM's tensor memory
+    // at least this much, so that one CTA owns the SM's tensor memory
     static constexpr int kSmemBytes = (kSmemUsed + 1024 > 120 * 1024) ? kSmemUsed + 1024 : 120 * 1024;
-    // tensor memory columns
-    static constexpr uint32_t kColS = 0;             // + b * BN
-    static constexpr uint32_t kColO = 2 * BN;
-    static constexpr uint32_t kColP = 2 * BN + D;    // + b * BN / 2
     static constexpr uint32_t kTmemCols = 512;
-    static_assert(kColP + BN <= kTmemCols, "tensor memory budget");
+    static_assert(2 * BN + 2 * D <= 512, "tensor memory budget");
     static_assert(kSmemUsed + 1024 <= 227 * 1024, "shared memory budget");
 };
 
-// The live kv tiles of one 128-row query tile.  With 128-wide mask tiles this
-// is one row of the mask; with 64-wide tiles the query tile spans two mask
-// rows and the lists are merged (a tile live in only one of them is partial
-// for the whole query tile).
-struct KvList {
-    const int32_t* a_idx;
-    const uint8_t* a_full;
-    const int32_t* b_idx;
-    const uint8_t* b_full;
-    int a_n, b_n, pa, pb;
-    bool two;
+// One work unit: up to two slots, each a 128-row query tile of one head.
+struct Unit {
+    int b, hkv;
+    int hq[2];
+    int qtile[2];
+    bool valid[2];
+};
 
-    __device__ void init(const FwdParams& p, int qtile, int BN)
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u)
+{
+    Unit w;
+    if (p.group >= 2) {
+        // u = ((n_qtiles - 1 - i) * B * Hkv + b * Hkv + hkv) * pairs + g: later (heavier) tiles first
+        const int g = u % p.pairs;
+        const int r = u / p.pairs;
+        const int bh = r % (p.B * p.Hkv);
+        const int i = p.n_qtiles - 1 - r / (p.B * p.Hkv);
+        w.b = bh / p.Hkv;
+        w.hkv = bh % p.Hkv;
+        w.hq[0] = w.hkv * p.group + 2 * g;
+        w.hq[1] = w.hq[0] + 1;
+        w.qtile[0] = w.qtile[1] = i;
+        w.valid[0] = true;
+        w.valid[1] = 2 * g + 1 < p.group;
+    } else {
+        // u = (pairs - 1 - pp) * B * Hq + b * Hq + h; the slots are q-tiles 2 pp and 2 pp + 1
+        const int bh = u % (p.B * p.Hq);
+        const int pp = p.pairs - 1 - u / (p.B * p.Hq);
+        w.b = bh / p.Hq;
+        w.hkv = bh % p.Hq;
+        w.hq[0] = w.hq[1] = w.hkv;
+        w.qtile[0] = 2 * pp;
+        w.qtile[1] = 2 * pp + 1;
+        w.valid[0] = true;
+        w.valid[1] = 2 * pp + 1 < p.n_qtiles;
+    }
+    return w;
+}
+
+// The union of the live kv tiles of a unit's mask rows (one row per slot with
+// 128-wide tiles, two with 64-wide), walked in ascending order.  Per step it
+// yields the kv tile and, per slot, whether every existing row of the slot
+// marks the tile full; otherwise the slot masks the tile element by element
+// (a tile that is empty for a slot is masked out entirely).
+struct UnitList {
+    const int32_t* idx[4];
+    const uint8_t* full[4];
+    int n[4];
+    int pos[4];
+    bool exists[4];
+
+    __device__ void init(const FwdParams& p, const Unit& w, int BN)
     {
         const int rows_per = kBM / BN;
-        const int r0 = qtile * rows_per;
-        a_idx = p.kv_index + static_cast<int64_t>(r0) * p.T;
-        a_full = p.kv_full + static_cast<int64_t>(r0) * p.T;
-        a_n = min(max(p.kv_count[r0], 0), p.T);  // a count past the row would read the next one
-        two = rows_per == 2 && r0 + 1 < p.T;
-        if (two) {
-            b_idx = a_idx + p.T;
-            b_full = a_full + p.T;
-            b_n = min(max(p.kv_count[r0 + 1], 0), p.T);
-        } else {
-            b_idx = nullptr;
-            b_full = nullptr;
-            b_n = 0;
+#pragma unroll
+        for (int r = 0; r < 4; r++) {
+            const int x = r / 2, k = r % 2;
+            const int row = w.qtile[x] * rows_per + k;
+            exists[r] = w.valid[x] && k < rows_per && row < p.T;
+            const int64_t base = static_cast<int64_t>(exists[r] ? row : 0) * p.T;
+            idx[r] = p.kv_index + base;
+            full[r] = p.kv_full + base;
+            // clamp a corrupt count: never read past the row
+            n[r] = exists[r] ? min(max(__ldg(&p.kv_count[row]), 0), p.T) : 0;
+            pos[r] = 0;
         }
-        pa = pb = 0;
     }
 
-    __device__ bool next(int& kv, bool& full)
+    __device__ bool next(int& kv, bool& fullA, bool& fullB)
     {
-        const bool ha = pa < a_n, hb = pb < b_n;
-        if (!ha && !hb) return false;
-        if (ha && hb) {
-            const int x = a_idx[pa], y = b_idx[pb];
-            if (x == y) {
-                kv = x;
-                full = a_full[pa] && b_full[pb];
-                pa++;
-                pb++;
-            } else if (x < y) {
-                kv = x;
-                full = false;
-                pa++;
-            } else {
-                kv = y;
-                full = false;
-                pb++;
-            }
-            return true;
+        constexpr int kNone = 0x7fffffff;
+        int cur[4];
+        int m = kNone;
+#pragma unroll
+        for (int r = 0; r < 4; r++) {
+            cur[r] = pos[r] < n[r] ? __ldg(&idx[r][pos[r]]) : kNone;
+            m = min(m, cur[r]);
         }
-        if (ha) {
-            kv = a_idx[pa];
-            full = two ? false : (a_full[pa] != 0);
-            pa++;
-        } else {
-            kv = b_idx[pb];
-            full = false;
-            pb++;
+        if (m == kNone) return false;
+        kv = m;
+        bool ok[4];
+#pragma unroll
+        for (int r = 0; r < 4; r++) {
+            const bool hit = cur[r] == m;
+            const bool f = hit && __ldg(&full[r][pos[r]]) != 0;
+            if (hit) pos[r]++;
+            ok[r] = !exists[r] || f;
         }
+        fullA = ok[0] && ok[1];
+        fullB = ok[2] && ok[3];
         return true;
     }
 
-    __device__ int count(const FwdParams& p, int qtile, int BN)
+    __device__ int count() const
     {
-        init(p, qtile, BN);
-        int n = 0, kv;
-        bool f;
-        while (next(kv, f)) n++;
-        init(p, qtile, BN);
-        return n;
+        UnitList c = *this;
+        int n_steps = 0, kv;
+        bool a, b;
+        while (c.next(kv, a, b)) n_steps++;
+        return n_steps;
     }
 };
+
+// Bits lo..hi (inclusive) of a 32-bit word, clipped to 0..31; 0 when empty.
+__device__ __forceinline__ uint32_t bits_between(int lo, int hi)
+{
+    lo = max(lo, 0);
+    hi = min(hi, 31);
+    return lo > hi ? 0u : ((0xffffffffu >> (31 - hi)) & (0xffffffffu << lo));
+}
 
 __device__ __forceinline__ void report(const FwdParams& p, volatile int* abort_flag, int32_t bit)
 {
     *abort_flag = 1;
     atomicOr(p.status, bit);
+}
+
+// packed fp32 pairs (sm_100 f32x2 arithmetic)
+__device__ __forceinline__ uint64_t f2_pack(float a, float b)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 template <int D, int BN>
@@ -181,51 +257,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap tmV, const FwdParams p)
 {
     using C = FwdCfg<D, BN>;
+    constexpr int NK = C::kStagesK, NV = C::kStagesV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem + C::kOffQ;
     uint8_t* sK = smem + C::kOffK;
     uint8_t* sV = smem + C::kOffV;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-    uint64_t* q_full = bars;
-    uint64_t* k_full = bars + 1;
-    uint64_t* k_empty = k_full + C::kStagesK;
-    uint64_t* v_full = k_empty + C::kStagesK;
-    uint64_t* v_empty = v_full + C::kStagesV;
-    uint64_t* s_full = v_empty + C::kStagesV;  // [2]
-    uint64_t* p_full = s_full + 2;             // [2]
-    uint64_t* pv_done = p_full + 2;            // [2]
-    uint64_t* mma_drain = pv_done + 2;         // [1]
+    uint64_t* k_full = bars;
+    uint64_t* k_empty = k_full + NK;
+    uint64_t* v_full = k_empty + NK;
+    uint64_t* v_empty = v_full + NV;
+    uint64_t* q_full = v_empty + NV;  // [2]
+    uint64_t* q_empty = q_full + 2;   // [2]
+    uint64_t* s_full = q_empty + 2;   // [2]
+    uint64_t* p_full = s_full + 2;    // [2]
+    uint64_t* o_full = p_full + 2;    // [2]
+    uint64_t* o_empty = o_full + 2;   // [2]
+    uint64_t* drain = o_empty + 2;    // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
 
-    // work unit: heavier (later) query tiles first
-    const int bh_count = p.B * p.Hq;
-    const int qtile = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) / bh_count;
-    const int bh = static_cast<int>(blockIdx.x) % bh_count;
-    const int b = bh / p.Hq;
-    const int hq = bh % p.Hq;
-    const int hkv = hq / p.group;
-
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
-        for (int s = 0; s < C::kStagesK; s++) {
+        for (int s = 0; s < NK; s++) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
         }
-        for (int s = 0; s < C::kStagesV; s++) {
+        for (int s = 0; s < NV; s++) {
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        for (int s = 0; s < 2; s++) {
-            mbar_init(&s_full[s], 1);
-            mbar_init(&p_full[s], 4 * 32);
-            mbar_init(&pv_done[s], 1);
+        for (int x = 0; x < 2; x++) {
+            mbar_init(&q_full[x], 1);
+            mbar_init(&q_empty[x], 1);
+            mbar_init(&s_full[x], 1);
+            mbar_init(&p_full[x], 128);
+            mbar_init(&o_full[x], 1);
+            mbar_init(&o_empty[x], 128);
         }
-        mbar_init(mma_drain, 1);
+        mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -243,273 +316,357 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const long long lim = p.timeout;
+    // warp-uniform warpgroup index, so that the register split applies per branch
+    const int wg = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x) / 128, 0);
 
-    KvList list;
-    const int n = list.count(p, qtile, BN);
-
+    if (wg == 0) {
+        regs_dec<kRegsControl>();
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ================================================================ producer
         if (lane == 0) {
             const uint64_t pol_q = policy_evict_first();
             const uint64_t pol_kv = policy_evict_last();
-            const int q_row0 = qtile * kBM;
-            const int q_plane = b * p.Hq + hq;
-            const int kv_plane = b * p.Hkv + hkv;
-            bool q_issued = false;
-            if (n > 0 && !(p.debug_flags & 1)) {
-                mbar_arrive_expect_tx(q_full, C::kQBytes);
-                for (int c = 0; c < D / 64; c++)
-                    tma_load_3d(sQ + c * C::kQPanel, &tmQ, q_full, c * 64, q_row0, q_plane, pol_q);
-                q_issued = true;
-            }
-            int k_issued = 0, v_issued = 0;
-            int kv;
-            bool full;
-            for (int j = 0; j < n && !*abort_flag; j++) {
-                list.next(kv, full);
-                const int sk = j % C::kStagesK, sv = j % C::kStagesV;
-                if (!mbar_wait(&k_empty[sk], ((j / C::kStagesK) & 1) ^ 1, lim)) {
-                    report(p, abort_flag, ST_PRODUCER_WAIT);
-                    break;
+            int t = 0;                  // kv steps loaded (K and V of one tile per step)
+            int k_done = 0, v_done = 0; // loads issued, for the drain
+            int q_loads[2] = {0, 0};    // Q loads per slot (phases of q_empty)
+            int q_issued[2] = {0, 0};   // of which actually issued (the test hook skips one)
+            bool dead = false;
+            for (int u = blockIdx.x; u < p.n_units && !dead; u += gridDim.x) {
+                const Unit w = decode_unit(p, u);
+                UnitList L;
+                L.init(p, w, BN);
+                int kv;
+                bool fa, fb;
+                if (!L.next(kv, fa, fb)) continue;  // nothing live: no loads
+#pragma unroll
+                for (int x = 0; x < 2; x++) {
+                    if (dead || !w.valid[x]) continue;
+                    if (!mbar_wait(&q_empty[x], (q_loads[x] & 1) ^ 1, lim)) {
+                        report(p, abort_flag, ST_PRODUCER_WAIT);
+                        dead = true;
+                        continue;
+                    }
+                    const bool skip = (p.debug_flags & 1) && x == 0 && q_loads[0] == 0;
+                    if (!skip) {
+                        mbar_arrive_expect_tx(&q_full[x], C::kQBytes);
+                        for (int c = 0; c < D / 64; c++)
+                            tma_load_3d(sQ + x * C::kQBytes + c * C::kQPanel, &tmQ, &q_full[x], c * 64,
+                                        w.qtile[x] * kBM, w.b * p.Hq + w.hq[x], pol_q);
+                        q_issued[x]++;
+                    }
+                    q_loads[x]++;
                 }
-                mbar_arrive_expect_tx(&k_full[sk], C::kKVBytes);
-                for (int c = 0; c < D / 64; c++)
-                    tma_load_3d(sK + sk * C::kKVBytes + c * C::kKVPanel, &tmK, &k_full[sk], c * 64, kv * BN,
-                                kv_plane, pol_kv);
-                k_issued = j + 1;
-                if (!mbar_wait(&v_empty[sv], ((j / C::kStagesV) & 1) ^ 1, lim)) {
-                    report(p, abort_flag, ST_PRODUCER_WAIT);
-                    break;
+                const int plane = w.b * p.Hkv + w.hkv;
+                bool more = !dead;
+                while (more) {
+                    const int sk = t % NK, sv = t % NV;
+                    if (!mbar_wait(&k_empty[sk], ((t / NK) & 1) ^ 1, lim)) {
+                        report(p, abort_flag, ST_PRODUCER_WAIT);
+                        dead = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&k_full[sk], C::kKVBytes);
+                    for (int c = 0; c < D / 64; c++)
+                        tma_load_3d(sK + sk * C::kKVBytes + c * C::kKVPanel, &tmK, &k_full[sk], c * 64, kv * BN,
+                                    plane, pol_kv);
+                    k_done = t + 1;
+                    if (!mbar_wait(&v_empty[sv], ((t / NV) & 1) ^ 1, lim)) {
+                        report(p, abort_flag, ST_PRODUCER_WAIT);
+                        dead = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&v_full[sv], C::kKVBytes);
+                    for (int c = 0; c < D / 64; c++)
+                        tma_load_3d(sV + sv * C::kKVBytes + c * C::kKVPanel, &tmV, &v_full[sv], c * 64, kv * BN,
+                                    plane, pol_kv);
+                    v_done = t + 1;
+                    t++;
+                    more = !*abort_flag && L.next(kv, fa, fb);
                 }
-                mbar_arrive_expect_tx(&v_full[sv], C::kKVBytes);
-                for (int c = 0; c < D / 64; c++)
-                    tma_load_3d(sV + sv * C::kKVBytes + c * C::kKVPanel, &tmV, &v_full[sv], c * 64, kv * BN,
-                                kv_plane, pol_kv);
-                v_issued = j + 1;
+                if (*abort_flag) dead = true;
             }
             if (*abort_flag) {
-                // Let copies still in flight land before the CTA's shared memory
-                // goes away.  Only the newest load of each stage can be pending.
+                // Copies still in flight land before the CTA's shared memory goes
+                // away; only the newest load of each buffer can be pending.
                 bool ok = true;
-                if (q_issued) ok &= mbar_wait(q_full, 0, lim);
-                for (int t = max(0, k_issued - C::kStagesK); t < k_issued; t++)
-                    ok &= mbar_wait(&k_full[t % C::kStagesK], (t / C::kStagesK) & 1, lim);
-                for (int t = max(0, v_issued - C::kStagesV); t < v_issued; t++)
-                    ok &= mbar_wait(&v_full[t % C::kStagesV], (t / C::kStagesV) & 1, lim);
+#pragma unroll
+                for (int x = 0; x < 2; x++)
+                    if (q_issued[x] > 0) ok &= mbar_wait(&q_full[x], (q_issued[x] - 1) & 1, lim);
+                for (int s = k_done > NK ? k_done - NK : 0; s < k_done; s++)
+                    ok &= mbar_wait(&k_full[s % NK], (s / NK) & 1, lim);
+                for (int s = v_done > NV ? v_done - NV : 0; s < v_done; s++)
+                    ok &= mbar_wait(&v_full[s % NV], (s / NV) & 1, lim);
                 if (!ok) atomicOr(p.status, ST_DRAIN_WAIT);
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && n > 0) {
+        // ================================================================ MMA issuer
+        if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false, false);
             constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, false, true);
-            const uint32_t q_base = smem_addr(sQ);
-            auto issue_pv = [&](int t) -> bool {
-                const int pb = t & 1, sv = t % C::kStagesV;
-                if (!mbar_wait(&v_full[sv], (t / C::kStagesV) & 1, lim)) return false;
-                if (!mbar_wait(&p_full[pb], (t >> 1) & 1, lim)) return false;
-                tc_fence_after_sync();
-                const uint32_t v_base = smem_addr(sV + sv * C::kKVBytes);
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; kk++) {
-                    const uint64_t bd = smem_desc_sw128(v_base + kk * 2048, C::kKVPanel, 1024);
-                    mma_ts(tmem + C::kColO, tmem + C::kColP + pb * (BN / 2) + kk * 8, bd, idesc_o,
-                           (t > 0 || kk > 0) ? 1u : 0u);
-                }
-                tc_commit(&v_empty[sv]);
-                tc_commit(&pv_done[pb]);
-                return true;
-            };
-            bool ok = mbar_wait(q_full, 0, lim);
-            if (!ok) report(p, abort_flag, ST_Q_WAIT);
-            for (int j = 0; ok && j < n && !*abort_flag; j++) {
-                const int sb = j & 1, sk = j % C::kStagesK;
-                ok = mbar_wait(&k_full[sk], (j / C::kStagesK) & 1, lim);
-                if (ok && j >= 2) ok = mbar_wait(&p_full[sb], ((j - 2) >> 1) & 1, lim);  // S buffer consumed
-                if (!ok) {
-                    report(p, abort_flag, ST_MMA_WAIT);
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t k_base = smem_addr(sK + sk * C::kKVBytes);
+            auto issue_s = [&](int x, int stage) {
+                const uint32_t q_base = smem_addr(sQ + x * C::kQBytes);
+                const uint32_t k_base = smem_addr(sK + stage * C::kKVBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; kk++) {
                     const uint32_t off = (kk % 4) * 32;
                     const uint64_t ad = smem_desc_sw128(q_base + (kk / 4) * C::kQPanel + off, 16, 1024);
                     const uint64_t bd = smem_desc_sw128(k_base + (kk / 4) * C::kKVPanel + off, 16, 1024);
-                    mma_ss(tmem + C::kColS + sb * BN, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + x * BN, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                tc_commit(&k_empty[sk]);
-                tc_commit(&s_full[sb]);
-                if (j >= 1 && !issue_pv(j - 1)) {
-                    report(p, abort_flag, ST_MMA_WAIT);
-                    ok = false;
+            };
+            auto issue_pv = [&](int x, int stage, bool accumulate) {
+                const uint32_t v_base = smem_addr(sV + stage * C::kKVBytes);
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; kk++) {
+                    const uint64_t bd = smem_desc_sw128(v_base + kk * 2048, C::kKVPanel, 1024);
+                    mma_ts(tmem + 2 * BN + x * D, tmem + x * BN + kk * 8, bd, idesc_o,
+                           (accumulate || kk > 0) ? 1u : 0u);
                 }
-            }
-            if (ok && !*abort_flag && !issue_pv(n - 1)) report(p, abort_flag, ST_MMA_WAIT);
-            // all issued tensor-core work finished before the memory is released
-            tc_commit(mma_drain);
-            if (!mbar_wait(mma_drain, 0, lim)) atomicOr(p.status, ST_DRAIN_WAIT);
-        }
-    } else {
-        // ------------------------------------------------------------ softmax
-        const int quarter = warp & 3;  // tensor-memory lanes this warp may access
-        const int row = quarter * 32 + lane;
-        const int q = qtile * kBM + row;
-        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32);
-        const int cols = max(p.sinks, p.n_global);
-        const bool row_all = q < p.n_global;
-        float m_ref = -INFINITY;  // running max, log2 units of the scaled score
-        float l_sum = 0.f;
-        bool ok = true;
-        int kv;
-        bool full;
-        for (int j = 0; j < n; j++) {
-            list.next(kv, full);
-            const int sb = j & 1;
-            ok = mbar_wait(&s_full[sb], (j >> 1) & 1, lim);
-            ok = __all_sync(0xffffffffu, ok && !*abort_flag);
-            if (!ok) break;
-            tc_fence_after_sync();
-
-            float s[BN];
+            };
+            int t = 0;                 // kv steps consumed
+            int steps[2] = {0, 0};     // S/P handshakes per slot
+            int units[2] = {0, 0};     // units with work per slot (phases of o_full / o_empty)
+            int q_loads[2] = {0, 0};
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+                const Unit w = decode_unit(p, u);
+                UnitList L;
+                L.init(p, w, BN);
+                const int n = L.count();
+                if (n == 0) continue;
+                const int nx = w.valid[1] ? 2 : 1;
+                // prologue: S_X(0)
+                ok = mbar_wait(&k_full[t % NK], (t / NK) & 1, lim);
 #pragma unroll
-            for (int c = 0; c < BN; c += 32) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_addr(tmem, lane_base, C::kColS + sb * BN + c), r);
-                tmem_wait_ld();
-                reg_fence(r);
-#pragma unroll
-                for (int i = 0; i < 32; i++) s[c + i] = __uint_as_float(r[i]);
-            }
-
-            const int kv0 = kv * BN;
-            if (!full || kv0 + BN > p.N) {
-                // per-element predicate, in tile-local column units
-                const int dq = q - kv0;                              // causal: c <= dq
-                const int c_max = min(dq, p.N - 1 - kv0);
-                const int band_lo = p.window >= 0 ? dq - p.window : 1 << 30;  // band: c >= dq - window
-                const int col_hi = cols - kv0;                       // columns: c < col_hi
-                int next_hit = 1 << 30;                              // stride: c = dq mod s, + k s
-                if (p.stride > 0) {
-                    int r0 = dq % p.stride;
-                    if (r0 < 0) r0 += p.stride;
-                    next_hit = r0;
-                }
-#pragma unroll
-                for (int c = 0; c < BN; c++) {
-                    const bool hit = c == next_hit;
-                    next_hit += hit ? p.stride : 0;
-                    const bool allowed = c <= c_max && (row_all || c >= band_lo || c < col_hi || hit);
-                    s[c] = allowed ? s[c] : -INFINITY;
-                }
-            }
-
-            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-            for (int c = 4; c < BN; c += 4) {
-                mx0 = fmaxf(mx0, s[c]);
-                mx1 = fmaxf(mx1, s[c + 1]);
-                mx2 = fmaxf(mx2, s[c + 2]);
-                mx3 = fmaxf(mx3, s[c + 3]);
-            }
-            const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
-            // Rescale only when the max has grown by more than 2^8: the stale
-            // reference is used for O and l alike, so the result is unchanged.
-            const bool grow = m_tile > m_ref + 8.f;
-            float alpha = 1.f;
-            if (grow) {
-                alpha = ex2_approx(m_ref - m_tile);  // 0 when m_ref = -inf
-                l_sum *= alpha;
-                m_ref = m_tile;
-            }
-            const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-
-            // P buffer sb was last read by PV(j - 2)
-            if (j >= 2) {
-                ok = mbar_wait(&pv_done[sb], ((j - 2) >> 1) & 1, lim);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-            }
-            float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
-            for (int c = 0; c < BN; c += 32) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; i++) {
-                    const float p0 = ex2_approx(fmaf(s[c + 2 * i], p.scale_log2, -m_use));
-                    const float p1 = ex2_approx(fmaf(s[c + 2 * i + 1], p.scale_log2, -m_use));
-                    ls0 += p0;
-                    ls1 += p1;
-                    pk[i] = pack_bf16x2(p0, p1);
-                }
-                tmem_st_32x32b_x16(tmem_addr(tmem, lane_base, C::kColP + sb * (BN / 2) + c / 2), pk);
-            }
-            l_sum += ls0 + ls1;
-
-            if (j >= 1 && __any_sync(0xffffffffu, grow)) {
-                // O holds the sum up to tile j-1 once PV(j-1) is done
-                ok = mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, lim);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-                tc_fence_after_sync();
-#pragma unroll
-                for (int c = 0; c < D; c += 32) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tmem_addr(tmem, lane_base, C::kColO + c), r);
-                    tmem_wait_ld();
-                    reg_fence(r);
-#pragma unroll
-                    for (int i = 0; i < 32; i++) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st_32x32b_x32(tmem_addr(tmem, lane_base, C::kColO + c), r);
-                }
-            }
-            tmem_wait_st();
-            tc_fence_before_sync();
-            mbar_arrive(&p_full[sb]);
-        }
-        if (!ok) {
-            report(p, abort_flag, ST_SOFTMAX_WAIT);
-        } else {
-            // ------------------------------------------------------------ epilogue
-            if (n > 0) {
-                ok = mbar_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, lim);
-                ok = __all_sync(0xffffffffu, ok && !*abort_flag);
-                if (!ok) report(p, abort_flag, ST_SOFTMAX_WAIT);
-                tc_fence_after_sync();
-            }
-            if (ok) {
-                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-                const int64_t orow = (static_cast<int64_t>(b) * p.Hq + hq) * p.N + q;
-                uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D);
-#pragma unroll
-                for (int c = 0; c < D; c += 32) {
-                    uint32_t r[32];
-                    if (n > 0) {
-                        tmem_ld_32x32b_x32(tmem_addr(tmem, lane_base, C::kColO + c), r);
-                        tmem_wait_ld();
-                        reg_fence(r);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; i++) r[i] = 0u;
+                for (int x = 0; x < 2; x++) {
+                    if (x >= nx || !ok) continue;
+                    ok = mbar_wait(&q_full[x], q_loads[x] & 1, lim);
+                    if (!ok) {
+                        report(p, abort_flag, ST_Q_WAIT);
+                        break;
                     }
-                    if (q < p.N) {
+                    q_loads[x]++;
+                    tc_fence_after_sync();
+                    issue_s(x, t % NK);
+                    tc_commit(&s_full[x]);
+                    if (n == 1) tc_commit(&q_empty[x]);
+                }
+                if (!ok) {
+                    report(p, abort_flag, ST_MMA_WAIT);
+                    break;
+                }
+                tc_commit(&k_empty[t % NK]);
+                for (int j = 0; j < n && ok; j++) {
+                    const bool last = j == n - 1;
+                    ok = mbar_wait(&v_full[t % NV], (t / NV) & 1, lim);
 #pragma unroll
-                        for (int i = 0; i < 32; i += 8) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(r[i + 0]) * inv, __uint_as_float(r[i + 1]) * inv);
-                            v.y = pack_bf16x2(__uint_as_float(r[i + 2]) * inv, __uint_as_float(r[i + 3]) * inv);
-                            v.z = pack_bf16x2(__uint_as_float(r[i + 4]) * inv, __uint_as_float(r[i + 5]) * inv);
-                            v.w = pack_bf16x2(__uint_as_float(r[i + 6]) * inv, __uint_as_float(r[i + 7]) * inv);
-                            dst[(c + i) / 8] = v;
+                    for (int x = 0; x < 2; x++) {
+                        if (x >= nx || !ok) continue;
+                        ok = mbar_wait(&p_full[x], steps[x] & 1, lim);
+                        if (ok && j == 0 && units[x] > 0) ok = mbar_wait(&o_empty[x], (units[x] - 1) & 1, lim);
+                        if (!ok) break;
+                        steps[x]++;
+                        tc_fence_after_sync();
+                        issue_pv(x, t % NV, j > 0);
+                        if (last) {
+                            tc_commit(&o_full[x]);
+                        } else {
+                            if (x == 0 && !mbar_wait(&k_full[(t + 1) % NK], ((t + 1) / NK) & 1, lim)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after_sync();
+                            issue_s(x, (t + 1) % NK);
+                            tc_commit(&s_full[x]);
+                            if (j + 1 == n - 1) tc_commit(&q_empty[x]);
                         }
                     }
+                    if (!ok || *abort_flag) {
+                        ok = false;
+                        report(p, abort_flag, ST_MMA_WAIT);
+                        break;
+                    }
+                    tc_commit(&v_empty[t % NV]);
+                    if (!last) tc_commit(&k_empty[(t + 1) % NK]);
+                    t++;
                 }
-                if (q < p.N)
-                    p.LSE[orow] = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
+#pragma unroll
+                for (int x = 0; x < 2; x++)
+                    if (x < nx) units[x]++;
+            }
+            // all issued tensor-core work is finished before the memory is released
+            tc_commit(drain);
+            if (!mbar_wait(drain, 0, lim)) atomicOr(p.status, ST_DRAIN_WAIT);
+        }
+    }
+    } else {
+        regs_inc<kRegsSoftmax>();
+        // ================================================================ softmax
+        const int x = (warp - 4) / 4;    // slot
+        const int quarter = warp & 3;    // tensor-memory lanes this warp may access
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32);
+        const uint32_t col_s = static_cast<uint32_t>(x * BN);
+        const uint32_t col_o = static_cast<uint32_t>(2 * BN + x * D);
+        const int cols = max(p.sinks, p.n_global);
+        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+        int steps = 0, units = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+            const Unit w = decode_unit(p, u);
+            if (!(x == 0 ? w.valid[0] : w.valid[1])) continue;
+            UnitList L;
+            L.init(p, w, BN);
+            const int n = L.count();
+            const int q = (x == 0 ? w.qtile[0] : w.qtile[1]) * kBM + row;
+            const int64_t orow = (static_cast<int64_t>(w.b) * p.Hq + (x == 0 ? w.hq[0] : w.hq[1])) * p.N + q;
+            const bool row_all = q < p.n_global;
+            float m_ref = -INFINITY;  // running max, log2 units of the scaled score
+            float l_sum = 0.f;
+            for (int j = 0; j < n; j++) {
+                int kv;
+                bool fa, fb;
+                L.next(kv, fa, fb);
+                const bool full = x == 0 ? fa : fb;
+                ok = mbar_wait(&s_full[x], steps & 1, lim);
+                ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+                if (!ok) break;
+                tc_fence_after_sync();
+
+                float s[BN];
+                {
+                    uint32_t r[BN / 32][32];
+#pragma unroll
+                    for (int c = 0; c < BN / 32; c++)
+                        tmem_ld_32x32b_x32(tmem_addr(tmem, lane_base, col_s + 32 * c), r[c]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < BN / 32; c++) reg_fence(r[c]);
+#pragma unroll
+                    for (int c = 0; c < BN; c++) s[c] = __uint_as_float(r[c / 32][c % 32]);
+                }
+
+                const int kv0 = kv * BN;
+                if (!full || kv0 + BN > p.N) {
+                    // Allowed columns c = kv - kv0 of this row as 32-bit words, from the
+                    // pattern's intervals: causal c <= dq (and kv < N), band c >= dq - window,
+                    // sink/global columns kv < cols, every stride-th distance, global rows.
+                    const int dq = q - kv0;
+                    const int c_max = min(dq, p.N - 1 - kv0);
+                    uint32_t allow[BN / 32];
+#pragma unroll
+                    for (int w = 0; w < BN / 32; w++) {
+                        const int base = 32 * w;
+                        uint32_t m = bits_between(0, cols - 1 - kv0 - base);
+                        if (p.window >= 0) m |= bits_between(dq - p.window - base, 31);
+                        if (p.stride > 0) {
+                            int r0 = dq % p.stride;
+                            if (r0 < 0) r0 += p.stride;
+                            int h = r0 >= base ? r0 : r0 + ((base - r0 + p.stride - 1) / p.stride) * p.stride;
+                            for (; h < base + 32; h += p.stride) m |= 1u << (h - base);
+                        }
+                        if (row_all) m = 0xffffffffu;
+                        allow[w] = m & bits_between(0, c_max - base);
+                    }
+#pragma unroll
+                    for (int c = 0; c < BN; c++) s[c] = (allow[c / 32] >> (c % 32)) & 1u ? s[c] : -INFINITY;
+                }
+
+                float mx[8];
+#pragma unroll
+                for (int i = 0; i < 8; i++) mx[i] = fmaxf(s[i], s[8 + i]);
+#pragma unroll
+                for (int c = 16; c + 16 <= BN; c += 16)
+#pragma unroll
+                    for (int i = 0; i < 8; i++) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
+                const float m_tile =
+                    fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7])) *
+                    p.scale_log2;
+                // Rescale only when the max grows by more than 2^8: the stale
+                // reference is used for O and l alike, so the result is unchanged.
+                const bool grow = m_tile > m_ref + 8.f;
+                float alpha = 1.f;
+                if (grow) {
+                    alpha = ex2_approx(m_ref - m_tile);  // 0 when m_ref = -inf
+                    l_sum *= alpha;
+                    m_ref = m_tile;
+                }
+                const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+                const uint64_t neg_m = f2_pack(-m_use, -m_use);
+
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                        const float p0 = ex2_approx(fmaf(s[c + 2 * i], p.scale_log2, -m_use));
+                        const float p1 = ex2_approx(fmaf(s[c + 2 * i + 1], p.scale_log2, -m_use));
+                        acc[(2 * i) & 7] += p0;
+                        acc[(2 * i + 1) & 7] += p1;
+                        pk[i] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st_32x32b_x16(tmem_addr(tmem, lane_base, col_s + c / 2), pk);
+                }
+                l_sum += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+
+                if (j > 0 && __any_sync(0xffffffffu, grow)) {
+                    // O_X holds every product up to tile j-1 (the commit of S_X(j) covers PV_X(j-1))
+#pragma unroll
+                    for (int c = 0; c < D; c += 32) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(tmem_addr(tmem, lane_base, col_o + c), r);
+                        tmem_wait_ld();
+                        reg_fence(r);
+#pragma unroll
+                        for (int i = 0; i < 32; i++) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tmem_st_32x32b_x32(tmem_addr(tmem, lane_base, col_o + c), r);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before_sync();
+                mbar_arrive(&p_full[x]);
+                steps++;
+            }
+            if (!ok) break;
+
+            // ---------------------------------------------------------------- epilogue
+            uint32_t o[D / 32][32];
+            if (n > 0) {
+                ok = mbar_wait(&o_full[x], units & 1, lim);
+                ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+                if (!ok) break;
+                tc_fence_after_sync();
+#pragma unroll
+                for (int c = 0; c < D / 32; c++) tmem_ld_32x32b_x32(tmem_addr(tmem, lane_base, col_o + 32 * c), o[c]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < D / 32; c++) reg_fence(o[c]);
+                tc_fence_before_sync();
+                mbar_arrive(&o_empty[x]);  // O_X may now be overwritten by the next unit
+                units++;
+            } else {
+#pragma unroll
+                for (int c = 0; c < D; c++) o[c / 32][c % 32] = 0u;
+            }
+            if (q < p.N) {
+                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+                uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D);
+#pragma unroll
+                for (int c = 0; c < D; c += 8) {
+                    uint4 v;
+                    const uint32_t* oc = &o[c / 32][c % 32];
+                    v.x = pack_bf16x2(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv);
+                    v.y = pack_bf16x2(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv);
+                    v.z = pack_bf16x2(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
+                    v.w = pack_bf16x2(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
+                    dst[c / 8] = v;
+                }
+                p.LSE[orow] = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
             }
         }
+        if (!ok) report(p, abort_flag, ST_SOFTMAX_WAIT);
     }
 
     tc_fence_before_sync();
