@@ -30,6 +30,8 @@ SA_ERR_BUFFER_TOO_SMALL = -4
 SA_ERR_CUDA = -5
 SA_ERR_DEVICE_TIMEOUT = -6
 SA_ERR_MASK_MISMATCH = -7
+SA_ERR_SCRATCH_TOO_SMALL = -8
+NOALLOC_SCRATCH_BYTES = 1 << 20
 
 DEBUG_SKIP_Q_LOAD = 1
 
@@ -37,7 +39,7 @@ EXPORTED = (
     "sparse_attn_num_tiles", "sparse_attn_build_block_mask", "sparse_attn_count_pairs",
     "sparse_attn_fwd", "sparse_attn_fwd_host", "sparse_attn_fwd_host_workspace",
     "sparse_attn_check_device", "sparse_attn_set_debug", "sparse_attn_status_string",
-    "sparse_attn_version",
+    "sparse_attn_version", "sparse_attn_fwd_noalloc",
 )
 
 
@@ -77,6 +79,7 @@ def _load() -> ctypes.CDLL:
     L.sparse_attn_fwd.argtypes = [vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp]
     L.sparse_attn_fwd_host.argtypes = [vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp]
     L.sparse_attn_fwd_host_workspace.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
+    L.sparse_attn_fwd_noalloc.argtypes = [vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp]
     L.sparse_attn_check_device.argtypes = [vp]
     L.sparse_attn_set_debug.argtypes = [ctypes.c_int32, ctypes.c_int64]
     L.sparse_attn_status_string.argtypes = [ctypes.c_int]
@@ -85,7 +88,7 @@ def _load() -> ctypes.CDLL:
     L.sparse_attn_version.restype = ctypes.c_int32
     for name in ("sparse_attn_build_block_mask", "sparse_attn_count_pairs", "sparse_attn_fwd",
                  "sparse_attn_fwd_host", "sparse_attn_fwd_host_workspace", "sparse_attn_check_device",
-                 "sparse_attn_set_debug"):
+                 "sparse_attn_set_debug", "sparse_attn_fwd_noalloc"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -233,6 +236,28 @@ def fwd_host(q_host, k_host, v_host, mask: BlockMask, pattern: Pattern, o_host, 
                                         ctypes.byref(shape), float(scale), o_host.data_ptr(),
                                         lse_host.data_ptr(), workspace.data_ptr(), nbytes, st),
                "sparse_attn_fwd_host")
+
+
+def fwd_noalloc(q, k, v, mask: BlockMask, pattern: Pattern, out, lse, scale: float | None = None,
+                stream=None) -> None:
+    """The forward pass for callers that cannot allocate device memory.
+
+    ``mask`` is the HOST block mask from ``build_block_mask``; ``out`` and
+    ``lse`` are caller-allocated device tensors.  The library keeps its scratch
+    (status word, device copy of the mask) in a static device array of
+    ``NOALLOC_SCRATCH_BYTES``; the call waits for the stream and raises on a
+    device timeout or a mask too large for that array.
+    """
+    import torch
+    B, Hq, N, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    shape = _Shape(B, Hq, k.shape[1], N, D)
+    with torch.cuda.device(q.device):
+        st = _stream_handle(stream, q.device)
+        _check(lib.sparse_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(mask._c()),
+                                           ctypes.byref(pattern._c()), ctypes.byref(shape), float(scale),
+                                           out.data_ptr(), lse.data_ptr(), st), "sparse_attn_fwd_noalloc")
 
 
 def check_device(stream=None, device=None) -> int:

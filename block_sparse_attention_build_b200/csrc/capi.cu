@@ -233,6 +233,7 @@ extern "C" const char* sparse_attn_status_string(int status)
     case SA_ERR_CUDA: return "CUDA error";
     case SA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case SA_ERR_MASK_MISMATCH: return "block mask does not match N and block";
+    case SA_ERR_SCRATCH_TOO_SMALL: return "block mask larger than the static scratch of the no-allocation entry point";
     default: return "unknown status";
     }
 }

@@ -43,6 +43,7 @@ extern "C" {
 #define SA_ERR_CUDA (-5)             /* a CUDA runtime call or kernel launch failed */
 #define SA_ERR_DEVICE_TIMEOUT (-6)   /* a bounded wait inside the kernel expired */
 #define SA_ERR_MASK_MISMATCH (-7)    /* block mask built for another N or block */
+#define SA_ERR_SCRATCH_TOO_SMALL (-8) /* sparse_attn_fwd_noalloc: mask larger than its static scratch */
 
 /*
  * A fixed sparsity pattern.  A pair (q, kv) is allowed when
@@ -154,6 +155,37 @@ int sparse_attn_check_device(void* stream);
  * wait in SM clock cycles (<= 0 restores the default, about one second).
  */
 int sparse_attn_set_debug(int32_t flags, int64_t timeout_cycles);
+
+/*
+ * No-allocation variant of sparse_attn_fwd.  The pages have no counterpart;
+ * it exists for callers that cannot allocate device memory: programs that
+ * reserve all their device memory up front in a pool of their own and must
+ * not call cudaMalloc afterwards (it can block the host, stall other work on
+ * the device, and fail under memory pressure mid-request).  sparse_attn_fwd
+ * allocates a status word on its first call on a device and reads the block
+ * mask from device memory the caller allocated; this call does neither.
+ *
+ * Arguments as sparse_attn_fwd, except that `mask` holds the HOST arrays
+ * returned by sparse_attn_build_block_mask.  Its scratch, the kernel's status
+ * word and a device copy of the mask, lives in one static device array of
+ * SA_NOALLOC_SCRATCH_BYTES that the library holds on every GPU that loads it
+ * until the process exits.  A mask that does not fit (with 256 bytes for the
+ * status word, 4 T + 5 T^2 bytes for T tiles per side: T <= 457) is rejected
+ * with SA_ERR_SCRATCH_TOO_SMALL before any device work.
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current; make it before any stream capture.  Every call clears the
+ * status word, copies the mask, launches on `stream`, then waits for the
+ * stream and returns the device status (SA_ERR_DEVICE_TIMEOUT if a bounded
+ * wait expired).  All calls share the array and it keeps the last call's
+ * contents; calls whose kernels overlap on the GPU race on it (calls from
+ * several host threads are serialised per device).  Calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ */
+#define SA_NOALLOC_SCRATCH_BYTES (1u << 20)
+int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void* V, const sa_block_mask* mask_host,
+                            const sa_pattern* pattern, const sa_shape* shape, float scale, void* O, float* LSE,
+                            void* stream);
 
 const char* sparse_attn_status_string(int status);
 

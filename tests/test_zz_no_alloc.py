@@ -1,0 +1,66 @@
+"""The no-allocation forward entry point, for callers that cannot allocate
+device memory (a program that reserves all of it up front in its own pool and
+must not call cudaMalloc on the request path).
+
+It runs the same kernel as sparse_attn_fwd, with the kernel's scratch (status
+word, device copy of the block mask) in a static device array of the library.
+Checked here through the C ABI: two calls in a row, with different shapes and
+patterns so the shared scratch is rewritten, each against sparse_attn_fwd on
+the same inputs, within the tolerance the parity tests use.  This file is
+collected last so that a stop at the first failure has run everything else.
+"""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+
+import block_sparse_attention_build_b200 as sa
+import synth
+
+O_TOL = 2e-2
+LSE_TOL = 1e-3
+
+
+def test_mask_larger_than_scratch_is_rejected_before_device_work():
+    # T = 458 tiles per side needs 256 + 4 T + 5 T^2 bytes (with alignment) > 1 MiB
+    N, block = 458 * 128, 128
+    mask = sa.build_block_mask(sa.Pattern(window=64), N, block)
+    shape = sa._Shape(1, 1, 1, N, 128)
+    fake = 1 << 20  # never dereferenced: the size check comes first
+    rc = sa.lib.sparse_attn_fwd_noalloc(fake, fake, fake, ctypes.byref(mask._c()),
+                                        ctypes.byref(sa.Pattern(window=64)._c()), ctypes.byref(shape), 0.1,
+                                        fake, fake, None)
+    assert rc == sa.SA_ERR_SCRATCH_TOO_SMALL
+    assert "static scratch" in sa.status_string(rc)
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_fwd_on_two_calls_in_a_row():
+    import torch
+
+    cases = [
+        # (B, Hq, Hkv, N, D, pattern, block): ragged tail and GQA, then a strided pattern on 64-wide tiles
+        (1, 4, 2, 1000, 128, sa.Pattern(window=200, sinks=4), 128),
+        (2, 2, 2, 700, 64, sa.Pattern(window=40, stride=64, n_global=3), 64),
+    ]
+    dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    for i, (B, Hq, Hkv, N, D, p, block) in enumerate(cases):
+        q, k, v = (dev(a) for a in synth.qkv(B, Hq, Hkv, N, D, seed=100 + i))
+        scale = 1 / math.sqrt(D)
+        host_mask = sa.build_block_mask(p, N, block)
+
+        O_ref, L_ref = sa.fwd(q, k, v, host_mask.to_device("cuda"), p, scale=scale)
+        assert sa.check_device() == sa.SA_OK
+
+        O = torch.full_like(q, float("nan"))
+        L = torch.full((B, Hq, N), float("nan"), dtype=torch.float32, device="cuda")
+        shape = sa._Shape(B, Hq, Hkv, N, D)
+        rc = sa.lib.sparse_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            ctypes.byref(host_mask._c()), ctypes.byref(p._c()),
+                                            ctypes.byref(shape), scale, O.data_ptr(), L.data_ptr(),
+                                            torch.cuda.current_stream().cuda_stream)
+        assert rc == sa.SA_OK, sa.status_string(rc)
+        o_err = (O.float() - O_ref.float()).abs().max().item()
+        l_err = (L - L_ref).abs().max().item()
+        assert o_err <= O_TOL and l_err <= LSE_TOL, (i, o_err, l_err)
