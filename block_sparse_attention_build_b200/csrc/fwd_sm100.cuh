@@ -251,6 +251,30 @@ __device__ __forceinline__ float fmax3(float a, float b, float c)
     return d;
 }
 
+// 2^x for two lanes on the FMA pipe: x = j + f with j = round(x) (added in
+// the float's exponent field) and f in [-1/2, 1/2], 2^f by a degree-3 minimax
+// polynomial (relative error 7.5e-5, fitted by csrc/fit_exp2.py).  Returns
+// exactly 0 for x < -125 (and for x = -inf), where the exponent field would
+// underflow.  Valid for x <= 127.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& p0, float& p1)
+{
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
+    const uint64_t t2 = f2_add(x2, f2_pack(kRound, kRound));
+    const uint64_t j2 = f2_add(t2, f2_pack(-kRound, -kRound));
+    const uint64_t f2 = f2_fma(j2, f2_pack(-1.f, -1.f), x2);
+    uint64_t q2 = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f2,
+                         f2_pack(0.2426111251115799f, 0.2426111251115799f));
+    q2 = f2_fma(q2, f2, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+    q2 = f2_fma(q2, f2, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+    float x0, x1, t0, t1, q0, q1;
+    f2_unpack(x2, x0, x1);
+    f2_unpack(t2, t0, t1);
+    f2_unpack(q2, q0, q1);
+    // the low bits of t hold j (two's complement); shifting them into the exponent field scales by 2^j
+    p0 = x0 < -125.f ? 0.f : __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+    p1 = x1 < -125.f ? 0.f : __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 template <int D, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -401,28 +425,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ================================================================ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs this loop converged (operands stay warp-uniform);
+        // one elected lane issues each tcgen05.mma and tcgen05.commit.
+        {
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false, false);
             constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, false, true);
+            const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+            // descriptors of stage / slot bases; a k-step adds its byte offset >> 4
+            const uint64_t q_desc0 = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+            const uint64_t k_desc0 = smem_desc_sw128(smem_addr(sK), 16, 1024);
+            const uint64_t v_desc0 = smem_desc_sw128(smem_addr(sV), C::kKVPanel, 1024);
+            auto commit = [&](uint64_t* bar) {
+                if (elect_one()) tc_commit(bar);
+                __syncwarp();
+            };
             auto issue_s = [&](int x, int stage) {
-                const uint32_t q_base = smem_addr(sQ + x * C::kQBytes);
-                const uint32_t k_base = smem_addr(sK + stage * C::kKVBytes);
+                const uint64_t a0 = q_desc0 + static_cast<uint64_t>((x * C::kQBytes) >> 4);
+                const uint64_t b0 = k_desc0 + static_cast<uint64_t>((stage * C::kKVBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; kk++) {
-                    const uint32_t off = (kk % 4) * 32;
-                    const uint64_t ad = smem_desc_sw128(q_base + (kk / 4) * C::kQPanel + off, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(k_base + (kk / 4) * C::kKVPanel + off, 16, 1024);
-                    mma_ss(tmem + x * BN, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t qo = static_cast<uint32_t>(((kk / 4) * C::kQPanel + (kk % 4) * 32) >> 4);
+                    const uint32_t ko = static_cast<uint32_t>(((kk / 4) * C::kKVPanel + (kk % 4) * 32) >> 4);
+                    if (elect_one()) mma_ss(tm + x * BN, a0 + qo, b0 + ko, idesc_s, kk > 0 ? 1u : 0u);
+                    __syncwarp();
                 }
             };
             auto issue_pv = [&](int x, int stage, bool accumulate) {
-                const uint32_t v_base = smem_addr(sV + stage * C::kKVBytes);
+                const uint64_t b0 = v_desc0 + static_cast<uint64_t>((stage * C::kKVBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; kk++) {
-                    const uint64_t bd = smem_desc_sw128(v_base + kk * 2048, C::kKVPanel, 1024);
-                    mma_ts(tmem + 2 * BN + x * D, tmem + x * BN + kk * 8, bd, idesc_o,
-                           (accumulate || kk > 0) ? 1u : 0u);
+                    if (elect_one())
+                        mma_ts(tm + 2 * BN + x * D, tm + x * BN + kk * 8, b0 + static_cast<uint32_t>(kk * 128),
+                               idesc_o, (accumulate || kk > 0) ? 1u : 0u);
+                    __syncwarp();
                 }
+            };
+            // every lane polls; the outcome is made warp-uniform
+            auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, lim));
             };
             int t = 0;                 // kv steps consumed
             int steps[2] = {0, 0};     // S/P handshakes per slot
@@ -431,64 +471,67 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
                 const Unit w = decode_unit(p, u);
-                UnitList L;
-                L.init(p, w, BN);
-                const int n = L.count();
+                int n, nx;
+                {
+                    UnitList L;
+                    L.init(p, w, BN);
+                    n = L.count();
+                    nx = w.valid[1] ? 2 : 1;
+                }
                 if (n == 0) continue;
-                const int nx = w.valid[1] ? 2 : 1;
                 // prologue: S_X(0)
-                ok = mbar_wait(&k_full[t % NK], (t / NK) & 1, lim);
+                ok = wait(&k_full[t % NK], (t / NK) & 1);
 #pragma unroll
                 for (int x = 0; x < 2; x++) {
                     if (x >= nx || !ok) continue;
-                    ok = mbar_wait(&q_full[x], q_loads[x] & 1, lim);
+                    ok = wait(&q_full[x], q_loads[x] & 1);
                     if (!ok) {
-                        report(p, abort_flag, ST_Q_WAIT);
+                        if (lane == 0) report(p, abort_flag, ST_Q_WAIT);
                         break;
                     }
                     q_loads[x]++;
                     tc_fence_after_sync();
                     issue_s(x, t % NK);
-                    tc_commit(&s_full[x]);
-                    if (n == 1) tc_commit(&q_empty[x]);
+                    commit(&s_full[x]);
+                    if (n == 1) commit(&q_empty[x]);
                 }
                 if (!ok) {
-                    report(p, abort_flag, ST_MMA_WAIT);
+                    if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
                     break;
                 }
-                tc_commit(&k_empty[t % NK]);
+                commit(&k_empty[t % NK]);
                 for (int j = 0; j < n && ok; j++) {
                     const bool last = j == n - 1;
-                    ok = mbar_wait(&v_full[t % NV], (t / NV) & 1, lim);
+                    ok = wait(&v_full[t % NV], (t / NV) & 1);
 #pragma unroll
                     for (int x = 0; x < 2; x++) {
                         if (x >= nx || !ok) continue;
-                        ok = mbar_wait(&p_full[x], steps[x] & 1, lim);
-                        if (ok && j == 0 && units[x] > 0) ok = mbar_wait(&o_empty[x], (units[x] - 1) & 1, lim);
+                        ok = wait(&p_full[x], steps[x] & 1);
+                        if (ok && j == 0 && units[x] > 0) ok = wait(&o_empty[x], (units[x] - 1) & 1);
                         if (!ok) break;
                         steps[x]++;
                         tc_fence_after_sync();
                         issue_pv(x, t % NV, j > 0);
                         if (last) {
-                            tc_commit(&o_full[x]);
+                            commit(&o_full[x]);
                         } else {
-                            if (x == 0 && !mbar_wait(&k_full[(t + 1) % NK], ((t + 1) / NK) & 1, lim)) {
+                            if (x == 0 && !wait(&k_full[(t + 1) % NK], ((t + 1) / NK) & 1)) {
                                 ok = false;
                                 break;
                             }
                             tc_fence_after_sync();
                             issue_s(x, (t + 1) % NK);
-                            tc_commit(&s_full[x]);
-                            if (j + 1 == n - 1) tc_commit(&q_empty[x]);
+                            commit(&s_full[x]);
+                            if (j + 1 == n - 1) commit(&q_empty[x]);
                         }
                     }
-                    if (!ok || *abort_flag) {
-                        ok = false;
-                        report(p, abort_flag, ST_MMA_WAIT);
+                    ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+                    if (!ok) {
+                        if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
                         break;
                     }
-                    tc_commit(&v_empty[t % NV]);
-                    if (!last) tc_commit(&k_empty[(t + 1) % NK]);
+                    commit(&v_empty[t % NV]);
+                    if (!last) commit(&k_empty[(t + 1) % NK]);
                     t++;
                 }
 #pragma unroll
@@ -496,8 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (x < nx) units[x]++;
             }
             // all issued tensor-core work is finished before the memory is released
-            tc_commit(drain);
-            if (!mbar_wait(drain, 0, lim)) atomicOr(p.status, ST_DRAIN_WAIT);
+            commit(drain);
+            if (!wait(drain, 0) && lane == 0) atomicOr(p.status, ST_DRAIN_WAIT);
         }
     }
     } else {
@@ -528,7 +571,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int kv;
                 bool fa, fb;
                 L.next(kv, fa, fb);
-                const bool full = x == 0 ? fa : fb;
+                const int kv0 = kv * BN;
+                const bool masked = !(x == 0 ? fa : fb) || kv0 + BN > p.N;
+                // Allowed columns c = kv - kv0 of this row as 32-bit words, from the
+                // pattern's intervals: causal c <= dq (and kv < N), band c >= dq - window,
+                // sink/global columns kv < cols, every stride-th distance, global rows.
+                // Built before S arrives; applied only on partial tiles.
+                uint32_t allow[BN / 32];
+                if (masked) {
+                    const int dq = q - kv0;
+                    const int c_max = min(dq, p.N - 1 - kv0);
+#pragma unroll
+                    for (int w = 0; w < BN / 32; w++) {
+                        const int base = 32 * w;
+                        uint32_t m = bits_between(0, cols - 1 - kv0 - base);
+                        if (p.window >= 0) m |= bits_between(dq - p.window - base, 31);
+                        if (p.stride > 0) {
+                            int r0 = dq % p.stride;
+                            if (r0 < 0) r0 += p.stride;
+                            int h = r0 >= base ? r0 : r0 + ((base - r0 + p.stride - 1) / p.stride) * p.stride;
+                            for (; h < base + 32; h += p.stride) m |= 1u << (h - base);
+                        }
+                        if (row_all) m = 0xffffffffu;
+                        allow[w] = m & bits_between(0, c_max - base);
+                    }
+                }
+
                 ok = mbar_wait(&s_full[x], steps & 1, lim);
                 ok = __all_sync(0xffffffffu, ok && !*abort_flag);
                 if (!ok) break;
@@ -546,42 +614,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int c = 0; c < BN; c++) s[c] = __uint_as_float(r[c / 32][c % 32]);
                 }
-
-                const int kv0 = kv * BN;
-                if (!full || kv0 + BN > p.N) {
-                    // Allowed columns c = kv - kv0 of this row as 32-bit words, from the
-                    // pattern's intervals: causal c <= dq (and kv < N), band c >= dq - window,
-                    // sink/global columns kv < cols, every stride-th distance, global rows.
-                    const int dq = q - kv0;
-                    const int c_max = min(dq, p.N - 1 - kv0);
-                    uint32_t allow[BN / 32];
-#pragma unroll
-                    for (int w = 0; w < BN / 32; w++) {
-                        const int base = 32 * w;
-                        uint32_t m = bits_between(0, cols - 1 - kv0 - base);
-                        if (p.window >= 0) m |= bits_between(dq - p.window - base, 31);
-                        if (p.stride > 0) {
-                            int r0 = dq % p.stride;
-                            if (r0 < 0) r0 += p.stride;
-                            int h = r0 >= base ? r0 : r0 + ((base - r0 + p.stride - 1) / p.stride) * p.stride;
-                            for (; h < base + 32; h += p.stride) m |= 1u << (h - base);
-                        }
-                        if (row_all) m = 0xffffffffu;
-                        allow[w] = m & bits_between(0, c_max - base);
-                    }
+                if (masked) {
 #pragma unroll
                     for (int c = 0; c < BN; c++) s[c] = (allow[c / 32] >> (c % 32)) & 1u ? s[c] : -INFINITY;
                 }
 
-                float mx[8];
+                // row max: 16 independent chains of three-input max
+                float mx[16];
 #pragma unroll
-                for (int i = 0; i < 8; i++) mx[i] = fmaxf(s[i], s[8 + i]);
+                for (int i = 0; i < 16; i++) mx[i] = fmax3(s[i], s[16 + i], s[32 + i]);
 #pragma unroll
-                for (int c = 16; c + 16 <= BN; c += 16)
+                for (int c = 48; c + 32 <= BN; c += 32)
 #pragma unroll
-                    for (int i = 0; i < 8; i++) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
+                    for (int i = 0; i < 16; i++) mx[i] = fmax3(mx[i], s[c + i], s[c + 16 + i]);
+                if ((BN - 48) % 32 == 16) {
+#pragma unroll
+                    for (int i = 0; i < 16; i++) mx[i] = fmaxf(mx[i], s[BN - 16 + i]);
+                }
                 const float m_tile =
-                    fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7])) *
+                    fmax3(fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmax3(mx[6], mx[7], mx[8])),
+                          fmax3(fmax3(mx[9], mx[10], mx[11]), fmax3(mx[12], mx[13], mx[14]), mx[15]), -INFINITY) *
                     p.scale_log2;
                 // Rescale only when the max grows by more than 2^8: the stale
                 // reference is used for O and l alike, so the result is unchanged.
@@ -595,21 +647,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
                 const uint64_t neg_m = f2_pack(-m_use, -m_use);
 
-                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                // p = 2^(s * scale_log2 - m): 5 of every 8 pairs on the MUFU unit,
+                // 3 on the FMA pipe (exp2_poly), packed two lanes at a time.
+                uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-                for (int c = 0; c < BN; c += 32) {
-                    uint32_t pk[16];
+                for (int c = 0; c < BN; c += 64) {
+                    uint32_t pk[32];
 #pragma unroll
-                    for (int i = 0; i < 16; i++) {
-                        const float p0 = ex2_approx(fmaf(s[c + 2 * i], p.scale_log2, -m_use));
-                        const float p1 = ex2_approx(fmaf(s[c + 2 * i + 1], p.scale_log2, -m_use));
-                        acc[(2 * i) & 7] += p0;
-                        acc[(2 * i + 1) & 7] += p1;
+                    for (int i = 0; i < 32; i++) {
+                        const uint64_t x2 = f2_fma(f2_pack(s[c + 2 * i], s[c + 2 * i + 1]), scale2, neg_m);
+                        float p0, p1;
+                        if (((c / 2 + i) & 7) < 3) {
+                            exp2_poly_x2(x2, p0, p1);
+                        } else {
+                            float x0, x1;
+                            f2_unpack(x2, x0, x1);
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
+                        }
+                        acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
                         pk[i] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st_32x32b_x16(tmem_addr(tmem, lane_base, col_s + c / 2), pk);
+                    tmem_st_32x32b_x32(tmem_addr(tmem, lane_base, col_s + c / 2), pk);
                 }
-                l_sum += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+                {
+                    float a0, a1, b0, b1, c0, c1, d0, d1;
+                    f2_unpack(acc[0], a0, a1);
+                    f2_unpack(acc[1], b0, b1);
+                    f2_unpack(acc[2], c0, c1);
+                    f2_unpack(acc[3], d0, d1);
+                    l_sum += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+                }
 
                 if (j > 0 && __any_sync(0xffffffffu, grow)) {
                     // O_X holds every product up to tile j-1 (the commit of S_X(j) covers PV_X(j-1))
