@@ -54,7 +54,7 @@ int sm_count()
 }
 
 template <int D, int BN>
-int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p, int grid,
+int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo, const FwdParams& p, int grid,
            cudaStream_t stream)
 {
     using C = FwdCfg<D, BN>;
@@ -67,7 +67,7 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, 
             return SA_ERR_CUDA;
         attr_set[dev] = true;
     }
-    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
     return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
@@ -92,6 +92,7 @@ extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, cons
     if (s.Hkv <= 0 || s.Hq % s.Hkv != 0) return SA_ERR_UNSUPPORTED;
     const int64_t T = (int64_t(s.N) + mask->block - 1) / mask->block;
     if (mask->n_q_tiles != T || mask->n_kv_tiles != T) return SA_ERR_MASK_MISMATCH;
+    if (T > kMaxTiles) return SA_ERR_UNSUPPORTED;
     if (!Q || !K || !V || !O || !LSE || !mask->kv_count || !mask->kv_index || !mask->kv_full)
         return SA_ERR_INVALID_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
@@ -109,11 +110,12 @@ extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, cons
     int32_t* status = nullptr;
     if (int rc = status_word(&status)) return rc;
 
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     const uint32_t bn = static_cast<uint32_t>(mask->block);
     if (!make_map_bf16_3d(&mq, Q, s.D, s.N, uint64_t(s.B) * s.Hq, kBM) ||
         !make_map_bf16_3d(&mk, K, s.D, s.N, uint64_t(s.B) * s.Hkv, bn) ||
-        !make_map_bf16_3d(&mv, V, s.D, s.N, uint64_t(s.B) * s.Hkv, bn))
+        !make_map_bf16_3d(&mv, V, s.D, s.N, uint64_t(s.B) * s.Hkv, bn) ||
+        !make_map_bf16_3d(&mo, O, s.D, s.N, uint64_t(s.B) * s.Hq, kBM))
         return SA_ERR_CUDA;
 
     FwdParams p;
@@ -144,10 +146,10 @@ extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, cons
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int g = static_cast<int>(grid);
-    if (s.D == 128 && mask->block == 128) return launch<128, 128>(mq, mk, mv, p, g, st);
-    if (s.D == 64 && mask->block == 128) return launch<64, 128>(mq, mk, mv, p, g, st);
-    if (s.D == 128 && mask->block == 64) return launch<128, 64>(mq, mk, mv, p, g, st);
-    return launch<64, 64>(mq, mk, mv, p, g, st);
+    if (s.D == 128 && mask->block == 128) return launch<128, 128>(mq, mk, mv, mo, p, g, st);
+    if (s.D == 64 && mask->block == 128) return launch<64, 128>(mq, mk, mv, mo, p, g, st);
+    if (s.D == 128 && mask->block == 64) return launch<128, 64>(mq, mk, mv, mo, p, g, st);
+    return launch<64, 64>(mq, mk, mv, mo, p, g, st);
 }
 
 extern "C" int sparse_attn_fwd_host_workspace(const sa_shape* shape, size_t* bytes)

@@ -54,7 +54,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 template <int D, int BN>
 int launch(int dev, int which, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-           const FwdParams& p, int grid, cudaStream_t stream)
+           const CUtensorMap& mo, const FwdParams& p, int grid, cudaStream_t stream)
 {
     using C = FwdCfg<D, BN>;
     auto kern = fwd_kernel<D, BN>;
@@ -63,7 +63,7 @@ int launch(int dev, int which, const CUtensorMap& mq, const CUtensorMap& mk, con
             return SA_ERR_CUDA;
         g_attr[dev][which] = true;
     }
-    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
     return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
@@ -126,11 +126,12 @@ extern "C" int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void*
         cudaMemcpyAsync(d_full, mask->kv_full, size_t(T) * size_t(T), cudaMemcpyHostToDevice, st) != cudaSuccess)
         return SA_ERR_CUDA;
 
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     const uint32_t bn = static_cast<uint32_t>(mask->block);
     if (!make_map_bf16_3d(&mq, Q, s.D, s.N, uint64_t(s.B) * s.Hq, kBM) ||
         !make_map_bf16_3d(&mk, K, s.D, s.N, uint64_t(s.B) * s.Hkv, bn) ||
-        !make_map_bf16_3d(&mv, V, s.D, s.N, uint64_t(s.B) * s.Hkv, bn))
+        !make_map_bf16_3d(&mv, V, s.D, s.N, uint64_t(s.B) * s.Hkv, bn) ||
+        !make_map_bf16_3d(&mo, O, s.D, s.N, uint64_t(s.B) * s.Hq, kBM))
         return SA_ERR_CUDA;
 
     FwdParams p;
@@ -159,13 +160,13 @@ extern "C" int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void*
     const int grid = static_cast<int>(n_units < n_sm ? n_units : n_sm);
     int rc;
     if (s.D == 128 && bn == 128)
-        rc = launch<128, 128>(dev, 0, mq, mk, mv, p, grid, st);
+        rc = launch<128, 128>(dev, 0, mq, mk, mv, mo, p, grid, st);
     else if (s.D == 64 && bn == 128)
-        rc = launch<64, 128>(dev, 1, mq, mk, mv, p, grid, st);
+        rc = launch<64, 128>(dev, 1, mq, mk, mv, mo, p, grid, st);
     else if (s.D == 128)
-        rc = launch<128, 64>(dev, 2, mq, mk, mv, p, grid, st);
+        rc = launch<128, 64>(dev, 2, mq, mk, mv, mo, p, grid, st);
     else
-        rc = launch<64, 64>(dev, 3, mq, mk, mv, p, grid, st);
+        rc = launch<64, 64>(dev, 3, mq, mk, mv, mo, p, grid, st);
     if (rc != SA_OK) return rc;
 
     int32_t word = 0;

@@ -12,8 +12,10 @@
 // cores, an online softmax, O += P V on the tensor cores.
 //
 // Warp roles (384 threads, three warpgroups):
-//   warp 0     TMA producer: Q of both slots per unit, then K and V of each
-//              kv tile of the union into two rings of shared-memory stages
+//   warp 0     producer: builds each unit's step list (the union of the
+//              slots' live kv tiles) into a two-entry shared-memory ring that
+//              the other roles read, then TMA-loads Q of both slots and K and
+//              V of each step into two rings of shared-memory stages
 //   warp 1     allocates tensor memory; one lane issues every tcgen05.mma
 //   warps 2-3  idle
 //   warps 4-7  softmax of slot A, warps 8-11 softmax of slot B: thread t of a
@@ -21,8 +23,8 @@
 //              tiles, keeps the running max and sum, writes P (bf16) over its
 //              S in tensor memory, rescales O when the max moves far, and
 //              writes O and LSE at the end of the unit
-// The first warpgroup gives registers up (56 per thread) so that the softmax
-// warpgroups can hold a whole row of S (224 per thread): 128 x 56 + 256 x 224
+// The first warpgroup gives registers up (88 per thread) so that the softmax
+// warpgroups can hold a whole row of S (208 per thread): 128 x 88 + 256 x 208
 // equals the 384 x 168 the block is launched with.
 //
 // Ping-pong: the MMA warp issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the
@@ -78,9 +80,12 @@ enum : int32_t {
 };
 
 constexpr int kThreads = 384;
-constexpr int kRegsControl = 56;
-constexpr int kRegsSoftmax = 224;
+constexpr int kRegsControl = 88;
+constexpr int kRegsSoftmax = 208;
 constexpr int kBM = 128;  // query rows per slot
+// Largest number of kv tiles per side the kernel handles (the per-unit step
+// list is staged in shared memory with 14-bit tile indices).
+constexpr int kMaxTiles = 4096;
 
 template <int D, int BN>
 struct FwdCfg {
@@ -93,8 +98,12 @@ struct FwdCfg {
     static constexpr int kOffQ = 0;            // two slots
     static constexpr int kOffK = kOffQ + 2 * kQBytes;
     static constexpr int kOffV = kOffK + kStagesK * kKVBytes;
-    static constexpr int kOffBar = kOffV + kStagesV * kKVBytes;
-    static constexpr int kNumBars = 2 * kStagesK + 2 * kStagesV + 2 * 6 + 1;
+    // unit-info ring: per unit its kv steps, 16 bits each (kv tile | fullA << 14 | fullB << 15)
+    static constexpr int kOffList = kOffV + kStagesV * kKVBytes;
+    static constexpr int kOffListN = kOffList + 2 * kMaxTiles * 2;              // int[2] step counts
+    static constexpr int kOffBitmap = kOffListN + 16;                          // live + 4 full bitmaps
+    static constexpr int kOffBar = kOffBitmap + 5 * (kMaxTiles / 32) * 4;
+    static constexpr int kNumBars = 2 * kStagesK + 2 * kStagesV + 2 * 6 + 2 * 2 + 2 + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemUsed = kOffMisc + 16;
     // at least this much, so that one CTA owns the SM's tensor memory
@@ -143,76 +152,79 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u)
     return w;
 }
 
-// The union of the live kv tiles of a unit's mask rows (one row per slot with
-// 128-wide tiles, two with 64-wide), walked in ascending order.  Per step it
-// yields the kv tile and, per slot, whether every existing row of the slot
-// marks the tile full; otherwise the slot masks the tile element by element
-// (a tile that is empty for a slot is masked out entirely).
-struct UnitList {
-    const int32_t* idx[4];
-    const uint8_t* full[4];
-    int n[4];
-    int pos[4];
-    bool exists[4];
-
-    __device__ void init(const FwdParams& p, const Unit& w, int BN)
-    {
-        const int rows_per = kBM / BN;
-#pragma unroll
-        for (int r = 0; r < 4; r++) {
-            const int x = r / 2, k = r % 2;
-            const int row = w.qtile[x] * rows_per + k;
-            exists[r] = w.valid[x] && k < rows_per && row < p.T;
-            const int64_t base = static_cast<int64_t>(exists[r] ? row : 0) * p.T;
-            idx[r] = p.kv_index + base;
-            full[r] = p.kv_full + base;
-            // clamp a corrupt count: never read past the row
-            n[r] = exists[r] ? min(max(__ldg(&p.kv_count[row]), 0), p.T) : 0;
-            pos[r] = 0;
-        }
-    }
-
-    __device__ bool next(int& kv, bool& fullA, bool& fullB)
-    {
-        constexpr int kNone = 0x7fffffff;
-        int cur[4];
-        int m = kNone;
-#pragma unroll
-        for (int r = 0; r < 4; r++) {
-            cur[r] = pos[r] < n[r] ? __ldg(&idx[r][pos[r]]) : kNone;
-            m = min(m, cur[r]);
-        }
-        if (m == kNone) return false;
-        kv = m;
-        bool ok[4];
-#pragma unroll
-        for (int r = 0; r < 4; r++) {
-            const bool hit = cur[r] == m;
-            const bool f = hit && __ldg(&full[r][pos[r]]) != 0;
-            if (hit) pos[r]++;
-            ok[r] = !exists[r] || f;
-        }
-        fullA = ok[0] && ok[1];
-        fullB = ok[2] && ok[3];
-        return true;
-    }
-
-    __device__ int count() const
-    {
-        UnitList c = *this;
-        int n_steps = 0, kv;
-        bool a, b;
-        while (c.next(kv, a, b)) n_steps++;
-        return n_steps;
-    }
-};
-
 // Bits lo..hi (inclusive) of a 32-bit word, clipped to 0..31; 0 when empty.
 __device__ __forceinline__ uint32_t bits_between(int lo, int hi)
 {
     lo = max(lo, 0);
     hi = min(hi, 31);
     return lo > hi ? 0u : ((0xffffffffu >> (31 - hi)) & (0xffffffffu << lo));
+}
+
+// Build the step list of work unit w (whole warp, converged): the ascending
+// union of the live kv tiles of the unit's mask rows, each entry
+// kv | fullA << 14 | fullB << 15, where a slot's flag is set when every
+// existing mask row of that slot marks the tile full.  The rows are read with
+// coalesced loads into shared-memory bitmaps (bm: live, then one full bitmap
+// per row, kMaxTiles / 32 words each), then a warp prefix scan emits the set
+// bits in order.  Returns the number of steps (the same in every lane).
+__device__ __forceinline__ int build_unit_list(const FwdParams& p, const Unit& w, int BN, uint16_t* list,
+                                               uint32_t* bm, int lane)
+{
+    constexpr int W = kMaxTiles / 32;
+    const int rows_per = kBM / BN;
+    const int words = (p.T + 31) / 32;
+    int row[4], cnt[4];
+    bool exists[4];
+#pragma unroll
+    for (int r = 0; r < 4; r++) {
+        const int x = r / 2, k = r % 2;
+        row[r] = w.qtile[x] * rows_per + k;
+        exists[r] = w.valid[x] && k < rows_per && row[r] < p.T;
+        // clamp a corrupt count: never read past the row
+        cnt[r] = exists[r] ? min(max(__ldg(&p.kv_count[row[r]]), 0), p.T) : 0;
+    }
+    for (int i = lane; i < words; i += 32) {
+        bm[i] = 0u;
+#pragma unroll
+        for (int r = 0; r < 4; r++) bm[(1 + r) * W + i] = exists[r] ? 0u : 0xffffffffu;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < 4; r++) {
+        if (!exists[r]) continue;
+        const int32_t* idx = p.kv_index + static_cast<int64_t>(row[r]) * p.T;
+        const uint8_t* fl = p.kv_full + static_cast<int64_t>(row[r]) * p.T;
+        for (int e = lane; e < cnt[r]; e += 32) {
+            const int kv = __ldg(&idx[e]);
+            if (kv < 0 || kv >= p.T) continue;  // a corrupt index is skipped, never followed
+            atomicOr(&bm[kv >> 5], 1u << (kv & 31));
+            if (__ldg(&fl[e])) atomicOr(&bm[(1 + r) * W + (kv >> 5)], 1u << (kv & 31));
+        }
+    }
+    __syncwarp();
+    int base = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+        const int wi = w0 + lane;
+        uint32_t lv = wi < words ? bm[wi] : 0u;
+        const uint32_t fa = wi < words ? (bm[W + wi] & bm[2 * W + wi]) : 0u;
+        const uint32_t fb = wi < words ? (bm[3 * W + wi] & bm[4 * W + wi]) : 0u;
+        const int c = __popc(lv);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int off = base + incl - c;
+        while (lv) {
+            const int b = __ffs(lv) - 1;
+            lv &= lv - 1;
+            list[off++] = static_cast<uint16_t>((wi * 32 + b) | (((fa >> b) & 1u) << 14) | (((fb >> b) & 1u) << 15));
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    __syncwarp();
+    return base;
 }
 
 __device__ __forceinline__ void report(const FwdParams& p, volatile int* abort_flag, int32_t bit)
@@ -278,7 +290,7 @@ __device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& p0, float& p1)
 template <int D, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const FwdParams p)
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const FwdParams p)
 {
     using C = FwdCfg<D, BN>;
     constexpr int NK = C::kStagesK, NV = C::kStagesV;
@@ -298,7 +310,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* p_full = s_full + 2;    // [2]
     uint64_t* o_full = p_full + 2;    // [2]
     uint64_t* o_empty = o_full + 2;   // [2]
-    uint64_t* drain = o_empty + 2;    // [1]
+    uint64_t* info_full = o_empty + 2;  // [2] unit-info ring: producer -> consumers
+    uint64_t* info_empty = info_full + 2;  // [2] consumers (MMA warp + 8 softmax warps) -> producer
+    uint64_t* stage_full = info_empty + 2;  // [2] O staged in the slot's Q buffer (128 softmax threads)
+    uint64_t* drain = stage_full + 2;  // [1]
+    uint16_t* unit_list = reinterpret_cast<uint16_t*>(smem + C::kOffList);  // [2][kMaxTiles]
+    volatile int* unit_n = reinterpret_cast<volatile int*>(smem + C::kOffListN);  // [2]
+    uint32_t* bitmaps = reinterpret_cast<uint32_t*>(smem + C::kOffBitmap);  // [5][kMaxTiles / 32]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -322,6 +340,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&o_full[x], 1);
             mbar_init(&o_empty[x], 128);
         }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(&info_full[b], 32);             // every producer lane
+            mbar_init(&info_empty[b], 32 + 8 * 32);   // every MMA and softmax lane
+            mbar_init(&stage_full[b], 128);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -334,6 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmO);
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -347,69 +371,90 @@ __global__ void __launch_bounds__(kThreads, 1)
         regs_dec<kRegsControl>();
     if (warp == 0) {
         // ================================================================ producer
-        if (lane == 0) {
+        // Whole warp, converged: builds each unit's step list into the
+        // unit-info ring, then one elected lane issues the TMA copies.
+        {
             const uint64_t pol_q = policy_evict_first();
             const uint64_t pol_kv = policy_evict_last();
+            auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, lim));
+            };
             int t = 0;                  // kv steps loaded (K and V of one tile per step)
             int k_done = 0, v_done = 0; // loads issued, for the drain
             int q_loads[2] = {0, 0};    // Q loads per slot (phases of q_empty)
             int q_issued[2] = {0, 0};   // of which actually issued (the test hook skips one)
             bool dead = false;
-            for (int u = blockIdx.x; u < p.n_units && !dead; u += gridDim.x) {
+            int k_unit = 0;             // units of this CTA so far: ring entry k_unit & 1
+            for (int u = blockIdx.x; u < p.n_units && !dead; u += gridDim.x, k_unit++) {
+                const int buf = k_unit & 1;
+                if (!wait(&info_empty[buf], ((k_unit >> 1) & 1) ^ 1)) {
+                    if (lane == 0) report(p, abort_flag, ST_PRODUCER_WAIT);
+                    dead = true;
+                    break;
+                }
                 const Unit w = decode_unit(p, u);
-                UnitList L;
-                L.init(p, w, BN);
-                int kv;
-                bool fa, fb;
-                if (!L.next(kv, fa, fb)) continue;  // nothing live: no loads
+                const uint16_t* list = unit_list + buf * kMaxTiles;
+                const int n = build_unit_list(p, w, BN, unit_list + buf * kMaxTiles, bitmaps, lane);
+                if (lane == 0) unit_n[buf] = n;
+                mbar_arrive(&info_full[buf]);  // every lane releases its own list writes
+                if (n == 0) continue;           // nothing live: no loads
 #pragma unroll
                 for (int x = 0; x < 2; x++) {
                     if (dead || !w.valid[x]) continue;
-                    if (!mbar_wait(&q_empty[x], (q_loads[x] & 1) ^ 1, lim)) {
-                        report(p, abort_flag, ST_PRODUCER_WAIT);
+                    if (!wait(&q_empty[x], (q_loads[x] & 1) ^ 1)) {
+                        if (lane == 0) report(p, abort_flag, ST_PRODUCER_WAIT);
                         dead = true;
                         continue;
                     }
                     const bool skip = (p.debug_flags & 1) && x == 0 && q_loads[0] == 0;
                     if (!skip) {
-                        mbar_arrive_expect_tx(&q_full[x], C::kQBytes);
-                        for (int c = 0; c < D / 64; c++)
-                            tma_load_3d(sQ + x * C::kQBytes + c * C::kQPanel, &tmQ, &q_full[x], c * 64,
-                                        w.qtile[x] * kBM, w.b * p.Hq + w.hq[x], pol_q);
+                        if (elect_one()) {
+                            mbar_arrive_expect_tx(&q_full[x], C::kQBytes);
+                            for (int c = 0; c < D / 64; c++)
+                                tma_load_3d(sQ + x * C::kQBytes + c * C::kQPanel, &tmQ, &q_full[x], c * 64,
+                                            w.qtile[x] * kBM, w.b * p.Hq + w.hq[x], pol_q);
+                        }
+                        __syncwarp();
                         q_issued[x]++;
                     }
                     q_loads[x]++;
                 }
                 const int plane = w.b * p.Hkv + w.hkv;
-                bool more = !dead;
-                while (more) {
+                for (int j = 0; j < n && !dead; j++) {
+                    const int kv = list[j] & 0x3fff;
                     const int sk = t % NK, sv = t % NV;
-                    if (!mbar_wait(&k_empty[sk], ((t / NK) & 1) ^ 1, lim)) {
-                        report(p, abort_flag, ST_PRODUCER_WAIT);
+                    if (!wait(&k_empty[sk], ((t / NK) & 1) ^ 1)) {
+                        if (lane == 0) report(p, abort_flag, ST_PRODUCER_WAIT);
                         dead = true;
                         break;
                     }
-                    mbar_arrive_expect_tx(&k_full[sk], C::kKVBytes);
-                    for (int c = 0; c < D / 64; c++)
-                        tma_load_3d(sK + sk * C::kKVBytes + c * C::kKVPanel, &tmK, &k_full[sk], c * 64, kv * BN,
-                                    plane, pol_kv);
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&k_full[sk], C::kKVBytes);
+                        for (int c = 0; c < D / 64; c++)
+                            tma_load_3d(sK + sk * C::kKVBytes + c * C::kKVPanel, &tmK, &k_full[sk], c * 64,
+                                        kv * BN, plane, pol_kv);
+                    }
+                    __syncwarp();
                     k_done = t + 1;
-                    if (!mbar_wait(&v_empty[sv], ((t / NV) & 1) ^ 1, lim)) {
-                        report(p, abort_flag, ST_PRODUCER_WAIT);
+                    if (!wait(&v_empty[sv], ((t / NV) & 1) ^ 1)) {
+                        if (lane == 0) report(p, abort_flag, ST_PRODUCER_WAIT);
                         dead = true;
                         break;
                     }
-                    mbar_arrive_expect_tx(&v_full[sv], C::kKVBytes);
-                    for (int c = 0; c < D / 64; c++)
-                        tma_load_3d(sV + sv * C::kKVBytes + c * C::kKVPanel, &tmV, &v_full[sv], c * 64, kv * BN,
-                                    plane, pol_kv);
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&v_full[sv], C::kKVBytes);
+                        for (int c = 0; c < D / 64; c++)
+                            tma_load_3d(sV + sv * C::kKVBytes + c * C::kKVPanel, &tmV, &v_full[sv], c * 64,
+                                        kv * BN, plane, pol_kv);
+                    }
+                    __syncwarp();
                     v_done = t + 1;
                     t++;
-                    more = !*abort_flag && L.next(kv, fa, fb);
+                    if (__any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
                 }
-                if (*abort_flag) dead = true;
+                if (__any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
             }
-            if (*abort_flag) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) {
                 // Copies still in flight land before the CTA's shared memory goes
                 // away; only the newest load of each buffer can be pending.
                 bool ok = true;
@@ -420,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok &= mbar_wait(&k_full[s % NK], (s / NK) & 1, lim);
                 for (int s = v_done > NV ? v_done - NV : 0; s < v_done; s++)
                     ok &= mbar_wait(&v_full[s % NV], (s / NV) & 1, lim);
-                if (!ok) atomicOr(p.status, ST_DRAIN_WAIT);
+                if (!ok && lane == 0) atomicOr(p.status, ST_DRAIN_WAIT);
             }
         }
     } else if (warp == 1) {
@@ -469,15 +514,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             int units[2] = {0, 0};     // units with work per slot (phases of o_full / o_empty)
             int q_loads[2] = {0, 0};
             bool ok = true;
-            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-                const Unit w = decode_unit(p, u);
-                int n, nx;
-                {
-                    UnitList L;
-                    L.init(p, w, BN);
-                    n = L.count();
-                    nx = w.valid[1] ? 2 : 1;
+            int k_unit = 0;  // units of this CTA so far: ring entry k_unit & 1
+            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, k_unit++) {
+                const int buf = k_unit & 1;
+                if (!wait(&info_full[buf], (k_unit >> 1) & 1)) {
+                    if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
+                    ok = false;
+                    break;
                 }
+                const int n = unit_n[buf];
+                mbar_arrive(&info_empty[buf]);  // the MMA warp needs only the step count
+                const Unit w = decode_unit(p, u);
+                const int nx = w.valid[1] ? 2 : 1;
                 if (n == 0) continue;
                 // prologue: S_X(0)
                 ok = wait(&k_full[t % NK], (t / NK) & 1);
@@ -493,7 +541,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after_sync();
                     issue_s(x, t % NK);
                     commit(&s_full[x]);
-                    if (n == 1) commit(&q_empty[x]);
                 }
                 if (!ok) {
                     if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
@@ -522,7 +569,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_after_sync();
                             issue_s(x, (t + 1) % NK);
                             commit(&s_full[x]);
-                            if (j + 1 == n - 1) commit(&q_empty[x]);
                         }
                     }
                     ok = __all_sync(0xffffffffu, ok && !*abort_flag);
@@ -556,23 +602,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
         int steps = 0, units = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        int k_unit = 0;  // units of this CTA so far: ring entry k_unit & 1
+        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, k_unit++) {
+            const int buf = k_unit & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&info_full[buf], (k_unit >> 1) & 1, lim) && !*abort_flag);
+            if (!ok) break;
+            const int n = unit_n[buf];
+            const uint16_t* list = unit_list + buf * kMaxTiles;
             const Unit w = decode_unit(p, u);
-            if (!(x == 0 ? w.valid[0] : w.valid[1])) continue;
-            UnitList L;
-            L.init(p, w, BN);
-            const int n = L.count();
+            if (!(x == 0 ? w.valid[0] : w.valid[1])) {
+                mbar_arrive(&info_empty[buf]);
+                continue;
+            }
             const int q = (x == 0 ? w.qtile[0] : w.qtile[1]) * kBM + row;
             const int64_t orow = (static_cast<int64_t>(w.b) * p.Hq + (x == 0 ? w.hq[0] : w.hq[1])) * p.N + q;
             const bool row_all = q < p.n_global;
             float m_ref = -INFINITY;  // running max, log2 units of the scaled score
             float l_sum = 0.f;
             for (int j = 0; j < n; j++) {
-                int kv;
-                bool fa, fb;
-                L.next(kv, fa, fb);
+                const uint32_t e = list[j];
+                const int kv = static_cast<int>(e & 0x3fffu);
                 const int kv0 = kv * BN;
-                const bool masked = !(x == 0 ? fa : fb) || kv0 + BN > p.N;
+                const bool masked = !((e >> (14 + x)) & 1u) || kv0 + BN > p.N;
                 // Allowed columns c = kv - kv0 of this row as 32-bit words, from the
                 // pattern's intervals: causal c <= dq (and kv < N), band c >= dq - window,
                 // sink/global columns kv < cols, every stride-th distance, global rows.
@@ -697,11 +748,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&p_full[x]);
                 steps++;
             }
+            mbar_arrive(&info_empty[buf]);  // this lane has read the unit's steps
             if (!ok) break;
 
             // ---------------------------------------------------------------- epilogue
-            uint32_t o[D / 32][32];
+            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
             if (n > 0) {
+                uint32_t o[D / 32][32];
                 ok = mbar_wait(&o_full[x], units & 1, lim);
                 ok = __all_sync(0xffffffffu, ok && !*abort_flag);
                 if (!ok) break;
@@ -714,13 +767,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before_sync();
                 mbar_arrive(&o_empty[x]);  // O_X may now be overwritten by the next unit
                 units++;
-            } else {
-#pragma unroll
-                for (int c = 0; c < D; c++) o[c / 32][c % 32] = 0u;
-            }
-            if (q < p.N) {
-                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-                uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D);
+                // The slot's Q buffer is free (the o_full commit covers every MMA
+                // that read it): stage the bf16 row there in the 128-byte-swizzled
+                // layout of the O map, and store the tile with TMA (coalesced;
+                // rows past N are clipped).  The producer reloads Q after the
+                // store has read the buffer.
+                uint8_t* stg = sQ + x * C::kQBytes;
 #pragma unroll
                 for (int c = 0; c < D; c += 8) {
                     uint4 v;
@@ -729,11 +781,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                     v.y = pack_bf16x2(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv);
                     v.z = pack_bf16x2(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
                     v.w = pack_bf16x2(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
-                    dst[c / 8] = v;
+                    const int chunk = (c % 64) / 8;
+                    *reinterpret_cast<uint4*>(stg + (c / 64) * C::kQPanel + row * 128 + ((chunk ^ (row & 7)) * 16)) = v;
                 }
-                p.LSE[orow] = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
+                fence_proxy_async_smem();
+                mbar_arrive(&stage_full[x]);
+                if ((warp & 3) == 0 && lane == 0) {
+                    if (mbar_wait(&stage_full[x], (units - 1) & 1, lim)) {
+                        const int plane = w.b * p.Hq + (x == 0 ? w.hq[0] : w.hq[1]);
+                        const int row0 = (x == 0 ? w.qtile[0] : w.qtile[1]) * kBM;
+                        for (int c = 0; c < D / 64; c++)
+                            tma_store_3d(&tmO, stg + c * C::kQPanel, c * 64, row0, plane);
+                        bulk_commit_group();
+                        bulk_wait_read_all();
+                        mbar_arrive(&q_empty[x]);  // the producer may load the next Q here
+                    } else {
+                        report(p, abort_flag, ST_SOFTMAX_WAIT);
+                    }
+                }
+            } else if (q < p.N) {
+                // no live tile for this unit: O = 0 (the slot's Q was never loaded)
+                uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D);
+#pragma unroll
+                for (int c = 0; c < D; c += 8) dst[c / 8] = make_uint4(0u, 0u, 0u, 0u);
             }
+            if (q < p.N)
+                p.LSE[orow] = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
         }
+        if ((warp & 3) == 0 && lane == 0) bulk_wait_all();  // this thread's O stores are complete
         if (!ok) report(p, abort_flag, ST_SOFTMAX_WAIT);
     }
 

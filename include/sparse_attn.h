@@ -120,7 +120,8 @@ int sparse_attn_count_pairs(const sa_pattern* pattern, int64_t N, int64_t* pairs
  * legacy default stream).  Asynchronous: returns once the kernel is queued;
  * launch errors come back as SA_ERR_CUDA, a device-side timeout through
  * sparse_attn_check_device.  Rows with no allowed key get O = 0, LSE = -inf.
- * Supported: D in {64, 128}, mask block in {64, 128}, Hq % Hkv == 0, causal.
+ * Supported: D in {64, 128}, mask block in {64, 128}, Hq % Hkv == 0, causal,
+ * at most 4096 tiles per side (N <= 4096 * block); else SA_ERR_UNSUPPORTED.
  */
 int sparse_attn_fwd(const void* Q, const void* K, const void* V, const sa_block_mask* mask,
                     const sa_pattern* pattern, const sa_shape* shape, float scale, void* O, float* LSE,
