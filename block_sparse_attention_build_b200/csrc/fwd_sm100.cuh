@@ -398,6 +398,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) unit_n[buf] = n;
                 mbar_arrive(&info_full[buf]);  // every lane releases its own list writes
                 if (n == 0) continue;           // nothing live: no loads
+                // Q of this unit into L2 now: its shared-memory load waits for the
+                // previous unit's epilogue to free the slot's Q buffer
+                if (elect_one()) {
+#pragma unroll
+                    for (int x = 0; x < 2; x++)
+                        if (w.valid[x])
+                            for (int c = 0; c < D / 64; c++)
+                                tma_prefetch_l2_3d(&tmQ, c * 64, w.qtile[x] * kBM, w.b * p.Hq + w.hq[x]);
+                }
+                __syncwarp();
 #pragma unroll
                 for (int x = 0; x < 2; x++) {
                     if (dead || !w.valid[x]) continue;
