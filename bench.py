@@ -238,6 +238,26 @@ def config_of(w, n_gpus, extra=None):
     return c
 
 
+def rank_seed(w, rank: int) -> int:
+    """Every rank runs its own, independent batch of the workload (weak scaling)."""
+    return w.seed + rank
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank's time: all_reduce(MAX) of a per-rank float (identity at world 1)."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flop_per_rank_step: float, steps: int, elapsed_ms: float) -> float:
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return world * flop_per_rank_step * steps / (elapsed_ms * 1e-3) / 1e12
+
+
 def run_gpu(args, w):
     import torch
     import torch.distributed as dist
@@ -259,7 +279,7 @@ def run_gpu(args, w):
     mask = mask_h.to_device(dev)
 
     # inputs: every rank its own batch (seed offset by rank); rotate sets past L2
-    q, k, v = synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=w.seed + rank)
+    q, k, v = synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=rank_seed(w, rank))
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
     set_bytes = min_bytes
     n_sets = args.sets if args.sets > 0 else max(1, min(8, math.ceil(3 * L2_BYTES / set_bytes)))
@@ -302,10 +322,7 @@ def run_gpu(args, w):
     status = sa.check_device(stream)
     if status != sa.SA_OK:
         raise SystemExit(f"device status {sa.status_string(status)}")
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist if world > 1 else None, dev)
     mean_launch_ms = float(np.mean(launch_ms))
     median_launch_ms = float(np.median(launch_ms))
 
@@ -331,13 +348,10 @@ def run_gpu(args, w):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, dist if world > 1 else None, dev)
         h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh))
         d2h = Oh.numel() * Oh.element_size() + Lh.numel() * Lh.element_size()
-        e2e = {"value": world * useful * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_tflops(world, useful, e2e_steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                "ms_per_step": e2e_ms / e2e_steps}
 
@@ -349,7 +363,7 @@ def run_gpu(args, w):
 
     peaks, peak_kind = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    value = world * useful * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = job_tflops(world, useful, args.steps, elapsed_ms)
     achieved = executed / (mean_launch_ms * 1e-3) / 1e12
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -367,7 +381,7 @@ def run_gpu(args, w):
             "live_tiles": int(mask_h.n_live), "full_tiles": int(mask_h.n_full),
             "allowed_pairs_per_head": int(pairs)}),
         "useful_frac_of_peak": value / world / peak,
-        "executed_tflops": world * executed * args.steps / (elapsed_ms * 1e-3) / 1e12,
+        "executed_tflops": job_tflops(world, executed, args.steps, elapsed_ms),
         "executed_frac_of_peak": executed / (elapsed_ms / args.steps * 1e-3) / 1e12 / peak,
         "peak_kind": f"bf16 dense, {peak_kind} ({peak} TFLOP/s burst)",
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
