@@ -115,7 +115,7 @@ extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, cons
     if (!make_map_bf16_3d(&mq, Q, s.D, s.N, uint64_t(s.B) * s.Hq, kBM) ||
         !make_map_bf16_3d(&mk, K, s.D, s.N, uint64_t(s.B) * s.Hkv, bn) ||
         !make_map_bf16_3d(&mv, V, s.D, s.N, uint64_t(s.B) * s.Hkv, bn) ||
-        !make_map_bf16_3d(&mo, O, s.D, s.N, uint64_t(s.B) * s.Hq, kBM))
+        !make_map_bf16_3d(&mo, O, s.D, s.N, uint64_t(s.B) * s.Hq, bn))
         return SA_ERR_CUDA;
 
     FwdParams p;

@@ -14,21 +14,31 @@
 // Warp roles (384 threads, three warpgroups):
 //   warp 0     producer: builds each unit's step list (the union of the
 //              slots' live kv tiles) into a two-entry shared-memory ring that
-//              the other roles read, then TMA-loads Q of both slots and K and
-//              V of each step into two rings of shared-memory stages
+//              the other roles read, TMA-loads Q of both slots, and streams the
+//              unit's items through one ring of shared-memory stages: K and V
+//              of every step, then, per slot, the stages that will hold that
+//              slot's O tile (granted without a load)
 //   warp 1     allocates tensor memory; one lane issues every tcgen05.mma
-//   warps 2-3  idle
+//   warp 2     O store: TMA-stores each staged O tile and hands its stages
+//              back to the producer once the store has read them
+//   warp 3     idle
 //   warps 4-7  softmax of slot A, warps 8-11 softmax of slot B: thread t of a
 //              group owns query row t (its tensor-memory lane), masks partial
 //              tiles, keeps the running max and sum, writes P (bf16) over its
-//              S in tensor memory, rescales O when the max moves far, and
-//              writes O and LSE at the end of the unit
+//              S in tensor memory, rescales O when the max moves far, and at
+//              the end of the unit writes its normalised O row (bf16) into the
+//              granted ring stage and its LSE to global memory
 // The first warpgroup gives registers up (88 per thread) so that the softmax
 // warpgroups can hold a whole row of S (208 per thread): 128 x 88 + 256 x 208
 // equals the 384 x 168 the block is launched with.
 //
 // Ping-pong: the MMA warp issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the
 // tensor cores work on one slot while the other slot's softmax runs.
+//
+// Unit boundaries: a slot's Q buffer is handed back by a commit after the
+// slot's last S MMA of the unit, so the next unit's Q is loaded while the last
+// step's softmax and PV run; the O tile goes out through ring stages, so
+// nothing waits for the store before the next unit's first S.
 //
 // Tensor memory (512 columns): S_A, S_B [BN each], O_A, O_B [D each].  P_X
 // (bf16 pairs, BN/2 columns) is written over the first columns of S_X once S_X
@@ -77,6 +87,7 @@ enum : int32_t {
     ST_MMA_WAIT = 4,
     ST_SOFTMAX_WAIT = 8,
     ST_DRAIN_WAIT = 16,
+    ST_STORE_WAIT = 32,
 };
 
 constexpr int kThreads = 384;
@@ -87,28 +98,31 @@ constexpr int kBM = 128;  // query rows per slot
 // list is staged in shared memory with 14-bit tile indices).
 constexpr int kMaxTiles = 4096;
 
+// Bytes of shared memory for the ring of K / V / O stages.
+constexpr int kRingBytes = 128 * 1024;
+
 template <int D, int BN>
 struct FwdCfg {
-    static constexpr int kStagesK = 2;
-    static constexpr int kStagesV = 2;
     static constexpr int kQBytes = kBM * D * 2;
-    static constexpr int kKVBytes = BN * D * 2;
+    static constexpr int kKVBytes = BN * D * 2;             // one ring stage: a K or V tile, or BN rows of O
+    static constexpr int kStages = kRingBytes / kKVBytes;   // 4 (D = BN = 128) to 16 (D = BN = 64)
+    static constexpr int kOBlocks = kBM / BN;               // ring stages per slot's O tile
     static constexpr int kQPanel = kBM * 128;  // 64 columns x 128 rows
     static constexpr int kKVPanel = BN * 128;  // 64 columns x BN rows
     static constexpr int kOffQ = 0;            // two slots
-    static constexpr int kOffK = kOffQ + 2 * kQBytes;
-    static constexpr int kOffV = kOffK + kStagesK * kKVBytes;
+    static constexpr int kOffRing = kOffQ + 2 * kQBytes;
     // unit-info ring: per unit its kv steps, 16 bits each (kv tile | fullA << 14 | fullB << 15)
-    static constexpr int kOffList = kOffV + kStagesV * kKVBytes;
-    static constexpr int kOffListN = kOffList + 2 * kMaxTiles * 2;              // int[2] step counts
+    static constexpr int kOffList = kOffRing + kStages * kKVBytes;
+    static constexpr int kOffListN = kOffList + 2 * kMaxTiles * 2;              // int[2] steps, int[2] ring positions
     static constexpr int kOffBitmap = kOffListN + 16;                          // live + 4 full bitmaps
     static constexpr int kOffBar = kOffBitmap + 5 * (kMaxTiles / 32) * 4;
-    static constexpr int kNumBars = 2 * kStagesK + 2 * kStagesV + 2 * 6 + 2 * 2 + 2 + 1;
+    static constexpr int kNumBars = 2 * kStages + 2 * 7 + 2 * 2 + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemUsed = kOffMisc + 16;
     // at least this much, so that one CTA owns the SM's tensor memory
     static constexpr int kSmemBytes = (kSmemUsed + 1024 > 120 * 1024) ? kSmemUsed + 1024 : 120 * 1024;
     static constexpr uint32_t kTmemCols = 512;
+    static_assert(kStages >= 4 && kRingBytes % kKVBytes == 0, "ring of at least four stages");
     static_assert(2 * BN + 2 * D <= 512, "tensor memory budget");
     static_assert(kSmemUsed + 1024 <= 227 * 1024, "shared memory budget");
 };
@@ -173,16 +187,23 @@ __device__ __forceinline__ int build_unit_list(const FwdParams& p, const Unit& w
     constexpr int W = kMaxTiles / 32;
     const int rows_per = kBM / BN;
     const int words = (p.T + 31) / 32;
-    int row[4], cnt[4];
-    bool exists[4];
+    int row[4], cnt[4], kv0[4];
+    bool exists[4], full0[4];
+    // one round trip: each row's count and its first 32 entries are loaded
+    // together (lane < T keeps every load inside the row)
 #pragma unroll
     for (int r = 0; r < 4; r++) {
         const int x = r / 2, k = r % 2;
         row[r] = w.qtile[x] * rows_per + k;
         exists[r] = w.valid[x] && k < rows_per && row[r] < p.T;
-        // clamp a corrupt count: never read past the row
-        cnt[r] = exists[r] ? min(max(__ldg(&p.kv_count[row[r]]), 0), p.T) : 0;
+        const int64_t off = static_cast<int64_t>(exists[r] ? row[r] : 0) * p.T + lane;
+        const bool in_row = exists[r] && lane < p.T;
+        cnt[r] = exists[r] ? __ldg(&p.kv_count[row[r]]) : 0;
+        kv0[r] = in_row ? __ldg(&p.kv_index[off]) : -1;
+        full0[r] = in_row ? __ldg(&p.kv_full[off]) != 0 : false;
     }
+#pragma unroll
+    for (int r = 0; r < 4; r++) cnt[r] = min(max(cnt[r], 0), p.T);  // clamp a corrupt count: never read past the row
     for (int i = lane; i < words; i += 32) {
         bm[i] = 0u;
 #pragma unroll
@@ -195,10 +216,11 @@ __device__ __forceinline__ int build_unit_list(const FwdParams& p, const Unit& w
         const int32_t* idx = p.kv_index + static_cast<int64_t>(row[r]) * p.T;
         const uint8_t* fl = p.kv_full + static_cast<int64_t>(row[r]) * p.T;
         for (int e = lane; e < cnt[r]; e += 32) {
-            const int kv = __ldg(&idx[e]);
+            const int kv = e < 32 ? kv0[r] : __ldg(&idx[e]);
+            const bool full = e < 32 ? full0[r] : __ldg(&fl[e]) != 0;
             if (kv < 0 || kv >= p.T) continue;  // a corrupt index is skipped, never followed
             atomicOr(&bm[kv >> 5], 1u << (kv & 31));
-            if (__ldg(&fl[e])) atomicOr(&bm[(1 + r) * W + (kv >> 5)], 1u << (kv & 31));
+            if (full) atomicOr(&bm[(1 + r) * W + (kv >> 5)], 1u << (kv & 31));
         }
     }
     __syncwarp();
@@ -293,29 +315,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const FwdParams p)
 {
     using C = FwdCfg<D, BN>;
-    constexpr int NK = C::kStagesK, NV = C::kStagesV;
+    constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem + C::kOffQ;
-    uint8_t* sK = smem + C::kOffK;
-    uint8_t* sV = smem + C::kOffV;
+    uint8_t* ring = smem + C::kOffRing;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-    uint64_t* k_full = bars;
-    uint64_t* k_empty = k_full + NK;
-    uint64_t* v_full = k_empty + NK;
-    uint64_t* v_empty = v_full + NV;
-    uint64_t* q_full = v_empty + NV;  // [2]
-    uint64_t* q_empty = q_full + 2;   // [2]
-    uint64_t* s_full = q_empty + 2;   // [2]
-    uint64_t* p_full = s_full + 2;    // [2]
-    uint64_t* o_full = p_full + 2;    // [2]
-    uint64_t* o_empty = o_full + 2;   // [2]
-    uint64_t* info_full = o_empty + 2;  // [2] unit-info ring: producer -> consumers
-    uint64_t* info_empty = info_full + 2;  // [2] consumers (MMA warp + 8 softmax warps) -> producer
-    uint64_t* stage_full = info_empty + 2;  // [2] O staged in the slot's Q buffer (128 softmax threads)
-    uint64_t* drain = stage_full + 2;  // [1]
+    uint64_t* ring_full = bars;             // [S] a K / V tile landed, or an O stage granted
+    uint64_t* ring_empty = ring_full + S;   // [S] the stage may be refilled
+    uint64_t* q_full = ring_empty + S;      // [2]
+    uint64_t* q_empty = q_full + 2;         // [2] the slot's last S MMA of the unit is done
+    uint64_t* s_full = q_empty + 2;         // [2]
+    uint64_t* p_full = s_full + 2;          // [2]
+    uint64_t* o_full = p_full + 2;          // [2]
+    uint64_t* o_empty = o_full + 2;         // [2]
+    uint64_t* o_staged = o_empty + 2;       // [2] the slot's O tile is in its ring stages (128 softmax threads)
+    uint64_t* info_full = o_staged + 2;     // [2] unit-info ring: producer -> consumers
+    uint64_t* info_empty = info_full + 2;   // [2] consumers (MMA, store and softmax lanes) -> producer
+    uint64_t* drain = info_empty + 2;       // [1]
     uint16_t* unit_list = reinterpret_cast<uint16_t*>(smem + C::kOffList);  // [2][kMaxTiles]
     volatile int* unit_n = reinterpret_cast<volatile int*>(smem + C::kOffListN);  // [2]
+    volatile int* unit_pos = unit_n + 2;  // [2] ring position of the unit's first item
     uint32_t* bitmaps = reinterpret_cast<uint32_t*>(smem + C::kOffBitmap);  // [5][kMaxTiles / 32]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -324,13 +344,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x % 32;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NK; s++) {
-            mbar_init(&k_full[s], 1);
-            mbar_init(&k_empty[s], 1);
-        }
-        for (int s = 0; s < NV; s++) {
-            mbar_init(&v_full[s], 1);
-            mbar_init(&v_empty[s], 1);
+        for (int i = 0; i < S; i++) {
+            mbar_init(&ring_full[i], 1);
+            mbar_init(&ring_empty[i], 1);
         }
         for (int x = 0; x < 2; x++) {
             mbar_init(&q_full[x], 1);
@@ -339,11 +355,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&p_full[x], 128);
             mbar_init(&o_full[x], 1);
             mbar_init(&o_empty[x], 128);
+            mbar_init(&o_staged[x], 128);
         }
         for (int b = 0; b < 2; b++) {
-            mbar_init(&info_full[b], 32);             // every producer lane
-            mbar_init(&info_empty[b], 32 + 8 * 32);   // every MMA and softmax lane
-            mbar_init(&stage_full[b], 128);
+            mbar_init(&info_full[b], 32);                 // every producer lane
+            mbar_init(&info_empty[b], 32 + 32 + 8 * 32);  // every MMA, store and softmax lane
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -379,38 +395,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
                 return __all_sync(0xffffffffu, mbar_wait(bar, parity, lim));
             };
-            int t = 0;                  // kv steps loaded (K and V of one tile per step)
-            int k_done = 0, v_done = 0; // loads issued, for the drain
+            int pos = 0;                // ring items issued (loads and O grants)
             int q_loads[2] = {0, 0};    // Q loads per slot (phases of q_empty)
             int q_issued[2] = {0, 0};   // of which actually issued (the test hook skips one)
             bool dead = false;
-            int k_unit = 0;             // units of this CTA so far: ring entry k_unit & 1
-            for (int u = blockIdx.x; u < p.n_units && !dead; u += gridDim.x, k_unit++) {
-                const int buf = k_unit & 1;
-                if (!wait(&info_empty[buf], ((k_unit >> 1) & 1) ^ 1)) {
+            // Take the next ring stage (bounded wait for its previous item to be released).
+            auto take_stage = [&]() -> bool {
+                if (!wait(&ring_empty[pos % S], ((pos / S) & 1) ^ 1)) {
                     if (lane == 0) report(p, abort_flag, ST_PRODUCER_WAIT);
                     dead = true;
-                    break;
+                    return false;
                 }
+                return true;
+            };
+            // Build unit u's step list into ring entry k & 1 and publish it with
+            // the ring position of the unit's first item.  Returns the step count.
+            auto publish = [&](int u, int k, int first_pos) -> int {
+                const int buf = k & 1;
+                if (!wait(&info_empty[buf], ((k >> 1) & 1) ^ 1)) {
+                    if (lane == 0) report(p, abort_flag, ST_PRODUCER_WAIT);
+                    dead = true;
+                    return 0;
+                }
+                const int n = build_unit_list(p, decode_unit(p, u), BN, unit_list + buf * kMaxTiles, bitmaps, lane);
+                if (lane == 0) {
+                    unit_n[buf] = n;
+                    unit_pos[buf] = first_pos;
+                }
+                mbar_arrive(&info_full[buf]);  // every lane releases its own list writes
+                return n;
+            };
+            int k_unit = 0;             // units of this CTA so far: ring entry k_unit & 1
+            int n = blockIdx.x < p.n_units ? publish(blockIdx.x, 0, 0) : 0;
+            for (int u = blockIdx.x; u < p.n_units && !dead; u += gridDim.x, k_unit++) {
+                const int buf = k_unit & 1;
                 const Unit w = decode_unit(p, u);
                 const uint16_t* list = unit_list + buf * kMaxTiles;
-                const int n = build_unit_list(p, w, BN, unit_list + buf * kMaxTiles, bitmaps, lane);
-                if (lane == 0) unit_n[buf] = n;
-                mbar_arrive(&info_full[buf]);  // every lane releases its own list writes
-                if (n == 0) continue;           // nothing live: no loads
-                // Q of this unit into L2 now: its shared-memory load waits for the
-                // previous unit's epilogue to free the slot's Q buffer
-                if (elect_one()) {
-#pragma unroll
-                    for (int x = 0; x < 2; x++)
-                        if (w.valid[x])
-                            for (int c = 0; c < D / 64; c++)
-                                tma_prefetch_l2_3d(&tmQ, c * 64, w.qtile[x] * kBM, w.b * p.Hq + w.hq[x]);
-                }
+                const int u_next = u + gridDim.x;
+                // Q of the next unit into L2 now; its shared-memory load waits
+                // for the slot's last S MMA of this unit
                 __syncwarp();
 #pragma unroll
                 for (int x = 0; x < 2; x++) {
-                    if (dead || !w.valid[x]) continue;
+                    if (dead || !w.valid[x] || n == 0) continue;
                     if (!wait(&q_empty[x], (q_loads[x] & 1) ^ 1)) {
                         if (lane == 0) report(p, abort_flag, ST_PRODUCER_WAIT);
                         dead = true;
@@ -432,49 +459,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int plane = w.b * p.Hkv + w.hkv;
                 for (int j = 0; j < n && !dead; j++) {
                     const int kv = list[j] & 0x3fff;
-                    const int sk = t % NK, sv = t % NV;
-                    if (!wait(&k_empty[sk], ((t / NK) & 1) ^ 1)) {
-                        if (lane == 0) report(p, abort_flag, ST_PRODUCER_WAIT);
-                        dead = true;
-                        break;
+#pragma unroll
+                    for (int v = 0; v < 2; v++) {  // K, then V
+                        if (!take_stage()) break;
+                        const int st = pos % S;
+                        if (elect_one()) {
+                            mbar_arrive_expect_tx(&ring_full[st], C::kKVBytes);
+                            for (int c = 0; c < D / 64; c++)
+                                tma_load_3d(ring + st * C::kKVBytes + c * C::kKVPanel, v == 0 ? &tmK : &tmV,
+                                            &ring_full[st], c * 64, kv * BN, plane, pol_kv);
+                        }
+                        __syncwarp();
+                        pos++;
                     }
-                    if (elect_one()) {
-                        mbar_arrive_expect_tx(&k_full[sk], C::kKVBytes);
-                        for (int c = 0; c < D / 64; c++)
-                            tma_load_3d(sK + sk * C::kKVBytes + c * C::kKVPanel, &tmK, &k_full[sk], c * 64,
-                                        kv * BN, plane, pol_kv);
-                    }
-                    __syncwarp();
-                    k_done = t + 1;
-                    if (!wait(&v_empty[sv], ((t / NV) & 1) ^ 1)) {
-                        if (lane == 0) report(p, abort_flag, ST_PRODUCER_WAIT);
-                        dead = true;
-                        break;
-                    }
-                    if (elect_one()) {
-                        mbar_arrive_expect_tx(&v_full[sv], C::kKVBytes);
-                        for (int c = 0; c < D / 64; c++)
-                            tma_load_3d(sV + sv * C::kKVBytes + c * C::kKVPanel, &tmV, &v_full[sv], c * 64,
-                                        kv * BN, plane, pol_kv);
-                    }
-                    __syncwarp();
-                    v_done = t + 1;
-                    t++;
                     if (__any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
                 }
+                // the next unit's step list, built while this unit's last steps run
+                const int n_o = n > 0 ? (w.valid[1] ? 2 : 1) * C::kOBlocks : 0;
+                const int n_next = (u_next < p.n_units && !dead) ? publish(u_next, k_unit + 1, pos + n_o) : 0;
+                // the stages that will hold each slot's O tile
+                for (int i = 0; i < n_o && !dead; i++) {
+                    if (!take_stage()) break;
+                    if (elect_one()) mbar_arrive(&ring_full[pos % S]);
+                    __syncwarp();
+                    pos++;
+                }
+                n = n_next;
                 if (__any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
             }
             if (__any_sync(0xffffffffu, *abort_flag != 0)) {
                 // Copies still in flight land before the CTA's shared memory goes
-                // away; only the newest load of each buffer can be pending.
+                // away; only the newest item of each stage can be pending (an O
+                // grant has already completed its phase).
                 bool ok = true;
 #pragma unroll
                 for (int x = 0; x < 2; x++)
                     if (q_issued[x] > 0) ok &= mbar_wait(&q_full[x], (q_issued[x] - 1) & 1, lim);
-                for (int s = k_done > NK ? k_done - NK : 0; s < k_done; s++)
-                    ok &= mbar_wait(&k_full[s % NK], (s / NK) & 1, lim);
-                for (int s = v_done > NV ? v_done - NV : 0; s < v_done; s++)
-                    ok &= mbar_wait(&v_full[s % NV], (s / NV) & 1, lim);
+                for (int i = pos > S ? pos - S : 0; i < pos; i++) ok &= mbar_wait(&ring_full[i % S], (i / S) & 1, lim);
                 if (!ok && lane == 0) atomicOr(p.status, ST_DRAIN_WAIT);
             }
         }
@@ -486,32 +507,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false, false);
             constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, false, true);
             const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
-            // descriptors of stage / slot bases; a k-step adds its byte offset >> 4
-            const uint64_t q_desc0 = smem_desc_sw128(smem_addr(sQ), 16, 1024);
-            const uint64_t k_desc0 = smem_desc_sw128(smem_addr(sK), 16, 1024);
-            const uint64_t v_desc0 = smem_desc_sw128(smem_addr(sV), C::kKVPanel, 1024);
+            // Descriptors of the Q and ring bases as 32-bit halves: a slot, stage
+            // or k-step moves the start address in the low half by (bytes >> 4).
+            const uint64_t qd = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+            const uint64_t kd = smem_desc_sw128(smem_addr(ring), 16, 1024);
+            const uint64_t vd = smem_desc_sw128(smem_addr(ring), C::kKVPanel, 1024);
+            const uint32_t q_lo = static_cast<uint32_t>(qd), k_lo = static_cast<uint32_t>(kd);
+            const uint32_t v_lo = static_cast<uint32_t>(vd), d_hi = static_cast<uint32_t>(qd >> 32);
             auto commit = [&](uint64_t* bar) {
                 if (elect_one()) tc_commit(bar);
                 __syncwarp();
             };
             auto issue_s = [&](int x, int stage) {
-                const uint64_t a0 = q_desc0 + static_cast<uint64_t>((x * C::kQBytes) >> 4);
-                const uint64_t b0 = k_desc0 + static_cast<uint64_t>((stage * C::kKVBytes) >> 4);
+                const uint32_t a0 = q_lo + static_cast<uint32_t>((x * C::kQBytes) >> 4);
+                const uint32_t b0 = k_lo + static_cast<uint32_t>((stage * C::kKVBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; kk++) {
                     const uint32_t qo = static_cast<uint32_t>(((kk / 4) * C::kQPanel + (kk % 4) * 32) >> 4);
                     const uint32_t ko = static_cast<uint32_t>(((kk / 4) * C::kKVPanel + (kk % 4) * 32) >> 4);
-                    if (elect_one()) mma_ss(tm + x * BN, a0 + qo, b0 + ko, idesc_s, kk > 0 ? 1u : 0u);
+                    if (elect_one())
+                        mma_ss(tm + x * BN, desc_from_halves(a0 + qo, d_hi), desc_from_halves(b0 + ko, d_hi), idesc_s,
+                               kk > 0 ? 1u : 0u);
                     __syncwarp();
                 }
             };
             auto issue_pv = [&](int x, int stage, bool accumulate) {
-                const uint64_t b0 = v_desc0 + static_cast<uint64_t>((stage * C::kKVBytes) >> 4);
+                const uint32_t b0 = v_lo + static_cast<uint32_t>((stage * C::kKVBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; kk++) {
                     if (elect_one())
-                        mma_ts(tm + 2 * BN + x * D, tm + x * BN + kk * 8, b0 + static_cast<uint32_t>(kk * 128),
-                               idesc_o, (accumulate || kk > 0) ? 1u : 0u);
+                        mma_ts(tm + 2 * BN + x * D, tm + x * BN + kk * 8,
+                               desc_from_halves(b0 + static_cast<uint32_t>(kk * 128), d_hi), idesc_o,
+                               (accumulate || kk > 0) ? 1u : 0u);
                     __syncwarp();
                 }
             };
@@ -519,7 +546,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
                 return __all_sync(0xffffffffu, mbar_wait(bar, parity, lim));
             };
-            int t = 0;                 // kv steps consumed
             int steps[2] = {0, 0};     // S/P handshakes per slot
             int units[2] = {0, 0};     // units with work per slot (phases of o_full / o_empty)
             int q_loads[2] = {0, 0};
@@ -533,12 +559,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const int n = unit_n[buf];
-                mbar_arrive(&info_empty[buf]);  // the MMA warp needs only the step count
+                const int pos = unit_pos[buf];  // ring position of K(0)
+                mbar_arrive(&info_empty[buf]);  // the MMA warp needs the step count and ring position
                 const Unit w = decode_unit(p, u);
                 const int nx = w.valid[1] ? 2 : 1;
                 if (n == 0) continue;
-                // prologue: S_X(0)
-                ok = wait(&k_full[t % NK], (t / NK) & 1);
+                // prologue: S_X(0) from K(0) at ring position pos
+                ok = wait(&ring_full[pos % S], (pos / S) & 1);
 #pragma unroll
                 for (int x = 0; x < 2; x++) {
                     if (x >= nx || !ok) continue;
@@ -549,17 +576,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     q_loads[x]++;
                     tc_fence_after_sync();
-                    issue_s(x, t % NK);
+                    issue_s(x, pos % S);
                     commit(&s_full[x]);
+                    if (n == 1) commit(&q_empty[x]);  // the slot's last read of Q
                 }
                 if (!ok) {
                     if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
                     break;
                 }
-                commit(&k_empty[t % NK]);
+                commit(&ring_empty[pos % S]);
                 for (int j = 0; j < n && ok; j++) {
                     const bool last = j == n - 1;
-                    ok = wait(&v_full[t % NV], (t / NV) & 1);
+                    const int pv = pos + 2 * j + 1;  // V(j)
+                    const int pk = pv + 1;           // K(j + 1)
+                    ok = wait(&ring_full[pv % S], (pv / S) & 1);
 #pragma unroll
                     for (int x = 0; x < 2; x++) {
                         if (x >= nx || !ok) continue;
@@ -568,17 +598,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!ok) break;
                         steps[x]++;
                         tc_fence_after_sync();
-                        issue_pv(x, t % NV, j > 0);
+                        issue_pv(x, pv % S, j > 0);
                         if (last) {
                             commit(&o_full[x]);
                         } else {
-                            if (x == 0 && !wait(&k_full[(t + 1) % NK], ((t + 1) / NK) & 1)) {
+                            if (x == 0 && !wait(&ring_full[pk % S], (pk / S) & 1)) {
                                 ok = false;
                                 break;
                             }
                             tc_fence_after_sync();
-                            issue_s(x, (t + 1) % NK);
+                            issue_s(x, pk % S);
                             commit(&s_full[x]);
+                            if (j + 2 == n) commit(&q_empty[x]);  // the slot's last read of Q
                         }
                     }
                     ok = __all_sync(0xffffffffu, ok && !*abort_flag);
@@ -586,9 +617,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
                         break;
                     }
-                    commit(&v_empty[t % NV]);
-                    if (!last) commit(&k_empty[(t + 1) % NK]);
-                    t++;
+                    commit(&ring_empty[pv % S]);
+                    if (!last) commit(&ring_empty[pk % S]);
                 }
 #pragma unroll
                 for (int x = 0; x < 2; x++)
@@ -598,6 +628,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             commit(drain);
             if (!wait(drain, 0) && lane == 0) atomicOr(p.status, ST_DRAIN_WAIT);
         }
+    } else if (warp == 2) {
+        // ================================================================ O store
+        // Lane 0 issues the TMA stores of each staged O tile and waits until they
+        // have read shared memory (bulk groups are per thread), then hands the
+        // stages back to the producer.  Rows past N are clipped by the map.
+        bool ok = true;
+        int staged[2] = {0, 0};
+        int k_unit = 0;
+        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, k_unit++) {
+            const int buf = k_unit & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&info_full[buf], (k_unit >> 1) & 1, lim));
+            if (!ok) break;
+            const int n = unit_n[buf];
+            const int pos = unit_pos[buf];
+            mbar_arrive(&info_empty[buf]);
+            const Unit w = decode_unit(p, u);
+            const int nx = w.valid[1] ? 2 : 1;
+            if (n == 0) continue;
+#pragma unroll
+            for (int x = 0; x < 2; x++) {
+                if (x >= nx || !ok) continue;
+                ok = __all_sync(0xffffffffu, mbar_wait(&o_staged[x], staged[x] & 1, lim) && !*abort_flag);
+                if (!ok) continue;
+                staged[x]++;
+                const int first = pos + 2 * n + x * C::kOBlocks;
+                if (lane == 0) {
+                    const int plane = w.b * p.Hq + w.hq[x];
+                    for (int b = 0; b < C::kOBlocks; b++)
+                        for (int c = 0; c < D / 64; c++)
+                            tma_store_3d(&tmO, ring + ((first + b) % S) * C::kKVBytes + c * C::kKVPanel, c * 64,
+                                         w.qtile[x] * kBM + b * BN, plane);
+                    bulk_commit_group();
+                    bulk_wait_read_all();
+                    for (int b = 0; b < C::kOBlocks; b++) mbar_arrive(&ring_empty[(first + b) % S]);
+                }
+                __syncwarp();
+            }
+        }
+        if (lane == 0) bulk_wait_all();  // the O stores are complete
+        if (!ok && lane == 0) report(p, abort_flag, ST_STORE_WAIT);
     }
     } else {
         regs_inc<kRegsSoftmax>();
@@ -758,16 +828,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&p_full[x]);
                 steps++;
             }
+            // first ring item of this slot's O tile
+            const int o_item = unit_pos[buf] + 2 * n + x * C::kOBlocks;
             mbar_arrive(&info_empty[buf]);  // this lane has read the unit's steps
             if (!ok) break;
 
             // ---------------------------------------------------------------- epilogue
             const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
             if (n > 0) {
-                uint32_t o[D / 32][32];
+                // the ring stage granted for this row's block of BN rows of O
+                const int item = o_item + row / BN;
                 ok = mbar_wait(&o_full[x], units & 1, lim);
+                ok = ok && mbar_wait(&ring_full[item % S], (item / S) & 1, lim);
                 ok = __all_sync(0xffffffffu, ok && !*abort_flag);
                 if (!ok) break;
+                uint32_t o[D / 32][32];
                 tc_fence_after_sync();
 #pragma unroll
                 for (int c = 0; c < D / 32; c++) tmem_ld_32x32b_x32(tmem_addr(tmem, lane_base, col_o + 32 * c), o[c]);
@@ -777,12 +852,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before_sync();
                 mbar_arrive(&o_empty[x]);  // O_X may now be overwritten by the next unit
                 units++;
-                // The slot's Q buffer is free (the o_full commit covers every MMA
-                // that read it): stage the bf16 row there in the 128-byte-swizzled
-                // layout of the O map, and store the tile with TMA (coalesced;
-                // rows past N are clipped).  The producer reloads Q after the
-                // store has read the buffer.
-                uint8_t* stg = sQ + x * C::kQBytes;
+                // Stage the bf16 row in the granted stage, in the 128-byte-swizzled
+                // layout of a K tile (the O map's box); the store warp writes it out.
+                uint8_t* stg = ring + (item % S) * C::kKVBytes;
+                const int r = row % BN;
 #pragma unroll
                 for (int c = 0; c < D; c += 8) {
                     uint4 v;
@@ -792,23 +865,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     v.z = pack_bf16x2(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
                     v.w = pack_bf16x2(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
                     const int chunk = (c % 64) / 8;
-                    *reinterpret_cast<uint4*>(stg + (c / 64) * C::kQPanel + row * 128 + ((chunk ^ (row & 7)) * 16)) = v;
+                    *reinterpret_cast<uint4*>(stg + (c / 64) * C::kKVPanel + r * 128 + ((chunk ^ (r & 7)) * 16)) = v;
                 }
                 fence_proxy_async_smem();
-                mbar_arrive(&stage_full[x]);
-                if ((warp & 3) == 0 && lane == 0) {
-                    if (mbar_wait(&stage_full[x], (units - 1) & 1, lim)) {
-                        const int plane = w.b * p.Hq + (x == 0 ? w.hq[0] : w.hq[1]);
-                        const int row0 = (x == 0 ? w.qtile[0] : w.qtile[1]) * kBM;
-                        for (int c = 0; c < D / 64; c++)
-                            tma_store_3d(&tmO, stg + c * C::kQPanel, c * 64, row0, plane);
-                        bulk_commit_group();
-                        bulk_wait_read_all();
-                        mbar_arrive(&q_empty[x]);  // the producer may load the next Q here
-                    } else {
-                        report(p, abort_flag, ST_SOFTMAX_WAIT);
-                    }
-                }
+                mbar_arrive(&o_staged[x]);
             } else if (q < p.N) {
                 // no live tile for this unit: O = 0 (the slot's Q was never loaded)
                 uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D);
@@ -818,7 +878,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (q < p.N)
                 p.LSE[orow] = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
         }
-        if ((warp & 3) == 0 && lane == 0) bulk_wait_all();  // this thread's O stores are complete
         if (!ok) report(p, abort_flag, ST_SOFTMAX_WAIT);
     }
 

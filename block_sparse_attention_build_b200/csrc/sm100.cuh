@@ -64,6 +64,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
     return true;
 }
 
+// As mbar_wait, for a role that waits long and is not on the critical path:
+// sleeps about `ns` nanoseconds between tests so that it takes few issue slots
+// from the warps it shares a scheduler with.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, long long limit, unsigned ns)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > limit) return false;
+        __nanosleep(ns);
+    }
+    return true;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (bulk tensor copies global -> shared, completion on an mbarrier)
 // ---------------------------------------------------------------------------
@@ -288,6 +302,17 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
     d |= static_cast<uint64_t>(1) << 46;   // descriptor version for sm_100
     d |= static_cast<uint64_t>(2) << 61;   // SWIZZLE_128B
+    return d;
+}
+
+// The same descriptor from its two 32-bit halves: the low half holds the
+// start address and the leading offset, the high half the stride offset, the
+// version and the swizzle mode.  Adding (bytes >> 4) to the low half moves the
+// start address (no carry out of its 14-bit field below 256 KB).
+__device__ __forceinline__ uint64_t desc_from_halves(uint32_t lo, uint32_t hi)
+{
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
     return d;
 }
 
