@@ -65,6 +65,10 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, 
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
             return SA_ERR_CUDA;
+        // the warpgroups' register split must fit what the kernel is launched with
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SA_ERR_CUDA;
+        if (fa.numRegs * kThreads < kRegSplitTotal) return SA_ERR_UNSUPPORTED;
         attr_set[dev] = true;
     }
     kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);

@@ -61,6 +61,10 @@ int launch(int dev, int which, const CUtensorMap& mq, const CUtensorMap& mk, con
     if (!g_attr[dev][which]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
             return SA_ERR_CUDA;
+        // the warpgroups' register split must fit what the kernel is launched with
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SA_ERR_CUDA;
+        if (fa.numRegs * kThreads < kRegSplitTotal) return SA_ERR_UNSUPPORTED;
         g_attr[dev][which] = true;
     }
     kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);

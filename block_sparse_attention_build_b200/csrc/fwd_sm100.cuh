@@ -93,6 +93,11 @@ enum : int32_t {
 constexpr int kThreads = 384;
 constexpr int kRegsControl = 88;
 constexpr int kRegsSoftmax = 208;
+// Registers the split hands out; the kernel must be launched with at least this
+// many (threads x registers per thread at launch), or setmaxnreg.inc would wait
+// forever.  The launchers check the compiled count before the first launch.
+constexpr int kRegSplitTotal = 128 * kRegsControl + 256 * kRegsSoftmax;
+static_assert(kRegSplitTotal <= kThreads * 168, "register split");
 constexpr int kBM = 128;  // query rows per slot
 // Largest number of kv tiles per side the kernel handles (the per-unit step
 // list is staged in shared memory with 14-bit tile indices).
