@@ -34,6 +34,7 @@ SA_ERR_SCRATCH_TOO_SMALL = -8
 NOALLOC_SCRATCH_BYTES = 1 << 20
 
 DEBUG_SKIP_Q_LOAD = 1
+DEBUG_SPLIT_ALL = 2
 
 EXPORTED = (
     "sparse_attn_num_tiles", "sparse_attn_build_block_mask", "sparse_attn_count_pairs",

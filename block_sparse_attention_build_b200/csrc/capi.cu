@@ -109,7 +109,17 @@ extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, cons
     if (n_units > INT32_MAX || int64_t(s.B) * s.Hq > INT32_MAX) return SA_ERR_UNSUPPORTED;
     const int n_sm = sm_count();
     if (n_sm <= 0) return SA_ERR_CUDA;
-    const int64_t grid = n_units < n_sm ? n_units : n_sm;
+    int32_t debug_flags = 0;
+    long long timeout = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        timeout = g_timeout;
+        debug_flags = g_debug_flags;
+    }
+    int64_t n_whole = 0, n_items = 0;
+    plan_items(n_units, n_sm, (debug_flags & kDebugSplitAll) != 0, &n_whole, &n_items);
+    if (n_items > INT32_MAX) return SA_ERR_UNSUPPORTED;
+    const int64_t grid = n_items < n_sm ? n_items : n_sm;
 
     int32_t* status = nullptr;
     if (int rc = status_word(&status)) return rc;
@@ -134,6 +144,8 @@ extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, cons
     p.group = s.Hq / s.Hkv;
     p.n_qtiles = static_cast<int32_t>(n_qtiles);
     p.n_units = static_cast<int32_t>(n_units);
+    p.n_whole = static_cast<int32_t>(n_whole);
+    p.n_items = static_cast<int32_t>(n_items);
     p.pairs = static_cast<int32_t>(pairs);
     p.window = pattern->window;
     p.sinks = pattern->sinks;
@@ -143,11 +155,8 @@ extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, cons
     p.O = static_cast<__nv_bfloat16*>(O);
     p.LSE = LSE;
     p.status = status;
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        p.timeout = g_timeout;
-        p.debug_flags = g_debug_flags;
-    }
+    p.timeout = timeout;
+    p.debug_flags = debug_flags;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int g = static_cast<int>(grid);
     if (s.D == 128 && mask->block == 128) return launch<128, 128>(mq, mk, mv, mo, p, g, st);

@@ -150,6 +150,11 @@ extern "C" int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void*
     p.group = static_cast<int32_t>(group);
     p.n_qtiles = static_cast<int32_t>(n_qtiles);
     p.n_units = static_cast<int32_t>(n_units);
+    int64_t n_whole = 0, n_items = 0;
+    plan_items(n_units, n_sm, false, &n_whole, &n_items);
+    if (n_items > INT32_MAX) return SA_ERR_UNSUPPORTED;
+    p.n_whole = static_cast<int32_t>(n_whole);
+    p.n_items = static_cast<int32_t>(n_items);
     p.pairs = static_cast<int32_t>(pairs);
     p.window = pattern->window;
     p.sinks = pattern->sinks;
@@ -161,7 +166,7 @@ extern "C" int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void*
     p.status = status;
     p.timeout = 2000000000LL;
     p.debug_flags = 0;
-    const int grid = static_cast<int>(n_units < n_sm ? n_units : n_sm);
+    const int grid = static_cast<int>(n_items < n_sm ? n_items : n_sm);
     int rc;
     if (s.D == 128 && bn == 128)
         rc = launch<128, 128>(dev, 0, mq, mk, mv, mo, p, grid, st);

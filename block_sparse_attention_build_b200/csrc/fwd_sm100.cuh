@@ -35,6 +35,16 @@
 // Ping-pong: the MMA warp issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the
 // tensor cores work on one slot while the other slot's softmax runs.
 //
+// Split units: when the units do not fill the last round of CTAs evenly, the
+// units of that round are split: each of their query tiles becomes a unit of
+// its own whose two slots hold the same 128 rows, slot A walking the first
+// half of the tile's kv list and slot B the second.  Each slot then streams
+// its own K and V, and at the end slot A's threads merge the two partial
+// results row by row (both accumulators live in the same tensor-memory lanes):
+// with M the larger running max, O = (O_A 2^(m_A - M) + O_B 2^(m_B - M)) /
+// (l_A 2^(m_A - M) + l_B 2^(m_B - M)).  The busiest CTA then does about half a
+// unit more than the mean instead of a whole unit.
+//
 // Unit boundaries: a slot's Q buffer is handed back by a commit after the
 // slot's last S MMA of the unit, so the next unit's Q is loaded while the last
 // step's softmax and PV run; the O tile goes out through ring stages, so
@@ -70,7 +80,9 @@ struct FwdParams {
     int32_t T;                // mask tiles per side
     int32_t N, B, Hq, Hkv, group;
     int32_t n_qtiles;         // ceil(N / 128): query tiles of 128 rows
-    int32_t n_units;          // work units
+    int32_t n_units;          // work units of two slots
+    int32_t n_whole;          // units processed whole; units n_whole.. are split
+    int32_t n_items;          // n_whole + 2 * (n_units - n_whole): what the CTAs walk
     int32_t pairs;            // grouped: ceil(group / 2); else ceil(n_qtiles / 2)
     int32_t window, sinks, stride, n_global;
     float scale_log2;         // scale * log2(e)
@@ -120,8 +132,9 @@ struct FwdCfg {
     static constexpr int kOffList = kOffRing + kStages * kKVBytes;
     static constexpr int kOffListN = kOffList + 2 * kMaxTiles * 2;              // int[2] steps, int[2] ring positions
     static constexpr int kOffBitmap = kOffListN + 16;                          // live + 4 full bitmaps
-    static constexpr int kOffBar = kOffBitmap + 5 * (kMaxTiles / 32) * 4;
-    static constexpr int kNumBars = 2 * kStages + 2 * 7 + 2 * 2 + 1;
+    static constexpr int kOffBar = kOffBitmap + 5 * (kMaxTiles / 32) * 4 + 2 * kBM * 4;
+    static constexpr int kOffMLX = kOffBitmap + 5 * (kMaxTiles / 32) * 4;     // [2][kBM] fp32: slot B's max, sum
+    static constexpr int kNumBars = 2 * kStages + 2 * 7 + 2 * 2 + 1 + 2;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemUsed = kOffMisc + 16;
     // at least this much, so that one CTA owns the SM's tensor memory
@@ -132,17 +145,39 @@ struct FwdCfg {
     static_assert(kSmemUsed + 1024 <= 227 * 1024, "shared memory budget");
 };
 
+// Work items (host side).  Units that fill whole rounds of the CTAs run whole.
+// When the rest would give at most half of the CTAs one more unit, those units
+// are split, two items each, so that the last round costs about half a unit.
+// `split_all` (a test switch) splits every unit.
+inline void plan_items(int64_t n_units, int64_t n_ctas, bool split_all, int64_t* n_whole, int64_t* n_items)
+{
+    int64_t whole = n_units;
+    if (split_all) {
+        whole = 0;
+    } else if (n_units > n_ctas) {
+        const int64_t r = n_units % n_ctas;
+        if (r > 0 && 2 * r <= n_ctas) whole = n_units - r;
+    }
+    *n_whole = whole;
+    *n_items = whole + 2 * (n_units - whole);
+}
+
+// Debug flag: split every unit (exercises the split path on small problems).
+constexpr int32_t kDebugSplitAll = 2;
+
 // One work unit: up to two slots, each a 128-row query tile of one head.
 struct Unit {
     int b, hkv;
     int hq[2];
     int qtile[2];
     bool valid[2];
+    bool split;  // one query tile: slot A takes the first half of its kv list, slot B the second
 };
 
-__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u)
+__device__ __forceinline__ Unit decode_pair(const FwdParams& p, int u)
 {
     Unit w;
+    w.split = false;
     if (p.group >= 2) {
         // u = ((n_qtiles - 1 - i) * B * Hkv + b * Hkv + hkv) * pairs + g: later (heavier) tiles first
         const int g = u % p.pairs;
@@ -170,6 +205,51 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u)
     }
     return w;
 }
+
+// Work item t of the CTAs' walk: a whole unit, or one query tile of a split unit.
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int t)
+{
+    if (t < p.n_whole) return decode_pair(p, t);
+    const int s = t - p.n_whole;
+    const Unit pr = decode_pair(p, p.n_whole + s / 2);
+    const bool x = s & 1;
+    Unit w = pr;
+    w.hq[0] = w.hq[1] = x ? pr.hq[1] : pr.hq[0];
+    w.qtile[0] = w.qtile[1] = x ? pr.qtile[1] : pr.qtile[0];
+    w.valid[0] = w.valid[1] = x ? pr.valid[1] : pr.valid[0];
+    w.split = true;
+    return w;
+}
+
+// Steps of slot x in a unit whose step list has n entries, and the list entry
+// of its step j.
+__device__ __forceinline__ int slot_steps(const Unit& w, int n, int x)
+{
+    if (!(x ? w.valid[1] : w.valid[0])) return 0;
+    if (!w.split) return n;
+    return x == 0 ? (n + 1) / 2 : n / 2;
+}
+__device__ __forceinline__ int slot_entry(const Unit& w, int n, int x, int j)
+{
+    return (w.split && x == 1) ? (n + 1) / 2 + j : j;
+}
+// Ring items of a unit, relative to its first: a whole unit loads K(j), V(j)
+// per step (2n items); a split unit loads K_A(j), K_B(j), V_A(j), V_B(j) while
+// both halves have a step j, then K_A(j), V_A(j) (again 2n items in all).
+__device__ __forceinline__ int k_item(const Unit& w, int n, int x, int j)
+{
+    if (!w.split) return 2 * j;
+    const int nb = n / 2;
+    return j < nb ? 4 * j + x : 4 * nb + 2 * (j - nb);
+}
+__device__ __forceinline__ int v_item(const Unit& w, int n, int x, int j)
+{
+    if (!w.split) return 2 * j + 1;
+    const int nb = n / 2;
+    return j < nb ? 4 * j + 2 + x : 4 * nb + 2 * (j - nb) + 1;
+}
+// Ring stages holding O tiles at the end of a unit: one slot's for a split unit.
+__device__ __forceinline__ int o_slots(const Unit& w) { return (w.split || !w.valid[1]) ? 1 : 2; }
 
 // Bits lo..hi (inclusive) of a 32-bit word, clipped to 0..31; 0 when empty.
 __device__ __forceinline__ uint32_t bits_between(int lo, int hi)
@@ -338,6 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* info_full = o_staged + 2;     // [2] unit-info ring: producer -> consumers
     uint64_t* info_empty = info_full + 2;   // [2] consumers (MMA, store and softmax lanes) -> producer
     uint64_t* drain = info_empty + 2;       // [1]
+    uint64_t* mlx_full = drain + 1;         // [1] split unit: slot B's max and sum are in shared memory
+    uint64_t* mlx_empty = mlx_full + 1;     // [1] slot A has read them
+    float* mlx = reinterpret_cast<float*>(smem + C::kOffMLX);  // [2][kBM]
     uint16_t* unit_list = reinterpret_cast<uint16_t*>(smem + C::kOffList);  // [2][kMaxTiles]
     volatile int* unit_n = reinterpret_cast<volatile int*>(smem + C::kOffListN);  // [2]
     volatile int* unit_pos = unit_n + 2;  // [2] ring position of the unit's first item
@@ -367,6 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&info_empty[b], 32 + 32 + 8 * 32);  // every MMA, store and softmax lane
         }
         mbar_init(drain, 1);
+        mbar_init(mlx_full, 128);
+        mbar_init(mlx_empty, 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -431,8 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return n;
             };
             int k_unit = 0;             // units of this CTA so far: ring entry k_unit & 1
-            int n = blockIdx.x < p.n_units ? publish(blockIdx.x, 0, 0) : 0;
-            for (int u = blockIdx.x; u < p.n_units && !dead; u += gridDim.x, k_unit++) {
+            int n = blockIdx.x < p.n_items ? publish(blockIdx.x, 0, 0) : 0;
+            for (int u = blockIdx.x; u < p.n_items && !dead; u += gridDim.x, k_unit++) {
                 const int buf = k_unit & 1;
                 const Unit w = decode_unit(p, u);
                 const uint16_t* list = unit_list + buf * kMaxTiles;
@@ -442,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
 #pragma unroll
                 for (int x = 0; x < 2; x++) {
-                    if (dead || !w.valid[x] || n == 0) continue;
+                    if (dead || slot_steps(w, n, x) == 0) continue;
                     if (!wait(&q_empty[x], (q_loads[x] & 1) ^ 1)) {
                         if (lane == 0) report(p, abort_flag, ST_PRODUCER_WAIT);
                         dead = true;
@@ -462,26 +547,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                     q_loads[x]++;
                 }
                 const int plane = w.b * p.Hkv + w.hkv;
-                for (int j = 0; j < n && !dead; j++) {
-                    const int kv = list[j] & 0x3fff;
+                if (__builtin_expect(!w.split, 1)) {
+                    for (int j = 0; j < n && !dead; j++) {
+                        const int kv = list[j] & 0x3fff;
 #pragma unroll
-                    for (int v = 0; v < 2; v++) {  // K, then V
-                        if (!take_stage()) break;
-                        const int st = pos % S;
-                        if (elect_one()) {
-                            mbar_arrive_expect_tx(&ring_full[st], C::kKVBytes);
-                            for (int c = 0; c < D / 64; c++)
-                                tma_load_3d(ring + st * C::kKVBytes + c * C::kKVPanel, v == 0 ? &tmK : &tmV,
-                                            &ring_full[st], c * 64, kv * BN, plane, pol_kv);
+                        for (int v = 0; v < 2; v++) {  // K, then V
+                            if (!take_stage()) break;
+                            const int st = pos % S;
+                            if (elect_one()) {
+                                mbar_arrive_expect_tx(&ring_full[st], C::kKVBytes);
+                                for (int c = 0; c < D / 64; c++)
+                                    tma_load_3d(ring + st * C::kKVBytes + c * C::kKVPanel, v == 0 ? &tmK : &tmV,
+                                                &ring_full[st], c * 64, kv * BN, plane, pol_kv);
+                            }
+                            __syncwarp();
+                            pos++;
                         }
-                        __syncwarp();
-                        pos++;
+                        if (__any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
                     }
-                    if (__any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
+                } else {
+                    const int rounds = (n + 1) / 2;
+                    for (int j = 0; j < rounds && !dead; j++) {
+                        // split unit: K_A, K_B, V_A, V_B of step j while both halves have a
+                        // step j, then K_A, V_A
+                        const int m = j < n / 2 ? 4 : 2;
+                        for (int it = 0; it < m; it++) {
+                            if (!take_stage()) break;
+                            const bool is_v = it >= m / 2;
+                            const int kv = list[slot_entry(w, n, m == 4 ? (it & 1) : 0, j)] & 0x3fff;
+                            const int st = pos % S;
+                            if (elect_one()) {
+                                mbar_arrive_expect_tx(&ring_full[st], C::kKVBytes);
+                                for (int c = 0; c < D / 64; c++)
+                                    tma_load_3d(ring + st * C::kKVBytes + c * C::kKVPanel, is_v ? &tmV : &tmK,
+                                                &ring_full[st], c * 64, kv * BN, plane, pol_kv);
+                            }
+                            __syncwarp();
+                            pos++;
+                        }
+                        if (__any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
+                    }
                 }
                 // the next unit's step list, built while this unit's last steps run
-                const int n_o = n > 0 ? (w.valid[1] ? 2 : 1) * C::kOBlocks : 0;
-                const int n_next = (u_next < p.n_units && !dead) ? publish(u_next, k_unit + 1, pos + n_o) : 0;
+                const int n_o = n > 0 ? o_slots(w) * C::kOBlocks : 0;
+                const int n_next = (u_next < p.n_items && !dead) ? publish(u_next, k_unit + 1, pos + n_o) : 0;
                 // the stages that will hold each slot's O tile
                 for (int i = 0; i < n_o && !dead; i++) {
                     if (!take_stage()) break;
@@ -556,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int q_loads[2] = {0, 0};
             bool ok = true;
             int k_unit = 0;  // units of this CTA so far: ring entry k_unit & 1
-            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, k_unit++) {
+            for (int u = blockIdx.x; u < p.n_items && ok; u += gridDim.x, k_unit++) {
                 const int buf = k_unit & 1;
                 if (!wait(&info_full[buf], (k_unit >> 1) & 1)) {
                     if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
@@ -564,16 +673,87 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const int n = unit_n[buf];
-                const int pos = unit_pos[buf];  // ring position of K(0)
+                const int pos = unit_pos[buf];  // ring position of the unit's first item
                 mbar_arrive(&info_empty[buf]);  // the MMA warp needs the step count and ring position
                 const Unit w = decode_unit(p, u);
-                const int nx = w.valid[1] ? 2 : 1;
-                if (n == 0) continue;
-                // prologue: S_X(0) from K(0) at ring position pos
-                ok = wait(&ring_full[pos % S], (pos / S) & 1);
+                if (__builtin_expect(!w.split, 1)) {
+                    const int nx = w.valid[1] ? 2 : 1;
+                    if (n == 0) continue;
+                    // prologue: S_X(0) from K(0) at ring position pos
+                    ok = wait(&ring_full[pos % S], (pos / S) & 1);
 #pragma unroll
-                for (int x = 0; x < 2; x++) {
-                    if (x >= nx || !ok) continue;
+                    for (int x = 0; x < 2; x++) {
+                        if (x >= nx || !ok) continue;
+                        ok = wait(&q_full[x], q_loads[x] & 1);
+                        if (!ok) {
+                            if (lane == 0) report(p, abort_flag, ST_Q_WAIT);
+                            break;
+                        }
+                        q_loads[x]++;
+                        tc_fence_after_sync();
+                        issue_s(x, pos % S);
+                        commit(&s_full[x]);
+                        if (n == 1) commit(&q_empty[x]);  // the slot's last read of Q
+                    }
+                    if (!ok) {
+                        if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
+                        break;
+                    }
+                    commit(&ring_empty[pos % S]);
+                    for (int j = 0; j < n && ok; j++) {
+                        const bool last = j == n - 1;
+                        const int pv = pos + 2 * j + 1;  // V(j)
+                        const int pk = pv + 1;           // K(j + 1)
+                        ok = wait(&ring_full[pv % S], (pv / S) & 1);
+#pragma unroll
+                        for (int x = 0; x < 2; x++) {
+                            if (x >= nx || !ok) continue;
+                            ok = wait(&p_full[x], steps[x] & 1);
+                            if (ok && j == 0 && units[x] > 0) ok = wait(&o_empty[x], (units[x] - 1) & 1);
+                            if (!ok) break;
+                            steps[x]++;
+                            tc_fence_after_sync();
+                            issue_pv(x, pv % S, j > 0);
+                            if (last) {
+                                commit(&o_full[x]);
+                            } else {
+                                if (x == 0 && !wait(&ring_full[pk % S], (pk / S) & 1)) {
+                                    ok = false;
+                                    break;
+                                }
+                                tc_fence_after_sync();
+                                issue_s(x, pk % S);
+                                commit(&s_full[x]);
+                                if (j + 2 == n) commit(&q_empty[x]);  // the slot's last read of Q
+                            }
+                        }
+                        ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+                        if (!ok) {
+                            if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
+                            break;
+                        }
+                        commit(&ring_empty[pv % S]);
+                        if (!last) commit(&ring_empty[pk % S]);
+                    }
+#pragma unroll
+                    for (int x = 0; x < 2; x++)
+                        if (x < nx) units[x]++;
+                    continue;
+                }
+                // split unit: each slot walks its own half of the list with its own K
+                // and V; a stage is released as soon as its one reader is done
+                const int ns0 = slot_steps(w, n, 0), ns1 = slot_steps(w, n, 1);
+                if (ns0 == 0 && ns1 == 0) continue;
+#pragma unroll
+                for (int x = 0; x < 2; x++) {  // prologue: S_X of each half's first step
+                    const int nsx = x ? ns1 : ns0;
+                    if (nsx == 0 || !ok) continue;
+                    const int k0 = pos + k_item(w, n, x, 0);
+                    ok = wait(&ring_full[k0 % S], (k0 / S) & 1);
+                    if (!ok) {
+                        if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
+                        break;
+                    }
                     ok = wait(&q_full[x], q_loads[x] & 1);
                     if (!ok) {
                         if (lane == 0) report(p, abort_flag, ST_Q_WAIT);
@@ -581,40 +761,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     q_loads[x]++;
                     tc_fence_after_sync();
-                    issue_s(x, pos % S);
+                    issue_s(x, k0 % S);
                     commit(&s_full[x]);
-                    if (n == 1) commit(&q_empty[x]);  // the slot's last read of Q
+                    if (nsx == 1) commit(&q_empty[x]);  // the slot's last read of Q
+                    commit(&ring_empty[k0 % S]);
                 }
-                if (!ok) {
-                    if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
-                    break;
-                }
-                commit(&ring_empty[pos % S]);
-                for (int j = 0; j < n && ok; j++) {
-                    const bool last = j == n - 1;
-                    const int pv = pos + 2 * j + 1;  // V(j)
-                    const int pk = pv + 1;           // K(j + 1)
-                    ok = wait(&ring_full[pv % S], (pv / S) & 1);
+                if (!ok) break;
+                for (int j = 0; j < ns0 && ok; j++) {  // slot A has at least as many steps as B
 #pragma unroll
                     for (int x = 0; x < 2; x++) {
-                        if (x >= nx || !ok) continue;
-                        ok = wait(&p_full[x], steps[x] & 1);
+                        const int nsx = x ? ns1 : ns0;
+                        if (j >= nsx || !ok) continue;
+                        const int pv = pos + v_item(w, n, x, j);
+                        ok = wait(&ring_full[pv % S], (pv / S) & 1);
+                        ok = ok && wait(&p_full[x], steps[x] & 1);
                         if (ok && j == 0 && units[x] > 0) ok = wait(&o_empty[x], (units[x] - 1) & 1);
                         if (!ok) break;
                         steps[x]++;
                         tc_fence_after_sync();
                         issue_pv(x, pv % S, j > 0);
-                        if (last) {
+                        commit(&ring_empty[pv % S]);
+                        if (j == nsx - 1) {
                             commit(&o_full[x]);
                         } else {
-                            if (x == 0 && !wait(&ring_full[pk % S], (pk / S) & 1)) {
+                            const int pk = pos + k_item(w, n, x, j + 1);
+                            if (!wait(&ring_full[pk % S], (pk / S) & 1)) {
                                 ok = false;
                                 break;
                             }
                             tc_fence_after_sync();
                             issue_s(x, pk % S);
                             commit(&s_full[x]);
-                            if (j + 2 == n) commit(&q_empty[x]);  // the slot's last read of Q
+                            if (j + 2 == nsx) commit(&q_empty[x]);  // the slot's last read of Q
+                            commit(&ring_empty[pk % S]);
                         }
                     }
                     ok = __all_sync(0xffffffffu, ok && !*abort_flag);
@@ -622,12 +801,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (lane == 0) report(p, abort_flag, ST_MMA_WAIT);
                         break;
                     }
-                    commit(&ring_empty[pv % S]);
-                    if (!last) commit(&ring_empty[pk % S]);
                 }
 #pragma unroll
                 for (int x = 0; x < 2; x++)
-                    if (x < nx) units[x]++;
+                    if ((x ? ns1 : ns0) > 0) units[x]++;
             }
             // all issued tensor-core work is finished before the memory is released
             commit(drain);
@@ -641,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         int staged[2] = {0, 0};
         int k_unit = 0;
-        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, k_unit++) {
+        for (int u = blockIdx.x; u < p.n_items && ok; u += gridDim.x, k_unit++) {
             const int buf = k_unit & 1;
             ok = __all_sync(0xffffffffu, mbar_wait(&info_full[buf], (k_unit >> 1) & 1, lim));
             if (!ok) break;
@@ -649,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int pos = unit_pos[buf];
             mbar_arrive(&info_empty[buf]);
             const Unit w = decode_unit(p, u);
-            const int nx = w.valid[1] ? 2 : 1;
+            const int nx = o_slots(w);  // a split unit's O is slot A's tile
             if (n == 0) continue;
 #pragma unroll
             for (int x = 0; x < 2; x++) {
@@ -686,9 +863,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cols = max(p.sinks, p.n_global);
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
         int steps = 0, units = 0;
+        int units_b = 0;   // slot A only: completed phases of o_full[1] (slot B's last PV of a unit)
+        int k_split = 0;   // split units passed (phases of the max / sum hand-off)
         bool ok = true;
         int k_unit = 0;  // units of this CTA so far: ring entry k_unit & 1
-        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, k_unit++) {
+        for (int u = blockIdx.x; u < p.n_items && ok; u += gridDim.x, k_unit++) {
             const int buf = k_unit & 1;
             ok = __all_sync(0xffffffffu, mbar_wait(&info_full[buf], (k_unit >> 1) & 1, lim) && !*abort_flag);
             if (!ok) break;
@@ -704,8 +883,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_all = q < p.n_global;
             float m_ref = -INFINITY;  // running max, log2 units of the scaled score
             float l_sum = 0.f;
-            for (int j = 0; j < n; j++) {
-                const uint32_t e = list[j];
+            const int n_self = slot_steps(w, n, x);
+            const int n_b = slot_steps(w, n, 1);
+            const uint16_t* slot_list = list + slot_entry(w, n, x, 0);
+            for (int j = 0; j < n_self; j++) {
+                const uint32_t e = slot_list[j];
                 const int kv = static_cast<int>(e & 0x3fffu);
                 const int kv0 = kv * BN;
                 const bool masked = !((e >> (14 + x)) & 1u) || kv0 + BN > p.N;
@@ -783,8 +965,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
                 const uint64_t neg_m = f2_pack(-m_use, -m_use);
 
-                // p = 2^(s * scale_log2 - m): 5 of every 8 pairs on the MUFU unit,
-                // 3 on the FMA pipe (exp2_poly), packed two lanes at a time.
+                // p = 2^(s * scale_log2 - m): 6 of every 8 pairs on the MUFU unit,
+                // 2 on the FMA pipe (exp2_poly), packed two lanes at a time.
                 uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
                 for (int c = 0; c < BN; c += 64) {
@@ -793,7 +975,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 32; i++) {
                         const uint64_t x2 = f2_fma(f2_pack(s[c + 2 * i], s[c + 2 * i + 1]), scale2, neg_m);
                         float p0, p1;
-                        if (((c / 2 + i) & 7) < 3) {
+                        if (((c / 2 + i) & 7) < 2) {
                             exp2_poly_x2(x2, p0, p1);
                         } else {
                             float x0, x1;
@@ -833,55 +1015,147 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&p_full[x]);
                 steps++;
             }
-            // first ring item of this slot's O tile
-            const int o_item = unit_pos[buf] + 2 * n + x * C::kOBlocks;
+            // first ring item of this slot's O tile (slot A's for a split unit)
+            const int o_item = unit_pos[buf] + 2 * n + (w.split ? 0 : x * C::kOBlocks);
             mbar_arrive(&info_empty[buf]);  // this lane has read the unit's steps
             if (!ok) break;
 
             // ---------------------------------------------------------------- epilogue
-            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-            if (n > 0) {
-                // the ring stage granted for this row's block of BN rows of O
-                const int item = o_item + row / BN;
-                ok = mbar_wait(&o_full[x], units & 1, lim);
-                ok = ok && mbar_wait(&ring_full[item % S], (item / S) & 1, lim);
+            if (__builtin_expect(!w.split, 1)) {
+                if (x == 0 && n_b > 0) units_b++;
+                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+                if (n > 0) {
+                    // the ring stage granted for this row's block of BN rows of O
+                    const int item = o_item + row / BN;
+                    ok = mbar_wait(&o_full[x], units & 1, lim);
+                    ok = ok && mbar_wait(&ring_full[item % S], (item / S) & 1, lim);
+                    ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+                    if (!ok) break;
+                    uint32_t o[D / 32][32];
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int c = 0; c < D / 32; c++) tmem_ld_32x32b_x32(tmem_addr(tmem, lane_base, col_o + 32 * c), o[c]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < D / 32; c++) reg_fence(o[c]);
+                    tc_fence_before_sync();
+                    mbar_arrive(&o_empty[x]);  // O_X may now be overwritten by the next unit
+                    units++;
+                    // Stage the bf16 row in the granted stage, in the 128-byte-swizzled
+                    // layout of a K tile (the O map's box); the store warp writes it out.
+                    uint8_t* stg = ring + (item % S) * C::kKVBytes;
+                    const int r = row % BN;
+#pragma unroll
+                    for (int c = 0; c < D; c += 8) {
+                        uint4 v;
+                        const uint32_t* oc = &o[c / 32][c % 32];
+                        v.x = pack_bf16x2(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv);
+                        v.y = pack_bf16x2(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv);
+                        v.z = pack_bf16x2(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
+                        v.w = pack_bf16x2(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
+                        const int chunk = (c % 64) / 8;
+                        *reinterpret_cast<uint4*>(stg + (c / 64) * C::kKVPanel + r * 128 + ((chunk ^ (r & 7)) * 16)) = v;
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(&o_staged[x]);
+                } else if (q < p.N) {
+                    // no live tile for this unit: O = 0 (the slot's Q was never loaded)
+                    uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D);
+#pragma unroll
+                    for (int c = 0; c < D; c += 8) dst[c / 8] = make_uint4(0u, 0u, 0u, 0u);
+                }
+                if (q < p.N)
+                    p.LSE[orow] = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
+            } else if (x == 1) {
+                // split unit, second half: hand this row's max and sum to slot A
+                ok = mbar_wait(mlx_empty, (k_split & 1) ^ 1, lim);
                 ok = __all_sync(0xffffffffu, ok && !*abort_flag);
                 if (!ok) break;
-                uint32_t o[D / 32][32];
-                tc_fence_after_sync();
+                mlx[row] = m_ref;
+                mlx[kBM + row] = l_sum;
+                mbar_arrive(mlx_full);
+                k_split++;
+                if (n_self > 0) units++;  // o_full[1] completed; slot A reads O_B and frees it
+            } else {
+                // split unit, first half: merge both halves of the row
+                ok = mbar_wait(mlx_full, k_split & 1, lim);
+                ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+                if (!ok) break;
+                const float m_b = mlx[row];
+                const float l_b = mlx[kBM + row];
+                mbar_arrive(mlx_empty);
+                k_split++;
+                const float mm = fmaxf(m_ref, m_b);
+                const float wa = (n_self > 0 && m_ref != -INFINITY) ? ex2_approx(m_ref - mm) : 0.f;
+                const float wb = (n_b > 0 && m_b != -INFINITY) ? ex2_approx(m_b - mm) : 0.f;
+                const float lt = l_sum * wa + l_b * wb;
+                const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                const float fa = wa * inv, fb = wb * inv;
+                if (n > 0) {
+                    const int item = o_item + row / BN;
+                    ok = n_self == 0 || mbar_wait(&o_full[0], units & 1, lim);
+                    ok = ok && (n_b == 0 || mbar_wait(&o_full[1], units_b & 1, lim));
+                    ok = ok && mbar_wait(&ring_full[item % S], (item / S) & 1, lim);
+                    ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    uint8_t* stg = ring + (item % S) * C::kKVBytes;
+                    const int r = row % BN;
+                    const uint32_t col_a = static_cast<uint32_t>(2 * BN);
+                    const uint32_t col_b = static_cast<uint32_t>(2 * BN + D);
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 32) {  // one 32-column chunk of both halves at a time
+                        uint32_t oa[32], ob[32];
+                        // both halves are read even when one has no step (its columns then
+                        // hold a stale tile, replaced by zeros below): loads under a branch
+                        // cost the softmax warps registers in their main loop
+                        tmem_ld_32x32b_x32(tmem_addr(tmem, lane_base, col_a + c0), oa);
+                        tmem_ld_32x32b_x32(tmem_addr(tmem, lane_base, col_b + c0), ob);
+                        tmem_wait_ld();
+                        reg_fence(oa);
+                        reg_fence(ob);
+                        if (n_self == 0) {
 #pragma unroll
-                for (int c = 0; c < D / 32; c++) tmem_ld_32x32b_x32(tmem_addr(tmem, lane_base, col_o + 32 * c), o[c]);
-                tmem_wait_ld();
+                            for (int i = 0; i < 32; i++) oa[i] = 0u;
+                        }
+                        if (n_b == 0) {
 #pragma unroll
-                for (int c = 0; c < D / 32; c++) reg_fence(o[c]);
-                tc_fence_before_sync();
-                mbar_arrive(&o_empty[x]);  // O_X may now be overwritten by the next unit
-                units++;
-                // Stage the bf16 row in the granted stage, in the 128-byte-swizzled
-                // layout of a K tile (the O map's box); the store warp writes it out.
-                uint8_t* stg = ring + (item % S) * C::kKVBytes;
-                const int r = row % BN;
+                            for (int i = 0; i < 32; i++) ob[i] = 0u;
+                        }
 #pragma unroll
-                for (int c = 0; c < D; c += 8) {
-                    uint4 v;
-                    const uint32_t* oc = &o[c / 32][c % 32];
-                    v.x = pack_bf16x2(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv);
-                    v.y = pack_bf16x2(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv);
-                    v.z = pack_bf16x2(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
-                    v.w = pack_bf16x2(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
-                    const int chunk = (c % 64) / 8;
-                    *reinterpret_cast<uint4*>(stg + (c / 64) * C::kKVPanel + r * 128 + ((chunk ^ (r & 7)) * 16)) = v;
+                        for (int c = 0; c < 32; c += 8) {
+                            float f[8];
+#pragma unroll
+                            for (int i = 0; i < 8; i++)
+                                f[i] = __uint_as_float(oa[c + i]) * fa + __uint_as_float(ob[c + i]) * fb;
+                            uint4 v;
+                            v.x = pack_bf16x2(f[0], f[1]);
+                            v.y = pack_bf16x2(f[2], f[3]);
+                            v.z = pack_bf16x2(f[4], f[5]);
+                            v.w = pack_bf16x2(f[6], f[7]);
+                            const int gc = c0 + c;  // column of O
+                            const int chunk = (gc % 64) / 8;
+                            *reinterpret_cast<uint4*>(stg + (gc / 64) * C::kKVPanel + r * 128 + ((chunk ^ (r & 7)) * 16)) = v;
+                        }
+                    }
+                    tc_fence_before_sync();
+                    if (n_self > 0) {
+                        mbar_arrive(&o_empty[0]);
+                        units++;
+                    }
+                    if (n_b > 0) {
+                        mbar_arrive(&o_empty[1]);  // slot A's 128 threads stand in for slot B's
+                        units_b++;
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(&o_staged[0]);
+                } else if (q < p.N) {
+                    uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D);
+#pragma unroll
+                    for (int c = 0; c < D; c += 8) dst[c / 8] = make_uint4(0u, 0u, 0u, 0u);
                 }
-                fence_proxy_async_smem();
-                mbar_arrive(&o_staged[x]);
-            } else if (q < p.N) {
-                // no live tile for this unit: O = 0 (the slot's Q was never loaded)
-                uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D);
-#pragma unroll
-                for (int c = 0; c < D; c += 8) dst[c / 8] = make_uint4(0u, 0u, 0u, 0u);
+                if (q < p.N) p.LSE[orow] = lt > 0.f ? (mm + log2f(lt)) * 0.69314718055994530942f : -INFINITY;
             }
-            if (q < p.N)
-                p.LSE[orow] = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
         }
         if (!ok) report(p, abort_flag, ST_SOFTMAX_WAIT);
     }

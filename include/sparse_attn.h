@@ -152,8 +152,12 @@ int sparse_attn_check_device(void* stream);
 /*
  * Test hook.  flags: bit 0 makes the next forward launches skip the Q tile
  * load, so the kernel's bounded waits expire and it reports
- * SA_ERR_DEVICE_TIMEOUT instead of computing.  timeout_cycles bounds every
- * wait in SM clock cycles (<= 0 restores the default, about one second).
+ * SA_ERR_DEVICE_TIMEOUT instead of computing.  Bit 1 makes sparse_attn_fwd
+ * split every work unit (each query tile's kv list walked in two halves that
+ * are merged at the end), the path the kernel otherwise takes only for the
+ * last, partial round of units; results agree within rounding.
+ * timeout_cycles bounds every wait in SM clock cycles (<= 0 restores the
+ * default, about one second).
  */
 int sparse_attn_set_debug(int32_t flags, int64_t timeout_cycles);
 

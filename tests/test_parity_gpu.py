@@ -67,7 +67,26 @@ SMALL = [
     (1, 1, 1, 1, 64, sa.Pattern(window=5), 64),                          # N = 1
     (1, 2, 2, 300, 128, sa.Pattern(window=-1, stride=1), 128),           # stride 1 = dense
     (1, 2, 2, 1100, 128, sa.Pattern(window=257, sinks=130), 64),         # sinks wider than a tile
+    (2, 3, 3, 700, 128, sa.Pattern(window=200, sinks=4), 128),           # odd head count: a one-slot unit
+    (1, 4, 4, 1536, 128, sa.Pattern(window=1024, sinks=4), 128),         # head pairs, own K/V per slot
+    (3, 1, 1, 900, 64, sa.Pattern(window=256, sinks=4), 64),             # one head, batched: q-tile pairs
 ]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"B{c[0]}H{c[1]}/{c[2]}N{c[3]}D{c[4]}b{c[6]}-{c[5]}")
+def test_small_full_parity_split_units(case):
+    """Every unit split: each query tile's kv list walked as two halves by the
+    two slots and merged at the end (the path of a partial last round)."""
+    B, Hq, Hkv, N, D, p, block = case
+    q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=N + D + 1)
+    scale = 1 / math.sqrt(D)
+    sa.set_debug(sa.DEBUG_SPLIT_ALL)
+    try:
+        O, LSE = run_gpu(q, k, v, p, block, scale)
+    finally:
+        sa.set_debug(0)
+    Oref, LSEref = oracle.attention(q, k, v, opattern(p), scale)
+    compare(O, LSE, Oref, LSEref)
 
 
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: f"B{c[0]}H{c[1]}/{c[2]}N{c[3]}D{c[4]}b{c[6]}-{c[5]}")
