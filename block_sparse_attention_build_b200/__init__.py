@@ -40,7 +40,7 @@ EXPORTED = (
     "sparse_attn_num_tiles", "sparse_attn_build_block_mask", "sparse_attn_count_pairs",
     "sparse_attn_fwd", "sparse_attn_fwd_host", "sparse_attn_fwd_host_workspace",
     "sparse_attn_check_device", "sparse_attn_set_debug", "sparse_attn_status_string",
-    "sparse_attn_version", "sparse_attn_fwd_noalloc",
+    "sparse_attn_version", "sparse_attn_fwd_noalloc", "sparse_attn_fwd_heads",
 )
 
 
@@ -81,6 +81,8 @@ def _load() -> ctypes.CDLL:
     L.sparse_attn_fwd_host.argtypes = [vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp]
     L.sparse_attn_fwd_host_workspace.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
     L.sparse_attn_fwd_noalloc.argtypes = [vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp]
+    L.sparse_attn_fwd_heads.argtypes = [vp, vp, vp, M, P, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32), S,
+                                        ctypes.c_float, vp, vp, vp]
     L.sparse_attn_check_device.argtypes = [vp]
     L.sparse_attn_set_debug.argtypes = [ctypes.c_int32, ctypes.c_int64]
     L.sparse_attn_status_string.argtypes = [ctypes.c_int]
@@ -89,7 +91,7 @@ def _load() -> ctypes.CDLL:
     L.sparse_attn_version.restype = ctypes.c_int32
     for name in ("sparse_attn_build_block_mask", "sparse_attn_count_pairs", "sparse_attn_fwd",
                  "sparse_attn_fwd_host", "sparse_attn_fwd_host_workspace", "sparse_attn_check_device",
-                 "sparse_attn_set_debug", "sparse_attn_fwd_noalloc"):
+                 "sparse_attn_set_debug", "sparse_attn_fwd_noalloc", "sparse_attn_fwd_heads"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -208,6 +210,41 @@ def fwd(q, k, v, mask: BlockMask, pattern: Pattern, scale: float | None = None, 
         _check(lib.sparse_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(mask._c()),
                                    ctypes.byref(pattern._c()), ctypes.byref(shape), float(scale),
                                    out.data_ptr(), lse.data_ptr(), st), "sparse_attn_fwd")
+    return out, lse
+
+
+def fwd_heads(q, k, v, masks, patterns, head_pattern, scale: float | None = None, out=None, lse=None,
+              stream=None):
+    """Forward pass with a pattern per query head: head h attends under
+    ``patterns[head_pattern[h]]`` with the device block mask ``masks[head_pattern[h]]``.
+
+    ``masks`` and ``patterns`` are sequences of equal length (1..8);
+    ``head_pattern`` holds Hq ints.  Otherwise as ``fwd``.
+    """
+    import torch
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError("q, k, v must be contiguous bf16 CUDA tensors")
+    if len(masks) != len(patterns):
+        raise ValueError("one block mask per pattern")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    n = len(patterns)
+    cmasks = (_BlockMask * max(n, 1))(*[m._c() for m in masks])
+    cpats = (_Pattern * max(n, 1))(*[p_._c() for p_ in patterns])
+    heads = (ctypes.c_int32 * max(len(head_pattern), 1))(*[int(h) for h in head_pattern])
+    shape = _Shape(B, Hq, Hkv, N, D)
+    with torch.cuda.device(q.device):
+        st = _stream_handle(stream, q.device)
+        _check(lib.sparse_attn_fwd_heads(q.data_ptr(), k.data_ptr(), v.data_ptr(), cmasks, cpats, n, heads,
+                                         ctypes.byref(shape), float(scale), out.data_ptr(), lse.data_ptr(), st),
+               "sparse_attn_fwd_heads")
     return out, lse
 
 

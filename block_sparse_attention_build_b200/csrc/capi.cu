@@ -53,12 +53,12 @@ int sm_count()
     return counts[dev];
 }
 
-template <int D, int BN>
-int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo, const FwdParams& p, int grid,
-           cudaStream_t stream)
+template <int D, int BN, bool MULTI>
+int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo, const FwdParams& p,
+           const HeadPatterns& hp, int grid, cudaStream_t stream)
 {
     using C = FwdCfg<D, BN>;
-    auto kern = fwd_kernel<D, BN>;
+    auto kern = fwd_kernel<D, BN, MULTI>;
     static bool attr_set[kMaxDevices] = {};  // per instantiation and device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SA_ERR_CUDA;
@@ -71,34 +71,61 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, 
         if (fa.numRegs * kThreads < kRegSplitTotal) return SA_ERR_UNSUPPORTED;
         attr_set[dev] = true;
     }
-    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p, hp);
     return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
-}  // namespace
-}  // namespace sa
-
-extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, const sa_block_mask* mask,
-                               const sa_pattern* pattern, const sa_shape* shape, float scale, void* O, float* LSE,
-                               void* stream)
+template <bool MULTI>
+int launch_any(int D, int block, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               const CUtensorMap& mo, const FwdParams& p, const HeadPatterns& hp, int g, cudaStream_t st)
 {
-    using namespace sa;
-    if (!mask || !pattern || !shape) return SA_ERR_INVALID_ARG;
+    if (D == 128 && block == 128) return launch<128, 128, MULTI>(mq, mk, mv, mo, p, hp, g, st);
+    if (D == 64 && block == 128) return launch<64, 128, MULTI>(mq, mk, mv, mo, p, hp, g, st);
+    if (D == 128 && block == 64) return launch<128, 64, MULTI>(mq, mk, mv, mo, p, hp, g, st);
+    return launch<64, 64, MULTI>(mq, mk, mv, mo, p, hp, g, st);
+}
+
+bool pattern_ok(const sa_pattern& pt)
+{
+    return pt.window >= -1 && pt.sinks >= 0 && pt.stride >= 0 && pt.n_global >= 0;
+}
+
+// The forward pass behind sparse_attn_fwd (one pattern: n_patterns = 1,
+// head_pattern = null) and sparse_attn_fwd_heads (a pattern per query head).
+int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* masks, const sa_pattern* patterns,
+             int32_t n_patterns, const int32_t* head_pattern, const sa_shape* shape, float scale, void* O, float* LSE,
+             void* stream)
+{
+    if (!masks || !patterns || !shape) return SA_ERR_INVALID_ARG;
+    const bool multi = head_pattern != nullptr;
+    if (n_patterns < 1 || n_patterns > (multi ? kMaxPatterns : 1)) return SA_ERR_INVALID_ARG;
+    const sa_block_mask* mask = &masks[0];
+    const sa_pattern* pattern = &patterns[0];
     const sa_shape s = *shape;
     if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
-    if (pattern->causal != 1) return SA_ERR_UNSUPPORTED;
-    if (pattern->window < -1 || pattern->sinks < 0 || pattern->stride < 0 || pattern->n_global < 0)
-        return SA_ERR_INVALID_ARG;
+    for (int i = 0; i < n_patterns; i++) {
+        if (patterns[i].causal != 1) return SA_ERR_UNSUPPORTED;
+        if (!pattern_ok(patterns[i])) return SA_ERR_INVALID_ARG;
+    }
     if (s.D != 64 && s.D != 128) return SA_ERR_UNSUPPORTED;
     if (mask->block != 64 && mask->block != 128) return SA_ERR_UNSUPPORTED;
+    for (int i = 1; i < n_patterns; i++)
+        if (masks[i].block != mask->block) return SA_ERR_MASK_MISMATCH;
+    if (multi && s.Hq > kMaxHeadsMulti) return SA_ERR_UNSUPPORTED;
+    if (multi)
+        for (int h = 0; h < s.Hq; h++)
+            if (head_pattern[h] < 0 || head_pattern[h] >= n_patterns) return SA_ERR_INVALID_ARG;
     if (s.B == 0 || s.Hq == 0 || s.N == 0) return SA_OK;  // nothing to compute
     if (s.Hkv <= 0 || s.Hq % s.Hkv != 0) return SA_ERR_UNSUPPORTED;
     const int64_t T = (int64_t(s.N) + mask->block - 1) / mask->block;
-    if (mask->n_q_tiles != T || mask->n_kv_tiles != T) return SA_ERR_MASK_MISMATCH;
+    for (int i = 0; i < n_patterns; i++) {
+        if (masks[i].n_q_tiles != T || masks[i].n_kv_tiles != T) return SA_ERR_MASK_MISMATCH;
+        if (!masks[i].kv_count || !masks[i].kv_index || !masks[i].kv_full) return SA_ERR_INVALID_ARG;
+    }
+
     if (T > kMaxTiles) return SA_ERR_UNSUPPORTED;
-    if (!Q || !K || !V || !O || !LSE || !mask->kv_count || !mask->kv_index || !mask->kv_full)
-        return SA_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !O || !LSE) return SA_ERR_INVALID_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
         return SA_ERR_MISALIGNED;
     const int64_t n_qtiles = (int64_t(s.N) + kBM - 1) / kBM;
@@ -159,10 +186,37 @@ extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, cons
     p.debug_flags = debug_flags;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int g = static_cast<int>(grid);
-    if (s.D == 128 && mask->block == 128) return launch<128, 128>(mq, mk, mv, mo, p, g, st);
-    if (s.D == 64 && mask->block == 128) return launch<64, 128>(mq, mk, mv, mo, p, g, st);
-    if (s.D == 128 && mask->block == 64) return launch<128, 64>(mq, mk, mv, mo, p, g, st);
-    return launch<64, 64>(mq, mk, mv, mo, p, g, st);
+    HeadPatterns hp{};
+    if (!multi) return launch_any<false>(s.D, mask->block, mq, mk, mv, mo, p, hp, g, st);
+    for (int i = 0; i < n_patterns; i++) {
+        hp.pat[i].kv_count = masks[i].kv_count;
+        hp.pat[i].kv_index = masks[i].kv_index;
+        hp.pat[i].kv_full = masks[i].kv_full;
+        hp.pat[i].window = patterns[i].window;
+        hp.pat[i].sinks = patterns[i].sinks;
+        hp.pat[i].stride = patterns[i].stride;
+        hp.pat[i].n_global = patterns[i].n_global;
+    }
+    for (int h = 0; h < s.Hq; h++) hp.head[h] = static_cast<uint8_t>(head_pattern[h]);
+    return launch_any<true>(s.D, mask->block, mq, mk, mv, mo, p, hp, g, st);
+}
+
+}  // namespace
+}  // namespace sa
+
+extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, const sa_block_mask* mask,
+                               const sa_pattern* pattern, const sa_shape* shape, float scale, void* O, float* LSE,
+                               void* stream)
+{
+    return sa::fwd_impl(Q, K, V, mask, pattern, 1, nullptr, shape, scale, O, LSE, stream);
+}
+
+extern "C" int sparse_attn_fwd_heads(const void* Q, const void* K, const void* V, const sa_block_mask* masks,
+                                     const sa_pattern* patterns, int32_t n_patterns, const int32_t* head_pattern,
+                                     const sa_shape* shape, float scale, void* O, float* LSE, void* stream)
+{
+    if (!head_pattern) return SA_ERR_INVALID_ARG;
+    return sa::fwd_impl(Q, K, V, masks, patterns, n_patterns, head_pattern, shape, scale, O, LSE, stream);
 }
 
 extern "C" int sparse_attn_fwd_host_workspace(const sa_shape* shape, size_t* bytes)

@@ -57,7 +57,7 @@ int launch(int dev, int which, const CUtensorMap& mq, const CUtensorMap& mk, con
            const CUtensorMap& mo, const FwdParams& p, int grid, cudaStream_t stream)
 {
     using C = FwdCfg<D, BN>;
-    auto kern = fwd_kernel<D, BN>;
+    auto kern = fwd_kernel<D, BN, false>;
     if (!g_attr[dev][which]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
             return SA_ERR_CUDA;
@@ -67,7 +67,8 @@ int launch(int dev, int which, const CUtensorMap& mq, const CUtensorMap& mk, con
         if (fa.numRegs * kThreads < kRegSplitTotal) return SA_ERR_UNSUPPORTED;
         g_attr[dev][which] = true;
     }
-    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+    const HeadPatterns hp{};  // one pattern: the per-head table is not read
+    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p, hp);
     return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 

@@ -93,6 +93,24 @@ struct FwdParams {
     int32_t debug_flags;      // bit 0: skip the first Q load (test hook)
 };
 
+// Per-head patterns: each query head follows one of up to kMaxPatterns
+// compiled patterns (its block mask and the rule parameters its partial tiles
+// are masked with).  Different heads of a layer may carry different patterns
+// ("Sparse-трансформеры" page, section "Комбинация — норма, а не
+// исключение").  Used by the kernels instantiated with MULTI = true.
+constexpr int kMaxPatterns = 8;
+constexpr int kMaxHeadsMulti = 256;
+struct PatternRef {
+    const int32_t* kv_count;  // [T]
+    const int32_t* kv_index;  // [T * T]
+    const uint8_t* kv_full;   // [T * T]
+    int32_t window, sinks, stride, n_global;
+};
+struct HeadPatterns {
+    PatternRef pat[kMaxPatterns];
+    uint8_t head[kMaxHeadsMulti];  // pattern of each query head
+};
+
 enum : int32_t {
     ST_Q_WAIT = 1,
     ST_PRODUCER_WAIT = 2,
@@ -266,9 +284,28 @@ __device__ __forceinline__ uint32_t bits_between(int lo, int hi)
 // coalesced loads into shared-memory bitmaps (bm: live, then one full bitmap
 // per row, kMaxTiles / 32 words each), then a warp prefix scan emits the set
 // bits in order.  Returns the number of steps (the same in every lane).
-__device__ __forceinline__ int build_unit_list(const FwdParams& p, const Unit& w, int BN, uint16_t* list,
-                                               uint32_t* bm, int lane)
+template <bool MULTI>
+__device__ __forceinline__ int build_unit_list(const FwdParams& p, const HeadPatterns& hp, const Unit& w, int BN,
+                                               uint16_t* list, uint32_t* bm, int lane)
 {
+    // the block mask each slot's rows come from
+    const int32_t* cnt_of[2];
+    const int32_t* idx_of[2];
+    const uint8_t* full_of[2];
+#pragma unroll
+    for (int x = 0; x < 2; x++) {
+        if constexpr (MULTI) {
+            // an absent slot B may name head Hq (one past the table): use slot A's
+            const PatternRef& pr = hp.pat[hp.head[(x && w.valid[1]) ? w.hq[1] : w.hq[0]]];
+            cnt_of[x] = pr.kv_count;
+            idx_of[x] = pr.kv_index;
+            full_of[x] = pr.kv_full;
+        } else {
+            cnt_of[x] = p.kv_count;
+            idx_of[x] = p.kv_index;
+            full_of[x] = p.kv_full;
+        }
+    }
     constexpr int W = kMaxTiles / 32;
     const int rows_per = kBM / BN;
     const int words = (p.T + 31) / 32;
@@ -283,9 +320,9 @@ __device__ __forceinline__ int build_unit_list(const FwdParams& p, const Unit& w
         exists[r] = w.valid[x] && k < rows_per && row[r] < p.T;
         const int64_t off = static_cast<int64_t>(exists[r] ? row[r] : 0) * p.T + lane;
         const bool in_row = exists[r] && lane < p.T;
-        cnt[r] = exists[r] ? __ldg(&p.kv_count[row[r]]) : 0;
-        kv0[r] = in_row ? __ldg(&p.kv_index[off]) : -1;
-        full0[r] = in_row ? __ldg(&p.kv_full[off]) != 0 : false;
+        cnt[r] = exists[r] ? __ldg(&cnt_of[x][row[r]]) : 0;
+        kv0[r] = in_row ? __ldg(&idx_of[x][off]) : -1;
+        full0[r] = in_row ? __ldg(&full_of[x][off]) != 0 : false;
     }
 #pragma unroll
     for (int r = 0; r < 4; r++) cnt[r] = min(max(cnt[r], 0), p.T);  // clamp a corrupt count: never read past the row
@@ -298,8 +335,8 @@ __device__ __forceinline__ int build_unit_list(const FwdParams& p, const Unit& w
 #pragma unroll
     for (int r = 0; r < 4; r++) {
         if (!exists[r]) continue;
-        const int32_t* idx = p.kv_index + static_cast<int64_t>(row[r]) * p.T;
-        const uint8_t* fl = p.kv_full + static_cast<int64_t>(row[r]) * p.T;
+        const int32_t* idx = idx_of[r / 2] + static_cast<int64_t>(row[r]) * p.T;
+        const uint8_t* fl = full_of[r / 2] + static_cast<int64_t>(row[r]) * p.T;
         for (int e = lane; e < cnt[r]; e += 32) {
             const int kv = e < 32 ? kv0[r] : __ldg(&idx[e]);
             const bool full = e < 32 ? full0[r] : __ldg(&fl[e]) != 0;
@@ -394,10 +431,11 @@ __device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& p0, float& p1)
     p1 = x1 < -125.f ? 0.f : __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
-template <int D, int BN>
+template <int D, int BN, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const FwdParams p)
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const FwdParams p,
+               const __grid_constant__ HeadPatterns hp)
 {
     using C = FwdCfg<D, BN>;
     constexpr int S = C::kStages;
@@ -507,7 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     dead = true;
                     return 0;
                 }
-                const int n = build_unit_list(p, decode_unit(p, u), BN, unit_list + buf * kMaxTiles, bitmaps, lane);
+                const int n = build_unit_list<MULTI>(p, hp, decode_unit(p, u), BN, unit_list + buf * kMaxTiles,
+                                                     bitmaps, lane);
                 if (lane == 0) {
                     unit_n[buf] = n;
                     unit_pos[buf] = first_pos;
@@ -860,7 +899,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32);
         const uint32_t col_s = static_cast<uint32_t>(x * BN);
         const uint32_t col_o = static_cast<uint32_t>(2 * BN + x * D);
-        const int cols = max(p.sinks, p.n_global);
+        int cols = max(p.sinks, p.n_global);
+        int pw = p.window, ps = p.stride, pg = p.n_global;  // this slot's pattern (per unit when MULTI)
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
         int steps = 0, units = 0;
         int units_b = 0;   // slot A only: completed phases of o_full[1] (slot B's last PV of a unit)
@@ -880,7 +920,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int q = (x == 0 ? w.qtile[0] : w.qtile[1]) * kBM + row;
             const int64_t orow = (static_cast<int64_t>(w.b) * p.Hq + (x == 0 ? w.hq[0] : w.hq[1])) * p.N + q;
-            const bool row_all = q < p.n_global;
+            if constexpr (MULTI) {
+                const PatternRef& pr = hp.pat[hp.head[x == 0 ? w.hq[0] : w.hq[1]]];
+                pw = pr.window;
+                ps = pr.stride;
+                pg = pr.n_global;
+                cols = max(pr.sinks, pr.n_global);
+            }
+            const bool row_all = q < pg;
             float m_ref = -INFINITY;  // running max, log2 units of the scaled score
             float l_sum = 0.f;
             const int n_self = slot_steps(w, n, x);
@@ -903,12 +950,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int w = 0; w < BN / 32; w++) {
                         const int base = 32 * w;
                         uint32_t m = bits_between(0, cols - 1 - kv0 - base);
-                        if (p.window >= 0) m |= bits_between(dq - p.window - base, 31);
-                        if (p.stride > 0) {
-                            int r0 = dq % p.stride;
-                            if (r0 < 0) r0 += p.stride;
-                            int h = r0 >= base ? r0 : r0 + ((base - r0 + p.stride - 1) / p.stride) * p.stride;
-                            for (; h < base + 32; h += p.stride) m |= 1u << (h - base);
+                        if (pw >= 0) m |= bits_between(dq - pw - base, 31);
+                        if (ps > 0) {
+                            int r0 = dq % ps;
+                            if (r0 < 0) r0 += ps;
+                            int h = r0 >= base ? r0 : r0 + ((base - r0 + ps - 1) / ps) * ps;
+                            for (; h < base + 32; h += ps) m |= 1u << (h - base);
                         }
                         if (row_all) m = 0xffffffffu;
                         allow[w] = m & bits_between(0, c_max - base);

@@ -139,6 +139,30 @@ int sparse_attn_fwd_host(const void* Q_host, const void* K_host, const void* V_h
                          const sa_pattern* pattern, const sa_shape* shape, float scale, void* O_host,
                          float* LSE_host, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Forward pass with a pattern per query head ("Sparse-трансформеры" page,
+ * section "Комбинация — норма, а не исключение": heads of one layer may carry
+ * different patterns, some local, some strided).  Query head h attends under
+ * patterns[head_pattern[h]], with the block mask masks[head_pattern[h]]
+ * compiled for it by sparse_attn_build_block_mask; a head's result is that of
+ * sparse_attn_fwd under its own pattern.
+ *
+ *   masks        [n_patterns] block masks in DEVICE memory, all for the same N
+ *                and block
+ *   patterns     [n_patterns] (host), each as for sparse_attn_fwd
+ *   n_patterns   1 .. 8
+ *   head_pattern [Hq] (host) pattern index of each query head; Hq <= 256
+ *   other arguments and layouts as sparse_attn_fwd; asynchronous on `stream`.
+ *
+ * Errors: SA_ERR_INVALID_ARG for a null argument, n_patterns out of range or
+ * an index outside [0, n_patterns); SA_ERR_MASK_MISMATCH when the masks differ
+ * in block or do not match N; SA_ERR_UNSUPPORTED for Hq > 256 and everything
+ * sparse_attn_fwd rejects.
+ */
+int sparse_attn_fwd_heads(const void* Q, const void* K, const void* V, const sa_block_mask* masks,
+                          const sa_pattern* patterns, int32_t n_patterns, const int32_t* head_pattern,
+                          const sa_shape* shape, float scale, void* O, float* LSE, void* stream);
+
 /* Device bytes sparse_attn_fwd_host needs for `shape`. */
 int sparse_attn_fwd_host_workspace(const sa_shape* shape, size_t* bytes);
 

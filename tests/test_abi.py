@@ -125,3 +125,34 @@ def test_fwd_argument_errors_without_gpu():
     ws = ctypes.c_size_t(0)
     assert sa.lib.sparse_attn_fwd_host_workspace(ctypes.byref(sa._Shape(1, 2, 1, 100, 64)), ctypes.byref(ws)) == 0
     assert ws.value >= 2 * (2 * 100 * 64 * 2) + 2 * (100 * 64 * 2) + 2 * 100 * 4
+
+
+def test_fwd_heads_argument_errors_without_gpu():
+    """Per-head entry point: checks that return before any CUDA call."""
+    p = sa.Pattern(window=8)._c()
+    p2 = sa.Pattern(window=4, stride=16)._c()
+    m = sa._BlockMask(1, 1, 128, 1, 1, 0, 16, 16, 16)
+    m64 = sa._BlockMask(2, 2, 64, 1, 1, 0, 16, 16, 16)
+    fake = 1 << 20  # never dereferenced: every case below fails validation first
+
+    def call(shape, heads, masks=(m, m), pats=(p, p2), n=None, ptr=fake):
+        n = len(pats) if n is None else n
+        cm = (sa._BlockMask * len(masks))(*masks)
+        cp = (sa._Pattern * len(pats))(*pats)
+        ch = (ctypes.c_int32 * max(len(heads), 1))(*heads)
+        return sa.lib.sparse_attn_fwd_heads(ptr, ptr, ptr, cm, cp, n, ch if heads is not None else None,
+                                            ctypes.byref(sa._Shape(*shape)), 0.125, ptr, ptr, None)
+
+    assert call((1, 2, 2, 100, 128), [0, 1], n=0) == sa.SA_ERR_INVALID_ARG          # no pattern
+    assert call((1, 2, 2, 100, 128), [0, 1], n=9) == sa.SA_ERR_INVALID_ARG          # more than 8
+    assert call((1, 2, 2, 100, 128), [0, 2]) == sa.SA_ERR_INVALID_ARG               # index out of range
+    assert call((1, 2, 2, 100, 128), [0, -1]) == sa.SA_ERR_INVALID_ARG
+    assert call((1, 2, 2, 100, 128), [0, 1], masks=(m, m64)) == sa.SA_ERR_MASK_MISMATCH  # blocks differ
+    assert call((1, 300, 300, 100, 128), [0] * 300) == sa.SA_ERR_UNSUPPORTED         # more than 256 heads
+    bad = sa.Pattern(window=8, causal=0)._c()
+    assert call((1, 2, 2, 100, 128), [0, 1], pats=(p, bad)) == sa.SA_ERR_UNSUPPORTED
+    assert call((1, 2, 2, 100, 128), [0, 1], ptr=fake + 8) == sa.SA_ERR_MISALIGNED
+    assert call((0, 2, 2, 100, 128), [0, 1]) == sa.SA_OK                             # nothing to compute
+    rc = sa.lib.sparse_attn_fwd_heads(fake, fake, fake, (sa._BlockMask * 1)(m), (sa._Pattern * 1)(p), 1, None,
+                                      ctypes.byref(sa._Shape(1, 2, 2, 100, 128)), 0.125, fake, fake, None)
+    assert rc == sa.SA_ERR_INVALID_ARG                                               # no head table

@@ -185,3 +185,62 @@ def test_device_timeout_is_reported_and_context_survives():
     O, LSE = run_gpu(q, k, v, p, 128, 1 / math.sqrt(D))
     Oref, LSEref = oracle.attention(q, k, v, opattern(p), 1 / math.sqrt(D))
     compare(O, LSE, Oref, LSEref)
+
+
+HEAD_CASES = [
+    # (B, Hq, Hkv, N, D, block, patterns, pattern index per query head)
+    (1, 4, 4, 1000, 128, 128,
+     [sa.Pattern(window=200, sinks=4), sa.Pattern(window=64, stride=128, n_global=16), sa.Pattern(window=-1, sinks=8)],
+     [0, 1, 2, 0]),
+    # two query heads of one kv group under different patterns (their unit's step list is a union)
+    (2, 4, 2, 777, 64, 64, [sa.Pattern(window=100, sinks=3), sa.Pattern(window=0, stride=37, n_global=5)], [0, 1, 1, 0]),
+    (1, 6, 2, 1300, 128, 128,
+     [sa.Pattern(window=300), sa.Pattern(window=1300), sa.Pattern(window=20, sinks=130)], [0, 1, 2, 2, 1, 0]),
+]
+
+
+def run_heads(q, k, v, patterns, heads, block, scale):
+    N = q.shape[2]
+    masks = [sa.build_block_mask(p, N, block).to_device("cuda") for p in patterns]
+    O, LSE = sa.fwd_heads(to_dev(q), to_dev(k), to_dev(v), masks, patterns, heads, scale=scale)
+    assert sa.check_device() == sa.SA_OK
+    return O.float().cpu().numpy(), LSE.cpu().numpy()
+
+
+def oracle_heads(q, k, v, patterns, heads, scale):
+    """Each query head by itself under its own pattern (heads are independent)."""
+    Hq, Hkv = q.shape[1], k.shape[1]
+    outs, lses = [], []
+    for h in range(Hq):
+        hk = h // (Hq // Hkv)
+        O, L = oracle.attention(np.ascontiguousarray(q[:, h:h + 1]), np.ascontiguousarray(k[:, hk:hk + 1]),
+                                np.ascontiguousarray(v[:, hk:hk + 1]), opattern(patterns[heads[h]]), scale)
+        outs.append(O)
+        lses.append(L)
+    return np.concatenate(outs, axis=1), np.concatenate(lses, axis=1)
+
+
+@pytest.mark.parametrize("split", [False, True], ids=["whole", "split"])
+@pytest.mark.parametrize("case", HEAD_CASES, ids=lambda c: f"B{c[0]}H{c[1]}/{c[2]}N{c[3]}D{c[4]}b{c[5]}")
+def test_per_head_patterns(case, split):
+    B, Hq, Hkv, N, D, block, patterns, heads = case
+    q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=N + 3)
+    scale = 1 / math.sqrt(D)
+    if split:
+        sa.set_debug(sa.DEBUG_SPLIT_ALL)
+    try:
+        O, LSE = run_heads(q, k, v, patterns, heads, block, scale)
+    finally:
+        sa.set_debug(0)
+    Oref, LSEref = oracle_heads(q, k, v, patterns, heads, scale)
+    compare(O, LSE, Oref, LSEref)
+
+
+def test_per_head_entry_with_one_pattern_equals_fwd():
+    B, Hq, Hkv, N, D = 1, 4, 2, 1500, 128
+    q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=11)
+    p = sa.Pattern(window=256, sinks=4)
+    scale = 1 / math.sqrt(D)
+    O1, L1 = run_heads(q, k, v, [p], [0] * Hq, 128, scale)
+    O2, L2 = run_gpu(q, k, v, p, 128, scale)
+    assert np.array_equal(O1, O2) and np.array_equal(L1, L2)
