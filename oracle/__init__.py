@@ -1,4 +1,4 @@
-"""CPU oracle for block-sparse causal attention forward (test infrastructure).
+"""CPU oracle for block-sparse causal attention, forward and backward (test infrastructure).
 
 Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The product path (the CUDA library and
@@ -80,6 +80,11 @@ class Oracle:
                                        ctypes.c_void_p, ctypes.c_int64,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
         L.oracle_attention.restype = ctypes.c_int
+        d = ctypes.c_void_p
+        L.oracle_attention_bwd.argtypes = [d, d, d, d, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_int64, ctypes.c_int64, P, ctypes.c_double,
+                                           d, d, d, d, d, ctypes.c_int32]
+        L.oracle_attention_bwd.restype = ctypes.c_int
         L.oracle_max_threads.argtypes = []
         L.oracle_max_threads.restype = ctypes.c_int
         self.L = L
@@ -138,6 +143,36 @@ class Oracle:
             raise ValueError("bad attention arguments")
         return O, LSE
 
+    def attention_bwd(self, q: np.ndarray, k: np.ndarray, v: np.ndarray, do: np.ndarray, p: Pattern,
+                      scale: float, n_threads: int = 0):
+        """fp64 gradients by definition.
+
+        q, do: [B, Hq, N, D]; k, v: [B, Hkv, N, D]; either uint16 bf16 bit
+        patterns (widened exactly) or float64.  Returns (O, LSE, dQ, dK, dV),
+        float64, shapes as the inputs (LSE [B, Hq, N]).
+        """
+        def wide(a):
+            if a.dtype == np.uint16:
+                return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            if a.dtype != np.float64:
+                raise TypeError("inputs must be uint16 (bf16 bit patterns) or float64")
+            return np.ascontiguousarray(a)
+        q, k, v, do = (wide(np.ascontiguousarray(a)) for a in (q, k, v, do))
+        B, Hq, N, D = q.shape
+        Hkv = k.shape[1]
+        if k.shape != (B, Hkv, N, D) or v.shape != k.shape or do.shape != q.shape:
+            raise ValueError("shape mismatch")
+        O = np.empty_like(q)
+        LSE = np.empty((B, Hq, N), dtype=np.float64)
+        dQ, dK, dV = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+        rc = self.L.oracle_attention_bwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, do.ctypes.data,
+                                         B, Hq, Hkv, N, D, ctypes.byref(p.c()), float(scale),
+                                         O.ctypes.data, LSE.ctypes.data, dQ.ctypes.data, dK.ctypes.data,
+                                         dV.ctypes.data, int(n_threads))
+        if rc != 0:
+            raise ValueError("bad attention_bwd arguments")
+        return O, LSE, dQ, dK, dV
+
     def max_threads(self) -> int:
         return int(self.L.oracle_max_threads())
 
@@ -166,6 +201,10 @@ def block_mask(p: Pattern, N: int, block: int):
 
 def attention(q, k, v, p: Pattern, scale: float, rows=None, n_threads: int = 0):
     return default().attention(q, k, v, p, scale, rows=rows, n_threads=n_threads)
+
+
+def attention_bwd(q, k, v, do, p: Pattern, scale: float, n_threads: int = 0):
+    return default().attention_bwd(q, k, v, do, p, scale, n_threads=n_threads)
 
 
 def max_threads() -> int:

@@ -35,6 +35,12 @@
  *
  *  - oracle_count_pairs: the number of allowed pairs, one by one.
  *
+ *  - oracle_attention_bwd: the gradients of that same function (the
+ *    masked_attention prototype of "Как это выглядит в коде") with respect to
+ *    Q, K and V for an upstream gradient dO.  The pages print no backward
+ *    pass; this is the chain rule through the softmax over each query's
+ *    allowed set, written out term by term (see the function's comment).
+ *
  * Inputs are bf16 bit patterns, widened exactly to double.
  */
 #include <math.h>
@@ -233,6 +239,143 @@ int oracle_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
         free(qrow);
         free(acc);
     }
+    return 0;
+}
+
+/*
+ * Backward of attention by definition.  Inputs are doubles (callers widen bf16
+ * exactly), contiguous:
+ *   Q, dO [B, Hq, N, D];  K, V [B, Hkv, N, D]
+ * Outputs (contiguous, double):
+ *   O [B, Hq, N, D], LSE [B, Hq, N]   the forward pass, as oracle_attention
+ *   dQ [B, Hq, N, D], dK, dV [B, Hkv, N, D]
+ *
+ * For query q of head hq, A(q) its allowed key set, s_kv = scale Q_q.K_kv and
+ * P_kv = exp(s_kv - LSE_q) the softmax weights over A(q) (zero outside), the
+ * output is O_q = sum_kv P_kv V_kv, and for a scalar loss with dL/dO = dO:
+ *   dP_kv = dO_q . V_kv                      (gradient of the weights)
+ *   Delta_q = sum_kv P_kv dP_kv              (the softmax Jacobian's row term)
+ *   dS_kv = P_kv (dP_kv - Delta_q)           (gradient of the scores)
+ *   dQ_q  = scale sum_kv dS_kv K_kv
+ *   dK_kv = scale sum_(hq in group, q) dS_kv Q_q
+ *   dV_kv = sum_(hq in group, q) P_kv dO_q
+ * A query with no allowed key has O = 0, LSE = -inf and contributes nothing.
+ * Pass 1 walks query rows (O, LSE, Delta, dQ); pass 2 walks key rows and sums
+ * over every query that may attend to it (dK, dV).  Returns 0, or -1 on a bad
+ * argument.
+ */
+int oracle_attention_bwd(const double *Q, const double *K, const double *V, const double *dO,
+                         int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t D,
+                         const oracle_pattern *p, double scale,
+                         double *O, double *LSE, double *dQ, double *dK, double *dV, int32_t n_threads)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || N < 0 || D <= 0)
+        return -1;
+    int64_t group = Hq / Hkv;
+    double *delta = (double *)malloc(sizeof(double) * (size_t)(B * Hq * N > 0 ? B * Hq * N : 1));
+    if (!delta)
+        return -1;
+#ifdef _OPENMP
+    if (n_threads > 0)
+        omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+
+    /* pass 1: per query row */
+#pragma omp parallel
+    {
+        int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (size_t)(N > 0 ? N : 1));
+        double *s = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+        double *dp = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t row = 0; row < B * Hq * N; row++) {
+            int64_t q = row % N, bh = row / N, b = bh / Hq, hq = bh % Hq, hkv = hq / group;
+            const double *qv = Q + row * D, *dov = dO + row * D;
+            const double *kb = K + (b * Hkv + hkv) * N * D, *vb = V + (b * Hkv + hkv) * N * D;
+            double *o = O + row * D, *dq = dQ + row * D;
+            int64_t n_keys = 0;
+            for (int64_t kv = 0; kv < N; kv++)
+                if (oracle_allowed(p, q, kv) == 1)
+                    keys[n_keys++] = kv;
+            for (int64_t c = 0; c < D; c++) {
+                o[c] = 0.0;
+                dq[c] = 0.0;
+            }
+            if (n_keys == 0) {
+                LSE[row] = -INFINITY;
+                delta[row] = 0.0;
+                continue;
+            }
+            double m = -INFINITY;
+            for (int64_t t = 0; t < n_keys; t++) {
+                double dot = 0.0;
+                for (int64_t c = 0; c < D; c++)
+                    dot += qv[c] * kb[keys[t] * D + c];
+                s[t] = scale * dot;
+                if (s[t] > m)
+                    m = s[t];
+            }
+            double l = 0.0;
+            for (int64_t t = 0; t < n_keys; t++)
+                l += exp(s[t] - m);
+            double lse = m + log(l);
+            LSE[row] = lse;
+            double dl = 0.0;
+            for (int64_t t = 0; t < n_keys; t++) {
+                double pw = exp(s[t] - lse);
+                double d = 0.0;
+                for (int64_t c = 0; c < D; c++) {
+                    o[c] += pw * vb[keys[t] * D + c];
+                    d += dov[c] * vb[keys[t] * D + c];
+                }
+                dp[t] = d;
+                dl += pw * d;
+            }
+            delta[row] = dl;
+            for (int64_t t = 0; t < n_keys; t++) {
+                double ds = exp(s[t] - lse) * (dp[t] - dl);
+                for (int64_t c = 0; c < D; c++)
+                    dq[c] += scale * ds * kb[keys[t] * D + c];
+            }
+        }
+        free(keys);
+        free(s);
+        free(dp);
+    }
+
+    /* pass 2: per key row, over every query of the group that may attend to it */
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t row = 0; row < B * Hkv * N; row++) {
+        int64_t kv = row % N, bh = row / N, b = bh / Hkv, hkv = bh % Hkv;
+        const double *kv_k = K + row * D, *kv_v = V + row * D;
+        double *dk = dK + row * D, *dv = dV + row * D;
+        for (int64_t c = 0; c < D; c++) {
+            dk[c] = 0.0;
+            dv[c] = 0.0;
+        }
+        for (int64_t hq = hkv * group; hq < (hkv + 1) * group; hq++) {
+            for (int64_t q = 0; q < N; q++) {
+                if (oracle_allowed(p, q, kv) != 1)
+                    continue;
+                int64_t qrow = (b * Hq + hq) * N + q;
+                const double *qv = Q + qrow * D, *dov = dO + qrow * D;
+                double dot = 0.0, d = 0.0;
+                for (int64_t c = 0; c < D; c++) {
+                    dot += qv[c] * kv_k[c];
+                    d += dov[c] * kv_v[c];
+                }
+                double pw = exp(scale * dot - LSE[qrow]);
+                double ds = pw * (d - delta[qrow]);
+                for (int64_t c = 0; c < D; c++) {
+                    dv[c] += pw * dov[c];
+                    dk[c] += scale * ds * qv[c];
+                }
+            }
+        }
+    }
+    free(delta);
     return 0;
 }
 

@@ -1,7 +1,9 @@
 """Plant plausible mistakes in copies of the oracle (on the CPU) and check that
 the pins catch each one: a wrong window bound, sink bound, stride reading, LSE
-base, head mapping, missing scale, or tile-fullness test.  A pin set that let
-one of these through would not be pinning the oracle."""
+base, head mapping, missing scale, or tile-fullness test; in the backward, a
+dropped softmax row term, a wrong sign, a missing scale, a transposed operand
+or a group head left out.  A pin set that let one of these through would not
+be pinning the oracle."""
 import math
 
 import numpy as np
@@ -14,6 +16,7 @@ from oracle import Pattern
 
 from test_oracle import (closed_live_window_sinks, closed_pairs_window_sinks,
                          closed_row_count_strided, rule_sets)
+from test_oracle_bwd import FD_CASES, autograd_pin_holds, fd_pin_holds
 
 MUTANTS = {
     "window_exclusive": ("delta <= p->window", "delta < p->window"),
@@ -21,7 +24,8 @@ MUTANTS = {
     "stride_absolute": ("delta % p->stride == 0", "kv % p->stride == 0"),
     "lse_base2": ("*lse = m + log(l);", "*lse = m + log2(l);"),
     "head_map_modulo": ("int64_t hkv = hq / group;", "int64_t hkv = hq % Hkv;"),
-    "scale_dropped": ("s[t] = scale * dot;", "s[t] = dot;"),
+    "scale_dropped": ("bf16_to_double(kp[c]);\n                        s[t] = scale * dot;",
+                      "bf16_to_double(kp[c]);\n                        s[t] = dot;"),
     "full_ignores_ragged": ("full[i * T + c] = allowed == (q1 - q0) * (k1 - k0);",
                             "full[i * T + c] = allowed == (int64_t)block * block;"),
 }
@@ -85,3 +89,32 @@ def test_mutant_is_caught(name, tmp_path):
     assert src.count(old) == 1, f"mutation site for {name} not found"
     path = oracle.compile_source(src.replace(old, new), str(tmp_path / f"lib_{name}.so"))
     assert not pins_hold(oracle.Oracle(path))
+
+
+BWD_MUTANTS = {
+    "bwd_dq_delta_dropped": ("double ds = exp(s[t] - lse) * (dp[t] - dl);", "double ds = exp(s[t] - lse) * dp[t];"),
+    "bwd_dk_delta_sign": ("double ds = pw * (d - delta[qrow]);", "double ds = pw * (d + delta[qrow]);"),
+    "bwd_dk_scale_dropped": ("dk[c] += scale * ds * qv[c];", "dk[c] += ds * qv[c];"),
+    "bwd_dv_takes_score_grad": ("dv[c] += pw * dov[c];", "dv[c] += ds * dov[c];"),
+    "bwd_dq_uses_values": ("dq[c] += scale * ds * kb[keys[t] * D + c];", "dq[c] += scale * ds * vb[keys[t] * D + c];"),
+    "bwd_first_group_head_only": ("for (int64_t hq = hkv * group; hq < (hkv + 1) * group; hq++)",
+                                  "for (int64_t hq = hkv * group; hq < hkv * group + 1; hq++)"),
+    "bwd_delta_from_values_only": ("dl += pw * d;", "dl += d;"),
+}
+
+
+def bwd_pins_hold(o: oracle.Oracle) -> bool:
+    return all(fd_pin_holds(o, c) for c in FD_CASES) and autograd_pin_holds(o)
+
+
+def test_unmutated_backward_passes():
+    assert bwd_pins_hold(oracle.default())
+
+
+@pytest.mark.parametrize("name", sorted(BWD_MUTANTS))
+def test_backward_mutant_is_caught(name, tmp_path):
+    old, new = BWD_MUTANTS[name]
+    src = oracle.source()
+    assert src.count(old) == 1, f"mutation site for {name} not found"
+    path = oracle.compile_source(src.replace(old, new), str(tmp_path / f"lib_{name}.so"))
+    assert not bwd_pins_hold(oracle.Oracle(path))
