@@ -1,4 +1,4 @@
-"""Block-sparse causal attention forward on B200 (sm_100a).
+"""Block-sparse causal attention forward and backward on B200 (sm_100a).
 
 Thin binding over the C ABI in ``include/sparse_attn.h`` (``libsparse_attn.so``,
 built in-tree).  This module only marshals arguments: torch tensors supply
@@ -41,6 +41,7 @@ EXPORTED = (
     "sparse_attn_fwd", "sparse_attn_fwd_host", "sparse_attn_fwd_host_workspace",
     "sparse_attn_check_device", "sparse_attn_set_debug", "sparse_attn_status_string",
     "sparse_attn_version", "sparse_attn_fwd_noalloc", "sparse_attn_fwd_heads",
+    "sparse_attn_transpose_block_mask", "sparse_attn_bwd_workspace", "sparse_attn_bwd",
 )
 
 
@@ -83,6 +84,10 @@ def _load() -> ctypes.CDLL:
     L.sparse_attn_fwd_noalloc.argtypes = [vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp]
     L.sparse_attn_fwd_heads.argtypes = [vp, vp, vp, M, P, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32), S,
                                         ctypes.c_float, vp, vp, vp]
+    L.sparse_attn_transpose_block_mask.argtypes = [M, M]
+    L.sparse_attn_bwd_workspace.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
+    L.sparse_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp, vp,
+                                  ctypes.c_size_t, vp]
     L.sparse_attn_check_device.argtypes = [vp]
     L.sparse_attn_set_debug.argtypes = [ctypes.c_int32, ctypes.c_int64]
     L.sparse_attn_status_string.argtypes = [ctypes.c_int]
@@ -91,7 +96,8 @@ def _load() -> ctypes.CDLL:
     L.sparse_attn_version.restype = ctypes.c_int32
     for name in ("sparse_attn_build_block_mask", "sparse_attn_count_pairs", "sparse_attn_fwd",
                  "sparse_attn_fwd_host", "sparse_attn_fwd_host_workspace", "sparse_attn_check_device",
-                 "sparse_attn_set_debug", "sparse_attn_fwd_noalloc", "sparse_attn_fwd_heads"):
+                 "sparse_attn_set_debug", "sparse_attn_fwd_noalloc", "sparse_attn_fwd_heads",
+                 "sparse_attn_transpose_block_mask", "sparse_attn_bwd_workspace", "sparse_attn_bwd"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -171,6 +177,22 @@ def build_block_mask(pattern: Pattern, N: int, block: int = 128) -> BlockMask:
     return BlockMask(counts, index, full, m.block, m.n_live, m.n_full, m.max_per_row, N)
 
 
+def transpose_block_mask(mask: BlockMask) -> BlockMask:
+    """Per-kv-tile lists of the query tiles that attend to it (host arrays);
+    ``counts[c]``, ``index[c, e]`` and ``full[c, e]`` with rows and columns
+    swapped relative to ``mask``.  The backward pass takes this form."""
+    T = mask.T
+    counts = np.zeros(T, dtype=np.int32)
+    index = np.zeros((T, T), dtype=np.int32)
+    full = np.zeros((T, T), dtype=np.uint8)
+    out = _BlockMask(T, T, 0, 0, 0, 0, counts.ctypes.data if T else None,
+                     index.ctypes.data if T else None, full.ctypes.data if T else None)
+    src = mask._c()
+    _check(lib.sparse_attn_transpose_block_mask(ctypes.byref(src), ctypes.byref(out)),
+           "sparse_attn_transpose_block_mask")
+    return BlockMask(counts, index, full, out.block, out.n_live, out.n_full, out.max_per_row, mask.N)
+
+
 def count_pairs(pattern: Pattern, N: int) -> int:
     out = ctypes.c_int64(0)
     _check(lib.sparse_attn_count_pairs(ctypes.byref(pattern._c()), N, ctypes.byref(out)),
@@ -246,6 +268,47 @@ def fwd_heads(q, k, v, masks, patterns, head_pattern, scale: float | None = None
                                          ctypes.byref(shape), float(scale), out.data_ptr(), lse.data_ptr(), st),
                "sparse_attn_fwd_heads")
     return out, lse
+
+
+def bwd_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, D: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.sparse_attn_bwd_workspace(ctypes.byref(_Shape(B, Hq, Hkv, N, D)), ctypes.byref(n)),
+           "sparse_attn_bwd_workspace")
+    return n.value
+
+
+def bwd(q, k, v, o, lse, do, mask_t: BlockMask, pattern: Pattern, scale: float | None = None,
+        dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients (dQ, dK, dV) for the upstream gradient ``do``.
+
+    q, o, do: [B, Hq, N, D] bf16 CUDA tensors; k, v: [B, Hkv, N, D]; lse: the
+    forward's [B, Hq, N] fp32.  ``mask_t`` is ``transpose_block_mask`` of the
+    pattern's block-128 mask, on the same device.  Asynchronous on ``stream``.
+    """
+    import torch
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    for t in (q, k, v, o, do):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError("q, k, v, o, do must be contiguous bf16 CUDA tensors")
+    if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+        raise TypeError("lse must be a contiguous fp32 CUDA tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_bytes(B, Hq, Hkv, N, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    shape = _Shape(B, Hq, Hkv, N, D)
+    with torch.cuda.device(q.device):
+        st = _stream_handle(stream, q.device)
+        _check(lib.sparse_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                   do.data_ptr(), ctypes.byref(mask_t._c()), ctypes.byref(pattern._c()),
+                                   ctypes.byref(shape), float(scale), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                   workspace.data_ptr(), workspace.numel(), st), "sparse_attn_bwd")
+    return dq, dk, dv
 
 
 def fwd_host_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, D: int) -> int:

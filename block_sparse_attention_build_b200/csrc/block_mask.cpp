@@ -157,3 +157,45 @@ extern "C" int sparse_attn_count_pairs(const sa_pattern* pattern, int64_t N, int
     *pairs = total;
     return SA_OK;
 }
+
+extern "C" int sparse_attn_transpose_block_mask(const sa_block_mask* rows, sa_block_mask* cols)
+{
+    if (!rows || !cols) return SA_ERR_INVALID_ARG;
+    const int32_t T = rows->n_q_tiles;
+    if (T < 0 || rows->n_kv_tiles != T) return SA_ERR_INVALID_ARG;
+    if (cols->n_q_tiles < T || cols->n_kv_tiles < T) return SA_ERR_BUFFER_TOO_SMALL;
+    if (T > 0 && (!rows->kv_count || !rows->kv_index || !rows->kv_full)) return SA_ERR_INVALID_ARG;
+    if (T > 0 && (!cols->kv_count || !cols->kv_index || !cols->kv_full)) return SA_ERR_INVALID_ARG;
+    for (int32_t c = 0; c < T; c++) cols->kv_count[c] = 0;
+    int64_t live = 0, nfull = 0;
+    // rows in ascending order, so every column list comes out ascending
+    for (int32_t i = 0; i < T; i++) {
+        const int32_t n = rows->kv_count[i];
+        if (n < 0 || n > T) return SA_ERR_INVALID_ARG;
+        for (int32_t e = 0; e < n; e++) {
+            const int32_t c = rows->kv_index[int64_t(i) * T + e];
+            if (c < 0 || c >= T) return SA_ERR_INVALID_ARG;
+            const int32_t pos = cols->kv_count[c]++;
+            if (pos >= T) return SA_ERR_INVALID_ARG;  // a row lists c twice
+            cols->kv_index[int64_t(c) * T + pos] = i;
+            cols->kv_full[int64_t(c) * T + pos] = rows->kv_full[int64_t(i) * T + e] ? 1 : 0;
+            live++;
+            nfull += cols->kv_full[int64_t(c) * T + pos];
+        }
+    }
+    int32_t max_col = 0;
+    for (int32_t c = 0; c < T; c++) {
+        for (int32_t t = cols->kv_count[c]; t < T; t++) {
+            cols->kv_index[int64_t(c) * T + t] = -1;
+            cols->kv_full[int64_t(c) * T + t] = 0;
+        }
+        max_col = std::max(max_col, cols->kv_count[c]);
+    }
+    cols->n_q_tiles = T;
+    cols->n_kv_tiles = T;
+    cols->block = rows->block;
+    cols->max_per_row = max_col;
+    cols->n_live = live;
+    cols->n_full = nfull;
+    return SA_OK;
+}

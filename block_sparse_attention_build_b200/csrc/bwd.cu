@@ -1,0 +1,149 @@
+// C ABI of the backward pass: argument checks, the workspace layout, TMA
+// descriptors and the three launches (prep, main, dQ conversion).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/sparse_attn.h"
+#include "bwd_sm100.cuh"
+#include "runtime.h"
+#include "tma_host.h"
+
+namespace sa {
+namespace {
+
+constexpr int kMaxDev = 64;
+
+struct BwdLayout {
+    size_t lse2, delta, dq, total;  // byte offsets in the workspace, each 256-aligned
+};
+
+BwdLayout bwd_layout(const sa_shape& s)
+{
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t rows = size_t(s.B) * size_t(s.Hq) * size_t(s.N);
+    BwdLayout w;
+    w.lse2 = 0;
+    w.delta = up(rows * 4);
+    w.dq = w.delta + up(rows * 4);
+    w.total = w.dq + up(rows * size_t(s.D) * 4);
+    return w;
+}
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int D>
+int bwd_run(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
+            const sa_block_mask& mt, const sa_pattern& pt, const sa_shape& s, float scale, void* dQ, void* dK,
+            void* dV, uint8_t* ws, cudaStream_t st)
+{
+    int32_t* status = nullptr;
+    if (int rc = device_status_word(&status)) return rc;
+    const BwdLayout L = bwd_layout(s);
+    float* lse2 = reinterpret_cast<float*>(ws + L.lse2);
+    float* delta = reinterpret_cast<float*>(ws + L.delta);
+    float* dq_acc = reinterpret_cast<float*>(ws + L.dq);
+    const int64_t rows = int64_t(s.B) * s.Hq * s.N;
+
+    CUtensorMap mq, mdo, mk, mv;
+    if (!make_map_bf16_3d(&mq, Q, D, s.N, uint64_t(s.B) * s.Hq, kBwdTile) ||
+        !make_map_bf16_3d(&mdo, dO, D, s.N, uint64_t(s.B) * s.Hq, kBwdTile) ||
+        !make_map_bf16_3d(&mk, K, D, s.N, uint64_t(s.B) * s.Hkv, kBwdTile) ||
+        !make_map_bf16_3d(&mv, V, D, s.N, uint64_t(s.B) * s.Hkv, kBwdTile))
+        return SA_ERR_CUDA;
+
+    bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, lse2, delta, dq_acc, rows);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+
+    BwdParams p;
+    p.t_count = mt.kv_count;
+    p.t_index = mt.kv_index;
+    p.t_full = mt.kv_full;
+    p.lse2 = lse2;
+    p.delta = delta;
+    p.dq_acc = dq_acc;
+    p.dK = static_cast<__nv_bfloat16*>(dK);
+    p.dV = static_cast<__nv_bfloat16*>(dV);
+    p.status = status;
+    p.timeout = wait_limit_cycles();
+    p.T = mt.n_q_tiles;
+    p.N = s.N;
+    p.B = s.B;
+    p.Hq = s.Hq;
+    p.Hkv = s.Hkv;
+    p.group = s.Hq / s.Hkv;
+    p.window = pt.window;
+    p.sinks = pt.sinks;
+    p.stride = pt.stride;
+    p.n_global = pt.n_global;
+    p.scale_log2 = scale * 1.44269504088896340736f;
+    p.scale = scale;
+
+    using C = BwdCfg<D>;
+    static bool attr_set[kMaxDev] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return SA_ERR_CUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+            cudaSuccess)
+            return SA_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    const unsigned grid = static_cast<unsigned>(int64_t(s.B) * s.Hkv * p.T);
+    bwd_kernel<D><<<grid, kBwdThreads, C::kSmemBytes, st>>>(mq, mdo, mk, mv, p);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+
+    const int64_t n8 = rows * D / 8;
+    const int n_sm = device_sm_count();
+    int64_t g = (n8 + 255) / 256;
+    if (n_sm > 0 && g > int64_t(n_sm) * 8) g = int64_t(n_sm) * 8;
+    bwd_dq_kernel<<<static_cast<unsigned>(g), 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), n8);
+    return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace sa
+
+extern "C" int sparse_attn_bwd_workspace(const sa_shape* shape, size_t* bytes)
+{
+    if (!shape || !bytes) return SA_ERR_INVALID_ARG;
+    const sa_shape s = *shape;
+    if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
+    *bytes = sa::bwd_layout(s).total;
+    return SA_OK;
+}
+
+extern "C" int sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const float* LSE,
+                               const void* dO, const sa_block_mask* mask_t, const sa_pattern* pattern,
+                               const sa_shape* shape, float scale, void* dQ, void* dK, void* dV, void* workspace,
+                               size_t workspace_bytes, void* stream)
+{
+    if (!mask_t || !pattern || !shape) return SA_ERR_INVALID_ARG;
+    const sa_shape s = *shape;
+    const sa_pattern pt = *pattern;
+    if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
+    if (pt.causal != 1) return SA_ERR_UNSUPPORTED;
+    if (pt.window < -1 || pt.sinks < 0 || pt.stride < 0 || pt.n_global < 0) return SA_ERR_INVALID_ARG;
+    if (s.D != 64 && s.D != 128) return SA_ERR_UNSUPPORTED;
+    if (mask_t->block != sa::kBwdTile) return SA_ERR_UNSUPPORTED;
+    if (s.B == 0 || s.Hq == 0 || s.N == 0) return SA_OK;  // nothing to compute
+    if (s.Hkv <= 0 || s.Hq % s.Hkv != 0) return SA_ERR_UNSUPPORTED;
+    const int64_t T = (int64_t(s.N) + sa::kBwdTile - 1) / sa::kBwdTile;
+    if (mask_t->n_q_tiles != T || mask_t->n_kv_tiles != T) return SA_ERR_MASK_MISMATCH;
+    if (!mask_t->kv_count || !mask_t->kv_index || !mask_t->kv_full) return SA_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV || !workspace) return SA_ERR_INVALID_ARG;
+    using sa::al16;
+    if (!al16(Q) || !al16(K) || !al16(V) || !al16(O) || !al16(LSE) || !al16(dO) || !al16(dQ) || !al16(dK) ||
+        !al16(dV) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return SA_ERR_MISALIGNED;
+    if (workspace_bytes < sa::bwd_layout(s).total) return SA_ERR_BUFFER_TOO_SMALL;
+    const int64_t rows = int64_t(s.B) * s.Hq * s.N;
+    if (int64_t(s.B) * s.Hkv * T > INT32_MAX || (rows + 7) / 8 > INT32_MAX) return SA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (s.D == 128) return sa::bwd_run<128>(Q, K, V, O, LSE, dO, *mask_t, pt, s, scale, dQ, dK, dV, ws, st);
+    return sa::bwd_run<64>(Q, K, V, O, LSE, dO, *mask_t, pt, s, scale, dQ, dK, dV, ws, st);
+}

@@ -1,0 +1,530 @@
+// Backward pass of block-sparse causal attention on sm_100a: dQ, dK, dV for
+// an upstream gradient dO, given Q, K, V, the forward output O and its LSE.
+//
+// The pages print no backward pass; what is computed is the gradient of the
+// masked attention of the "Sparse-трансформеры" page (section "Как это
+// выглядит в коде"): with P the softmax weights of each query over its
+// allowed keys,
+//   dV = Pᵀ dO,  dP = dO Vᵀ,  Δ_q = Σ_d dO[q,d] O[q,d],  dS = P ∘ (dP − Δ),
+//   dQ = scale · dS K,  dK = scale · dSᵀ Q,
+// summed over the query heads of a GQA group for dK and dV.  Tiles the block
+// mask marks empty are skipped, as in the forward ("Sparse Attention" glossary
+// page, section "Ein Muster in Einsparungen verwandeln").
+//
+// Kernels, in launch order on one stream:
+//   bwd_prep_kernel  per query row: Δ from O and dO, the LSE in base 2, and a
+//                    zeroed fp32 dQ accumulator row;
+//   bwd_kernel       one CTA per (kv tile, batch, kv head): walks the query
+//                    tiles that attend to its kv tile (the transposed block
+//                    mask) for every query head of the group, accumulating dK
+//                    and dV in tensor memory and adding each step's dQ tile to
+//                    the fp32 accumulator with vector reductions;
+//   bwd_dq_kernel    dQ accumulator -> bf16.
+//
+// bwd_kernel, 192 threads: warps 0-3 the element-wise work (one kv row per
+// thread, tensor-memory lane = kv row), warp 4 the TMA producer, warp 5 tensor
+// memory allocation and the single MMA-issuing lane.  Per step (one query
+// tile of one head):
+//   Sᵀ = K Qᵀ, dPᵀ = V dOᵀ                 tcgen05 SS, fp32 in tensor memory
+//   Pᵀ = exp2(Sᵀ·scale·log2e − LSE₂)      masked on partial tiles; bf16 back
+//                                           into the Sᵀ columns
+//   dSᵀ = Pᵀ ∘ (dPᵀ − Δ) · scale           bf16 into shared memory
+//   dV += Pᵀ dO  (TS: Pᵀ from tensor memory), dK += dSᵀ Q  (SS)
+//   dQ  = dS K   (SS, dS read MN-major from the same shared tile) into the dPᵀ
+//                columns, then read out and reduced into global memory.
+// Every wait is bounded; on expiry a role sets a status bit, raises an abort
+// flag and leaves its loop; the MMA lane drains its MMAs and the producer its
+// copies before tensor memory is freed.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "sm100.cuh"
+
+namespace sa {
+
+constexpr int kBwdThreads = 192;
+constexpr int kBwdTile = 128;  // query and kv tile edge (the block mask's block)
+
+enum : int32_t {
+    ST_BWD_PRODUCER_WAIT = 1 << 8,
+    ST_BWD_MMA_WAIT = 1 << 9,
+    ST_BWD_ELEM_WAIT = 1 << 10,
+    ST_BWD_DRAIN_WAIT = 1 << 11,
+};
+
+struct BwdParams {
+    const int32_t* t_count;  // [T] query tiles listed for kv tile c (transposed block mask)
+    const int32_t* t_index;  // [T * T] their indices, ascending
+    const uint8_t* t_full;   // [T * T] 1 when every in-range pair of the tile is allowed
+    const float* lse2;       // [B * Hq * N] LSE in base 2; +inf for a row without keys
+    const float* delta;      // [B * Hq * N] Δ = rowsum(dO ∘ O)
+    float* dq_acc;           // [B * Hq * N * D] fp32, zeroed by the prep kernel
+    __nv_bfloat16* dK;       // [B * Hkv * N * D]
+    __nv_bfloat16* dV;       // [B * Hkv * N * D]
+    int32_t* status;
+    long long timeout;       // SM cycles per bounded wait
+    int32_t T, N, B, Hq, Hkv, group;
+    int32_t window, sinks, stride, n_global;
+    float scale_log2;        // scale * log2(e)
+    float scale;
+};
+
+template <int D>
+struct BwdCfg {
+    static constexpr int kTileBytes = kBwdTile * D * 2;    // a Q, dO, K or V tile (bf16)
+    static constexpr int kPanel = kBwdTile * 128;          // 64 columns x 128 rows, 128-byte swizzled
+    static constexpr int kOffK = 0;
+    static constexpr int kOffV = kOffK + kTileBytes;
+    static constexpr int kOffQ = kOffV + kTileBytes;       // two buffers
+    static constexpr int kOffdO = kOffQ + 2 * kTileBytes;  // two buffers
+    static constexpr int kOffdS = kOffdO + 2 * kTileBytes; // dSᵀ: 128 kv rows x 128 q columns, two panels
+    static constexpr int kOffBar = kOffdS + 2 * kPanel;
+    static constexpr int kNumBars = 10;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tensor-memory base, abort flag
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
+    static constexpr uint32_t kColS = 0;         // Sᵀ (fp32), then Pᵀ (bf16 pairs) in its first 64 columns
+    static constexpr uint32_t kColdP = 128;      // dPᵀ (fp32), then the step's dQ tile
+    static constexpr uint32_t kColdV = 256;
+    static constexpr uint32_t kColdK = 256 + D;
+    static constexpr uint32_t kTmemCols = 512;
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+    static_assert(kColdK + D <= kTmemCols, "tensor memory columns");
+};
+
+__device__ __forceinline__ void bwd_report(const BwdParams& p, volatile int* abort_flag, int32_t bit)
+{
+    *abort_flag = 1;
+    atomicOr(p.status, bit);
+}
+
+// Bits lo..hi of a 32-bit word, clipped to [0, 31]; 0 when the range is empty.
+__device__ __forceinline__ uint32_t bwd_bits(int lo, int hi)
+{
+    lo = max(lo, 0);
+    hi = min(hi, 31);
+    if (lo > hi) return 0u;
+    const uint32_t upto_hi = hi == 31 ? 0xffffffffu : ((1u << (hi + 1)) - 1u);
+    return upto_hi & ~((1u << lo) - 1u);
+}
+
+// Allowed pairs (q, kv) for q = qb + i, i in [0, 32), as bits: the pattern's
+// rule (band, sink and global columns, global rows, stride) under causality
+// and the sequence bound.
+__device__ __forceinline__ uint32_t bwd_allow_word(const BwdParams& p, int qb, int kv)
+{
+    if (kv >= p.N) return 0u;
+    const uint32_t in_range = bwd_bits(kv - qb, p.N - 1 - qb);  // kv <= q < N
+    if (kv < max(p.sinks, p.n_global)) return in_range;
+    uint32_t m = 0u;
+    if (p.window >= 0) m |= bwd_bits(kv - qb, kv + p.window - qb);
+    if (p.n_global > 0) m |= bwd_bits(0, p.n_global - 1 - qb);
+    if (p.stride > 0) {
+        int i = (kv - qb) % p.stride;
+        if (i < 0) i += p.stride;
+        for (; i < 32; i += p.stride) m |= 1u << i;
+    }
+    return m & in_range;
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+// One warp per query row: Δ = Σ_d dO·O (fp32 from the bf16 tensors), LSE₂ =
+// LSE·log2(e) (+inf where LSE = -inf), and the row of the dQ accumulator zeroed.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ O,
+                                                       const __nv_bfloat16* __restrict__ dO,
+                                                       const float* __restrict__ LSE, float* __restrict__ lse2,
+                                                       float* __restrict__ delta, float* __restrict__ dq_acc,
+                                                       int64_t rows)
+{
+    static_assert(D == 64 || D == 128, "head dimension");
+    constexpr int E = D / 32;  // elements per lane
+    const int64_t row = int64_t(blockIdx.x) * 8 + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (row >= rows) return;
+    const __nv_bfloat16* o = O + row * D + lane * E;
+    const __nv_bfloat16* g = dO + row * D + lane * E;
+    float s = 0.f;
+    if constexpr (E == 4) {
+        const uint2 ov = *reinterpret_cast<const uint2*>(o);
+        const uint2 gv = *reinterpret_cast<const uint2*>(g);
+        const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov.x));
+        const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov.y));
+        const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.x));
+        const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.y));
+        s = o0.x * g0.x + o0.y * g0.y + o1.x * g1.x + o1.y * g1.y;
+        *reinterpret_cast<float4*>(dq_acc + row * D + lane * E) = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+        const uint32_t ov = *reinterpret_cast<const uint32_t*>(o);
+        const uint32_t gv = *reinterpret_cast<const uint32_t*>(g);
+        const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov));
+        const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv));
+        s = o0.x * g0.x + o0.y * g0.y;
+        *reinterpret_cast<float2*>(dq_acc + row * D + lane * E) = make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off /= 2) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) {
+        delta[row] = s;
+        const float L = LSE[row];
+        lse2[row] = L == -INFINITY ? INFINITY : L * 1.44269504088896340736f;
+    }
+}
+
+// dQ (bf16) from the fp32 accumulator, eight elements per thread and pass.
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dQ,
+                                                     int64_t n8)
+{
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
+        const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+        const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+        uint4 v;
+        v.x = pack_bf16x2(a.x, a.y);
+        v.y = pack_bf16x2(a.z, a.w);
+        v.z = pack_bf16x2(b.x, b.y);
+        v.w = pack_bf16x2(b.z, b.w);
+        reinterpret_cast<uint4*>(dQ)[i] = v;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const BwdParams p)
+{
+    using C = BwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sK = smem + C::kOffK;
+    uint8_t* sV = smem + C::kOffV;
+    uint8_t* sQ = smem + C::kOffQ;
+    uint8_t* sdO = smem + C::kOffdO;
+    uint8_t* sdS = smem + C::kOffdS;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint64_t* kv_full = bars;         // K and V landed
+    uint64_t* qd_full = bars + 1;     // [2] Q and dO of a step landed
+    uint64_t* qd_empty = bars + 3;    // [2] the step's dV and dK MMAs are done with them
+    uint64_t* s_full = bars + 5;      // Sᵀ and dPᵀ are in tensor memory
+    uint64_t* ds_full = bars + 6;     // Pᵀ (tensor memory) and dSᵀ (shared memory) written (128 threads)
+    uint64_t* dq_full = bars + 7;     // the step's dQ tile is in tensor memory (and every earlier MMA done)
+    uint64_t* dq_empty = bars + 8;    // the dQ tile has been read (128 threads)
+    uint64_t* drain = bars + 9;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    // kv tile c slowest, so the tiles near the sequence start (longest lists) start first
+    const int bh = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.B * p.Hkv));
+    const int c = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.B * p.Hkv));
+    const int b = bh / p.Hkv;
+    const int hkv = bh % p.Hkv;
+    const int n_list = min(max(__ldg(&p.t_count[c]), 0), p.T);
+    const int steps = p.group * n_list;
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int x = 0; x < 2; x++) {
+            mbar_init(&qd_full[x], 1);
+            mbar_init(&qd_empty[x], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(ds_full, 128);
+        mbar_init(dq_full, 1);
+        mbar_init(dq_empty, 128);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 4 && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmdO);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const long long lim = p.timeout;
+
+    // query head and query tile of step j (heads outer, list entries inner)
+    auto step_of = [&](int j, int& hq, int& r, bool& full) {
+        const int h = j / n_list;
+        const int e = j - h * n_list;
+        r = min(max(__ldg(&p.t_index[int64_t(c) * p.T + e]), 0), p.T - 1);
+        full = __ldg(&p.t_full[int64_t(c) * p.T + e]) != 0;
+        hq = hkv * p.group + h;
+    };
+
+    if (warp == 4) {
+        // ================================================================ producer (one lane)
+        if (lane == 0 && steps > 0) {
+            const uint64_t pol = policy_evict_last();
+            const int kvplane = b * p.Hkv + hkv;
+            mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
+            for (int pc = 0; pc < D / 64; pc++) {
+                tma_load_3d(sK + pc * C::kPanel, &tmK, kv_full, pc * 64, c * kBwdTile, kvplane, pol);
+                tma_load_3d(sV + pc * C::kPanel, &tmV, kv_full, pc * 64, c * kBwdTile, kvplane, pol);
+            }
+            int issued = 0;
+            for (int j = 0; j < steps; j++) {
+                const int buf = j & 1;
+                if (j >= 2 && !mbar_wait(&qd_empty[buf], ((j >> 1) - 1) & 1, lim)) {
+                    bwd_report(p, abort_flag, ST_BWD_PRODUCER_WAIT);
+                    break;
+                }
+                if (*abort_flag) break;
+                int hq, r;
+                bool full;
+                step_of(j, hq, r, full);
+                const int qplane = b * p.Hq + hq;
+                mbar_arrive_expect_tx(&qd_full[buf], 2 * C::kTileBytes);
+                for (int pc = 0; pc < D / 64; pc++) {
+                    tma_load_3d(sQ + buf * C::kTileBytes + pc * C::kPanel, &tmQ, &qd_full[buf], pc * 64,
+                                r * kBwdTile, qplane, pol);
+                    tma_load_3d(sdO + buf * C::kTileBytes + pc * C::kPanel, &tmdO, &qd_full[buf], pc * 64,
+                                r * kBwdTile, qplane, pol);
+                }
+                issued = j + 1;
+            }
+            // copies in flight land before the CTA's shared memory goes away
+            bool ok = mbar_wait(kv_full, 0, lim);
+            for (int j = issued > 2 ? issued - 2 : 0; j < issued; j++) ok &= mbar_wait(&qd_full[j & 1], (j >> 1) & 1, lim);
+            if (!ok) bwd_report(p, abort_flag, ST_BWD_DRAIN_WAIT);
+        }
+    } else if (warp == 5) {
+        // ================================================================ MMA issuer
+        // The warp runs converged; one elected lane issues each MMA and commit.
+        if (steps > 0) {
+            constexpr uint32_t id_s = idesc_bf16_f32(kBwdTile, kBwdTile, false, false);
+            constexpr uint32_t id_kv = idesc_bf16_f32(kBwdTile, D, false, true);
+            constexpr uint32_t id_q = idesc_bf16_f32(kBwdTile, D, true, true);
+            constexpr uint32_t kTileU = C::kTileBytes >> 4;  // descriptor units (16 bytes)
+            const uint64_t d0 = smem_desc_sw128(smem_addr(sK), 16, 1024);
+            const uint32_t hi = static_cast<uint32_t>(d0 >> 32);
+            const uint32_t k_km = static_cast<uint32_t>(d0);
+            const uint32_t k_mn = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sK), C::kPanel, 1024));
+            const uint32_t v_km = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sV), 16, 1024));
+            const uint32_t q_km = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sQ), 16, 1024));
+            const uint32_t q_mn = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sQ), C::kPanel, 1024));
+            const uint32_t o_km = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sdO), 16, 1024));
+            const uint32_t o_mn = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sdO), C::kPanel, 1024));
+            const uint32_t s_km = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sdS), 16, 1024));
+            const uint32_t s_mn = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sdS), C::kPanel, 1024));
+            // k-step offsets (16 elements of the contraction), in descriptor units
+            auto km = [](int kk) { return static_cast<uint32_t>(((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4); };
+            auto mn = [](int kk) { return static_cast<uint32_t>((kk * 16 * 128) >> 4); };
+            auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, lim));
+            };
+            auto commit = [&](uint64_t* bar) {
+                if (elect_one()) tc_commit(bar);
+                __syncwarp();
+            };
+            bool ok = wait(kv_full, 0);
+            for (int j = 0; j < steps && ok; j++) {
+                const int buf = j & 1;
+                const uint32_t bo = buf * kTileU;
+                ok = wait(&qd_full[buf], (j >> 1) & 1) && (j == 0 || wait(dq_empty, (j - 1) & 1));
+                if (!ok || __any_sync(0xffffffffu, *abort_flag != 0)) break;
+                tc_fence_after_sync();
+                // Sᵀ = K Qᵀ and dPᵀ = V dOᵀ (M = kv rows, N = query rows, K = D)
+#pragma unroll
+                for (int kk = 0; kk < D / 16; kk++) {
+                    if (elect_one())
+                        mma_ss(tmem + C::kColS, desc_from_halves(k_km + km(kk), hi),
+                               desc_from_halves(q_km + bo + km(kk), hi), id_s, kk > 0 ? 1u : 0u);
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; kk++) {
+                    if (elect_one())
+                        mma_ss(tmem + C::kColdP, desc_from_halves(v_km + km(kk), hi),
+                               desc_from_halves(o_km + bo + km(kk), hi), id_s, kk > 0 ? 1u : 0u);
+                    __syncwarp();
+                }
+                commit(s_full);
+                ok = wait(ds_full, j & 1);
+                if (!ok || __any_sync(0xffffffffu, *abort_flag != 0)) break;
+                tc_fence_after_sync();
+                // dV += Pᵀ dO (Pᵀ bf16 in the Sᵀ columns) and dK += dSᵀ Q (M = kv rows, N = D, K = query rows)
+#pragma unroll
+                for (int kk = 0; kk < kBwdTile / 16; kk++) {
+                    if (elect_one())
+                        mma_ts(tmem + C::kColdV, tmem + C::kColS + kk * 8, desc_from_halves(o_mn + bo + mn(kk), hi),
+                               id_kv, (j > 0 || kk > 0) ? 1u : 0u);
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int kk = 0; kk < kBwdTile / 16; kk++) {
+                    if (elect_one())
+                        mma_ss(tmem + C::kColdK, desc_from_halves(s_km + km(kk), hi),
+                               desc_from_halves(q_mn + bo + mn(kk), hi), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
+                    __syncwarp();
+                }
+                commit(&qd_empty[buf]);
+                // dQ = dS K (M = query rows, N = D, K = kv rows), into the dPᵀ columns
+#pragma unroll
+                for (int kk = 0; kk < kBwdTile / 16; kk++) {
+                    if (elect_one())
+                        mma_ss(tmem + C::kColdP, desc_from_halves(s_mn + mn(kk), hi),
+                               desc_from_halves(k_mn + mn(kk), hi), id_q, kk > 0 ? 1u : 0u);
+                    __syncwarp();
+                }
+                commit(dq_full);
+            }
+            if (!ok && lane == 0) bwd_report(p, abort_flag, ST_BWD_MMA_WAIT);
+            // every MMA issued so far is complete before tensor memory is freed
+            commit(drain);
+            if (!wait(drain, 0) && lane == 0) bwd_report(p, abort_flag, ST_BWD_DRAIN_WAIT);
+        }
+    } else {
+        // ================================================================ element-wise warps 0-3
+        // Each warp decides to leave its loop as a whole (every test goes
+        // through a vote); the four warps never wait on one another except
+        // through bounded mbarrier waits.
+        const int t = threadIdx.x;  // kv row of Sᵀ / dPᵀ / dK / dV, query row of dQ (tensor-memory lane)
+        const uint32_t lanes = static_cast<uint32_t>(warp * 32) << 16;
+        const int kv = c * kBwdTile + t;
+        const bool kv_ragged = (c + 1) * kBwdTile > p.N;
+        bool ok = true;
+        for (int j = 0; j < steps; j++) {
+            int hq, r;
+            bool full;
+            step_of(j, hq, r, full);
+            const int q0 = r * kBwdTile;
+            const int64_t qrow0 = (int64_t(b) * p.Hq + hq) * p.N;
+            // LSE₂ and Δ of query column 32cc + lane, handed to the other lanes by shuffles
+            float lse_r[4], dl_r[4];
+#pragma unroll
+            for (int cc = 0; cc < 4; cc++) {
+                const int q = q0 + cc * 32 + lane;
+                lse_r[cc] = q < p.N ? __ldg(&p.lse2[qrow0 + q]) : INFINITY;
+                dl_r[cc] = q < p.N ? __ldg(&p.delta[qrow0 + q]) : 0.f;
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, lim) && !*abort_flag);
+            if (!ok) break;
+            tc_fence_after_sync();
+            const bool masked = !full || kv_ragged || q0 + kBwdTile > p.N;
+#pragma unroll 1
+            for (int cc = 0; cc < kBwdTile / 32; cc++) {
+                uint32_t s[32], d[32];
+                tmem_ld_32x32b_x32(tmem + lanes + C::kColS + cc * 32, s);
+                tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + cc * 32, d);
+                const float lse_c = cc == 0 ? lse_r[0] : cc == 1 ? lse_r[1] : cc == 2 ? lse_r[2] : lse_r[3];
+                const float dl_c = cc == 0 ? dl_r[0] : cc == 1 ? dl_r[1] : cc == 2 ? dl_r[2] : dl_r[3];
+                const uint32_t allow = masked ? bwd_allow_word(p, q0 + cc * 32, kv) : 0xffffffffu;
+                tmem_wait_ld();
+                reg_fence(s);
+                reg_fence(d);
+                uint32_t pk[16], gk[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const float l0 = __shfl_sync(0xffffffffu, lse_c, i);
+                    const float l1 = __shfl_sync(0xffffffffu, lse_c, i + 1);
+                    const float e0 = __shfl_sync(0xffffffffu, dl_c, i);
+                    const float e1 = __shfl_sync(0xffffffffu, dl_c, i + 1);
+                    float p0 = ex2_approx(fmaf(__uint_as_float(s[i]), p.scale_log2, -l0));
+                    float p1 = ex2_approx(fmaf(__uint_as_float(s[i + 1]), p.scale_log2, -l1));
+                    p0 = (allow >> i) & 1u ? p0 : 0.f;
+                    p1 = (allow >> (i + 1)) & 1u ? p1 : 0.f;
+                    const float g0 = p0 * (__uint_as_float(d[i]) - e0) * p.scale;
+                    const float g1 = p1 * (__uint_as_float(d[i + 1]) - e1) * p.scale;
+                    pk[i / 2] = pack_bf16x2(p0, p1);
+                    gk[i / 2] = pack_bf16x2(g0, g1);
+                }
+                // Pᵀ (bf16 pairs) over Sᵀ columns already read
+                tmem_st_32x32b_x16(tmem + lanes + C::kColS + cc * 16, pk);
+                // dSᵀ row t, query columns 32cc..32cc+31: four 16-byte units of panel cc / 2
+                uint8_t* rowp = sdS + (cc / 2) * C::kPanel + t * 128;
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    const int u = (cc % 2) * 4 + k;
+                    *reinterpret_cast<uint4*>(rowp + ((u ^ (t & 7)) << 4)) =
+                        make_uint4(gk[4 * k], gk[4 * k + 1], gk[4 * k + 2], gk[4 * k + 3]);
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(ds_full);
+            ok = __all_sync(0xffffffffu, mbar_wait(dq_full, j & 1, lim) && !*abort_flag);
+            if (!ok) break;
+            tc_fence_after_sync();
+            // dQ row q0 + t of head hq into the fp32 accumulator
+            {
+                const int q = q0 + t;
+                float* dst = p.dq_acc + (qrow0 + q) * D;
+#pragma unroll 1
+                for (int k = 0; k < D / 32; k++) {
+                    uint32_t g[32];
+                    tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + k * 32, g);
+                    tmem_wait_ld();
+                    reg_fence(g);
+                    if (q < p.N) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            red_add_v4(dst + k * 32 + i, __uint_as_float(g[i]), __uint_as_float(g[i + 1]),
+                                       __uint_as_float(g[i + 2]), __uint_as_float(g[i + 3]));
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(dq_empty);
+        }
+        if (!ok && lane == 0) bwd_report(p, abort_flag, ST_BWD_ELEM_WAIT);
+        // dK and dV rows of this kv tile (zeros when no query attends to it);
+        // the tensor-memory loads are warp-collective, the stores per row
+        if (ok) {
+            const int64_t orow = (int64_t(b) * p.Hkv + hkv) * p.N + kv;
+#pragma unroll 1
+            for (int which = 0; which < 2; which++) {
+                uint4* dst = reinterpret_cast<uint4*>((which == 0 ? p.dV : p.dK) + orow * D);
+                const uint32_t col = which == 0 ? C::kColdV : C::kColdK;
+#pragma unroll 1
+                for (int k = 0; k < D / 32; k++) {
+                    uint32_t g[32];
+                    if (steps > 0) {
+                        tmem_ld_32x32b_x32(tmem + lanes + col + k * 32, g);
+                        tmem_wait_ld();
+                        reg_fence(g);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; i++) g[i] = 0u;
+                    }
+                    if (kv < p.N) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8)
+                            dst[(k * 32 + i) / 8] = make_uint4(
+                                pack_bf16x2(__uint_as_float(g[i]), __uint_as_float(g[i + 1])),
+                                pack_bf16x2(__uint_as_float(g[i + 2]), __uint_as_float(g[i + 3])),
+                                pack_bf16x2(__uint_as_float(g[i + 4]), __uint_as_float(g[i + 5])),
+                                pack_bf16x2(__uint_as_float(g[i + 6]), __uint_as_float(g[i + 7])));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+}  // namespace sa

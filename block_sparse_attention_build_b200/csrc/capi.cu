@@ -8,6 +8,7 @@
 
 #include "../../include/sparse_attn.h"
 #include "fwd_sm100.cuh"
+#include "runtime.h"
 #include "tma_host.h"
 
 namespace sa {
@@ -202,6 +203,17 @@ int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* m
 }
 
 }  // namespace
+
+int device_status_word(int32_t** out) { return status_word(out); }
+
+long long wait_limit_cycles()
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    return g_timeout;
+}
+
+int device_sm_count() { return sm_count(); }
+
 }  // namespace sa
 
 extern "C" int sparse_attn_fwd(const void* Q, const void* K, const void* V, const sa_block_mask* mask,

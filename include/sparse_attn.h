@@ -216,6 +216,54 @@ int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void* V, const s
                             const sa_pattern* pattern, const sa_shape* shape, float scale, void* O, float* LSE,
                             void* stream);
 
+/*
+ * Transpose a compiled block mask: for every kv tile c, the ascending list of
+ * query tiles whose list holds c, with the same full flags.  The result uses
+ * the sa_block_mask fields with rows and columns swapped: kv_count[c] is the
+ * number of query tiles listed for kv tile c, kv_index[c*T + e] the e-th of
+ * them (-1 after the last), kv_full[c*T + e] its flag (0 after the last).
+ * Host-only; `rows` as written by sparse_attn_build_block_mask, `cols` with
+ * caller-owned host arrays of capacity cols->n_q_tiles x cols->n_kv_tiles, both
+ * at least T (else SA_ERR_BUFFER_TOO_SMALL).  SA_ERR_INVALID_ARG for null
+ * arguments or an inconsistent input (counts or indices out of range).
+ */
+int sparse_attn_transpose_block_mask(const sa_block_mask* rows, sa_block_mask* cols);
+
+/* Device workspace bytes that sparse_attn_bwd needs for `shape`:
+ * 4 B * Hq * N (LSE in base 2) + 4 B * Hq * N (row term) + 4 B * Hq * N * D
+ * (fp32 dQ accumulator), each rounded up to 256 bytes. */
+int sparse_attn_bwd_workspace(const sa_shape* shape, size_t* bytes);
+
+/*
+ * Backward pass: the gradients dQ, dK, dV of the attention computed by
+ * sparse_attn_fwd, for an upstream gradient dO.  The pages print no backward
+ * pass; this is the chain rule through the masked softmax of the
+ * "Sparse-трансформеры" page, section "Как это выглядит в коде": with P the
+ * softmax weights of each query over its allowed keys,
+ *   dV = P^T dO,  dS = P * (dO V^T - rowsum(dO * O)),
+ *   dQ = scale * dS K,  dK = scale * dS^T Q,
+ * and for grouped heads dK, dV summed over the query heads of the group.
+ *
+ * All tensors in DEVICE memory, contiguous, 16-byte aligned:
+ *   Q, O, dO, dQ [B, Hq, N, D] bf16;  K, V, dK, dV [B, Hkv, N, D] bf16;
+ *   LSE [B, Hq, N] fp32 as written by sparse_attn_fwd (natural log).
+ *   mask_t     the TRANSPOSED block mask (sparse_attn_transpose_block_mask of
+ *              the pattern's mask) with its arrays in device memory; block 128
+ *   pattern    the pattern the mask was compiled from (partial tiles are
+ *              masked element by element from it)
+ *   workspace  device memory of at least sparse_attn_bwd_workspace bytes,
+ *              256-byte aligned; caller-owned, contents need not be preserved
+ * Launches three kernels on `stream` and returns without waiting; the
+ * workspace must not be reused until they finish.  The caller owns every
+ * buffer.  Errors as sparse_attn_fwd, plus SA_ERR_UNSUPPORTED for a mask block
+ * other than 128 and SA_ERR_BUFFER_TOO_SMALL for a short workspace; a bounded
+ * wait that expires inside the kernel sets the status word that
+ * sparse_attn_check_device reports.
+ */
+int sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
+                    const sa_block_mask* mask_t, const sa_pattern* pattern, const sa_shape* shape, float scale,
+                    void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes, void* stream);
+
 const char* sparse_attn_status_string(int status);
 
 /* ABI version: major * 10000 + minor * 100 + patch. */

@@ -156,3 +156,67 @@ def test_fwd_heads_argument_errors_without_gpu():
     rc = sa.lib.sparse_attn_fwd_heads(fake, fake, fake, (sa._BlockMask * 1)(m), (sa._Pattern * 1)(p), 1, None,
                                       ctypes.byref(sa._Shape(1, 2, 2, 100, 128)), 0.125, fake, fake, None)
     assert rc == sa.SA_ERR_INVALID_ARG                                               # no head table
+
+
+def transpose_of_oracle(p, N, b):
+    """The oracle's brute-force classification, read column by column."""
+    c, i, f = oracle.block_mask(opattern(p), N, b)
+    T = len(c)
+    tc = np.zeros(T, dtype=np.int32)
+    ti = np.full((T, T), -1, dtype=np.int32)
+    tf = np.zeros((T, T), dtype=np.uint8)
+    for r in range(T):
+        for e in range(c[r]):
+            col = i[r, e]
+            ti[col, tc[col]] = r
+            tf[col, tc[col]] = f[r, e]
+            tc[col] += 1
+    return tc, ti, tf
+
+
+@pytest.mark.parametrize("p,N,b", SWEEP[::3])
+def test_transposed_mask_matches_oracle(p, N, b):
+    m = sa.transpose_block_mask(sa.build_block_mask(p, N, b))
+    tc, ti, tf = transpose_of_oracle(p, N, b)
+    assert np.array_equal(m.counts, tc) and np.array_equal(m.index, ti) and np.array_equal(m.full, tf)
+    assert m.n_live == tc.sum() and m.block == b
+
+
+def test_transpose_errors():
+    good = sa.build_block_mask(sa.Pattern(window=300, sinks=4), 1000, 128)
+    bad_index = good.index.copy()
+    bad_index[3, 0] = 99
+    broken = sa.BlockMask(good.counts, bad_index, good.full, 128, good.n_live, good.n_full, good.max_per_row, 1000)
+    with pytest.raises(sa.SparseAttnError) as e:
+        sa.transpose_block_mask(broken)
+    assert e.value.status == sa.SA_ERR_INVALID_ARG
+    small = sa._BlockMask(2, 2, 0, 0, 0, 0, None, None, None)
+    rc = sa.lib.sparse_attn_transpose_block_mask(ctypes.byref(good._c()), ctypes.byref(small))
+    assert rc == sa.SA_ERR_BUFFER_TOO_SMALL
+
+
+def test_bwd_argument_errors_without_gpu():
+    """Checks that return before any CUDA call."""
+    p = sa.Pattern(window=8)._c()
+    m = sa._BlockMask(1, 1, 128, 1, 1, 0, 16, 16, 16)
+    fake = 1 << 20
+    ws_ok = sa.bwd_workspace_bytes(1, 2, 2, 100, 128)
+
+    def call(shape, scale=0.125, mask=m, pat=p, ptr=fake, ws=fake, ws_bytes=ws_ok):
+        return sa.lib.sparse_attn_bwd(ptr, ptr, ptr, ptr, ptr, ptr, ctypes.byref(mask), ctypes.byref(pat),
+                                      ctypes.byref(sa._Shape(*shape)), scale, ptr, ptr, ptr, ws, ws_bytes, None)
+
+    assert call((1, 2, 2, 100, 96)) == sa.SA_ERR_UNSUPPORTED                       # D
+    assert call((1, 2, 2, 100, 128), scale=0.0) == sa.SA_ERR_INVALID_ARG
+    assert call((1, 3, 2, 100, 128)) == sa.SA_ERR_UNSUPPORTED                      # Hq % Hkv
+    assert call((1, 2, 2, 1000, 128)) == sa.SA_ERR_MASK_MISMATCH                   # T != ceil(N / 128)
+    m64 = sa._BlockMask(2, 2, 64, 1, 1, 0, 16, 16, 16)
+    assert call((1, 2, 2, 100, 128), mask=m64) == sa.SA_ERR_UNSUPPORTED            # block 64
+    assert call((1, 2, 2, 100, 128), ptr=fake + 8) == sa.SA_ERR_MISALIGNED
+    assert call((1, 2, 2, 100, 128), ws=fake + 16) == sa.SA_ERR_MISALIGNED         # workspace 256-aligned
+    assert call((1, 2, 2, 100, 128), ws_bytes=ws_ok - 1) == sa.SA_ERR_BUFFER_TOO_SMALL
+    assert call((0, 2, 2, 100, 128)) == sa.SA_OK
+    bad = sa.Pattern(window=8, causal=0)._c()
+    assert call((1, 2, 2, 100, 128), pat=bad) == sa.SA_ERR_UNSUPPORTED
+    rows = 1 * 2 * 100
+    assert ws_ok >= 2 * rows * 4 + rows * 128 * 4
