@@ -17,6 +17,12 @@ e2e        the same metric through the host-buffer C ABI call (pinned host
            Q/K/V in, O/LSE out, copies inside the timed region).
 cpu_baseline  the fp64 CPU oracle on a bounded row sample, host cores.
 
+With --pass bwd one step is one backward pass (three launches: prep, the
+tensor-core kernel, dQ conversion) for an upstream gradient dO, with the
+forward's O and LSE computed once before timing; value counts 10 * D useful
+FLOP per allowed pair (S, dP, dV, dK, dQ) and the roofline takes the whole
+step's device time (the launch list in profiles/ gives each kernel's share).
+
 With --impl reference the oracle is the timed program (rank 0 only).
 Multi-GPU (torchrun): every rank runs its own batch of the workload (the
 problems are independent; no collective on the data path); value is the sum
@@ -44,6 +50,7 @@ import synth  # noqa: E402
 from synth.workloads import HEADLINE, WORKLOADS  # noqa: E402
 
 METRIC = "block-sparse attn fwd useful TFLOP/s (bf16, 1 B200) and % of tensor peak"
+METRIC_BWD = "block-sparse attn bwd useful TFLOP/s (bf16, 1 B200) and % of tensor peak"
 UNIT = "TFLOP/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
@@ -208,6 +215,18 @@ class OracleSample:
 
 def run_reference(args, w):
     if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    if args.which == "bwd":
+        # whole heads of the fp64 backward oracle, about 20 s in all
+        cpu = oracle_bwd_baseline(w, 20.0)
+        line = {
+            "impl": "reference", "metric": METRIC_BWD, "value": cpu["value"], "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, args.gpus, {"pass": "bwd"}), "cpu_baseline": cpu,
+            "e2e": {"value": cpu["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line))
         return 0
     per_step = min(2.0, max(0.01, 120.0 / (args.steps + args.warmup)))
     sample = OracleSample(w, per_step)
@@ -397,6 +416,173 @@ def run_gpu(args, w):
     return 0
 
 
+def run_gpu_bwd(args, w):
+    """The backward pass of the workload: one step = sparse_attn_bwd over the batch."""
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_build_b200 as sa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    if w.block != 128:
+        raise SystemExit("the backward pass takes block-128 masks")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    p, mask_h, pairs, _, _, _ = workload_counts(w)
+    useful = 10.0 * w.D * pairs * w.B * w.Hq
+    executed = 10.0 * w.D * w.block * w.block * mask_h.n_live * w.B * w.Hq
+    mask = mask_h.to_device(dev)
+    mask_t = sa.transpose_block_mask(mask_h).to_device(dev)
+
+    seed = rank_seed(w, rank)
+    q, k, v = synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=seed)
+    do = synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=seed + 7919)[0]
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    Q0, K0, V0, dO0 = to_dev(q), to_dev(k), to_dev(v), to_dev(do)
+    O0, L0 = sa.fwd(Q0, K0, V0, mask, p, scale=w.scale)
+    ws_bytes = sa.bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.D)
+    qo = w.B * w.Hq * w.N * w.D * 2
+    kv = w.B * w.Hkv * w.N * w.D * 2
+    set_bytes = 4 * qo + 4 * kv + w.B * w.Hq * w.N * 4 + ws_bytes  # Q O dO dQ, K V dK dV, LSE, workspace
+    n_sets = args.sets if args.sets > 0 else max(2, min(8, math.ceil(3 * L2_BYTES / set_bytes)))
+    sets = []
+    for i in range(n_sets):
+        ins = (Q0, K0, V0, O0, L0, dO0) if i == 0 else tuple(t.clone() for t in (Q0, K0, V0, O0, L0, dO0))
+        outs = (torch.empty_like(Q0), torch.empty_like(K0), torch.empty_like(V0),
+                torch.empty(ws_bytes, dtype=torch.uint8, device=dev))
+        sets.append((ins, outs))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        (Qi, Ki, Vi, Oi, Li, dOi), (dQi, dKi, dVi, Wi) = sets[i % n_sets]
+        sa.bwd(Qi, Ki, Vi, Oi, Li, dOi, mask_t, p, scale=w.scale, dq=dQi, dk=dKi, dv=dVi, workspace=Wi,
+               stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if sa.check_device(stream) != sa.SA_OK:
+        raise SystemExit("device status not ok after warm-up")
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    local_ms = t_start.elapsed_time(t_end)
+    status = sa.check_device(stream)
+    if status != sa.SA_OK:
+        raise SystemExit(f"device status {sa.status_string(status)}")
+    elapsed_ms = max_over_ranks(local_ms, dist if world > 1 else None, dev)
+    step_ms = local_ms / args.steps
+
+    # end to end: pinned host inputs in, gradients out, every step
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: t.cpu().pin_memory()
+        hins = [pin(t) for t in (Q0, K0, V0, O0, L0, dO0)]
+        houts = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (Q0, K0, V0)]
+        dins = [torch.empty_like(t) for t in (Q0, K0, V0, O0, L0, dO0)]
+        douts = [torch.empty_like(t) for t in (Q0, K0, V0)]
+        W = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            for d, h in zip(dins, hins):
+                d.copy_(h, non_blocking=True)
+            sa.bwd(*dins, mask_t, p, scale=w.scale, dq=douts[0], dk=douts[1], dv=douts[2], workspace=W,
+                   stream=stream)
+            for h, d in zip(houts, douts):
+                h.copy_(d, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 20))
+        for _ in range(2):
+            e2e_step()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
+        e2e = {"value": job_tflops(world, useful, e2e_steps, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hins),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in houts), "steps": e2e_steps,
+               "ms_per_step": e2e_ms / e2e_steps}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    value = job_tflops(world, useful, args.steps, elapsed_ms)
+    achieved = executed / (step_ms * 1e-3) / 1e12
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_bwd_baseline(w, args.cpu_seconds)
+    line = {
+        "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(w, world, {
+            "pass": "bwd",
+            "l2": f"{n_sets} rotating input sets of {set_bytes / 1e6:.1f} MB "
+                  f"({n_sets * set_bytes / 1e6:.0f} MB > {L2_BYTES / 1e6:.0f} MB L2)",
+            "live_tiles": int(mask_h.n_live), "allowed_pairs_per_head": int(pairs)}),
+        "useful_frac_of_peak": value / world / peak,
+        "executed_tflops": job_tflops(world, executed, args.steps, elapsed_ms),
+        "peak_kind": f"bf16 dense, {peak_kind} ({peak} TFLOP/s burst)",
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "backward step: bwd_prep_kernel + bwd_kernel<D> + bwd_dq_kernel",
+                     "mean_step_us": step_ms * 1e3, "algorithmic_flop_per_step": executed},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def oracle_bwd_baseline(w, target_s: float):
+    """The fp64 backward oracle on whole heads of the workload (host cores),
+    as many heads as fit in about target_s seconds (at least one)."""
+    import oracle
+    p = oracle.Pattern(**w.pattern_args())
+    q, k, v = synth.qkv(1, 1, 1, w.N, w.D, seed=w.seed)
+    do = synth.qkv(1, 1, 1, w.N, w.D, seed=w.seed + 7919)[0]
+    pairs = oracle.count_pairs(p, w.N)
+    heads, t0 = 0, time.perf_counter()
+    while True:
+        oracle.attention_bwd(q, k, v, do, p, w.scale)
+        heads += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s or dt / heads * (heads + 1) > 2 * target_s:
+            break
+    rate = 10.0 * w.D * pairs * heads / dt / 1e12
+    return {"value": rate, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{heads} whole head(s) of N={w.N} (dQ, dK, dV in fp64), {dt:.1f} s"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -408,12 +594,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling runs)")
     ap.add_argument("--sets", type=int, default=0, help="rotating input sets (0: enough to exceed L2)")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"])
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.which == "bwd":
+        return run_gpu_bwd(args, w)
     return run_gpu(args, w)
 
 

@@ -21,9 +21,10 @@
 //                    the fp32 accumulator with vector reductions;
 //   bwd_dq_kernel    dQ accumulator -> bf16.
 //
-// bwd_kernel, 192 threads: warps 0-3 the element-wise work (one kv row per
-// thread, tensor-memory lane = kv row), warp 4 the TMA producer, warp 5 tensor
-// memory allocation and the single MMA-issuing lane.  Per step (one query
+// bwd_kernel, 320 threads: warps 0-7 the element-wise work (two threads per
+// kv row, each one half of the columns; tensor-memory lane = kv row), warp 8
+// the TMA producer, warp 9 tensor memory allocation and the single
+// MMA-issuing lane.  Per step (one query
 // tile of one head):
 //   Sᵀ = K Qᵀ, dPᵀ = V dOᵀ                 tcgen05 SS, fp32 in tensor memory
 //   Pᵀ = exp2(Sᵀ·scale·log2e − LSE₂)      masked on partial tiles; bf16 back
@@ -31,7 +32,10 @@
 //   dSᵀ = Pᵀ ∘ (dPᵀ − Δ) · scale           bf16 into shared memory
 //   dV += Pᵀ dO  (TS: Pᵀ from tensor memory), dK += dSᵀ Q  (SS)
 //   dQ  = dS K   (SS, dS read MN-major from the same shared tile) into the dPᵀ
-//                columns, then read out and reduced into global memory.
+//                columns, then read out (releasing tensor memory for the next
+//                step's MMAs) and reduced into global memory through a
+//                shared-memory transpose, so that each reduction instruction
+//                covers whole 128-byte lines.
 // Every wait is bounded; on expiry a role sets a status bit, raises an abort
 // flag and leaves its loop; the MMA lane drains its MMAs and the producer its
 // copies before tensor memory is freed.
@@ -46,7 +50,10 @@
 
 namespace sa {
 
-constexpr int kBwdThreads = 192;
+constexpr int kBwdThreads = 320;
+constexpr int kBwdElemThreads = 256;  // warps 0-7
+constexpr int kBwdProducerWarp = 8;
+constexpr int kBwdMmaWarp = 9;
 constexpr int kBwdTile = 128;  // query and kv tile edge (the block mask's block)
 
 enum : int32_t {
@@ -86,7 +93,7 @@ struct BwdCfg {
     static constexpr int kNumBars = 10;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tensor-memory base, abort flag
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
-    static constexpr uint32_t kColS = 0;         // Sᵀ (fp32), then Pᵀ (bf16 pairs) in its first 64 columns
+    static constexpr uint32_t kColS = 0;         // Sᵀ (fp32), then Pᵀ (bf16 pairs) in columns 0-31 and 64-95
     static constexpr uint32_t kColdP = 128;      // dPᵀ (fp32), then the step's dQ tile
     static constexpr uint32_t kColdV = 256;
     static constexpr uint32_t kColdK = 256 + D;
@@ -213,9 +220,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t* qd_full = bars + 1;     // [2] Q and dO of a step landed
     uint64_t* qd_empty = bars + 3;    // [2] the step's dV and dK MMAs are done with them
     uint64_t* s_full = bars + 5;      // Sᵀ and dPᵀ are in tensor memory
-    uint64_t* ds_full = bars + 6;     // Pᵀ (tensor memory) and dSᵀ (shared memory) written (128 threads)
+    uint64_t* ds_full = bars + 6;     // Pᵀ (tensor memory) and dSᵀ (shared memory) written (256 threads)
     uint64_t* dq_full = bars + 7;     // the step's dQ tile is in tensor memory (and every earlier MMA done)
-    uint64_t* dq_empty = bars + 8;    // the dQ tile has been read (128 threads)
+    uint64_t* dq_empty = bars + 8;    // the dQ tile has been read out of tensor memory (256 threads)
     uint64_t* drain = bars + 9;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -237,18 +244,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&qd_empty[x], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(ds_full, 128);
+        mbar_init(ds_full, kBwdElemThreads);
         mbar_init(dq_full, 1);
-        mbar_init(dq_empty, 128);
+        mbar_init(dq_empty, kBwdElemThreads);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 5) {
+    if (warp == kBwdMmaWarp) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == kBwdProducerWarp && lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmdO);
         tma_prefetch_desc(&tmK);
@@ -269,7 +276,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         hq = hkv * p.group + h;
     };
 
-    if (warp == 4) {
+    if (warp == kBwdProducerWarp) {
         // ================================================================ producer (one lane)
         if (lane == 0 && steps > 0) {
             const uint64_t pol = policy_evict_last();
@@ -305,7 +312,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int j = issued > 2 ? issued - 2 : 0; j < issued; j++) ok &= mbar_wait(&qd_full[j & 1], (j >> 1) & 1, lim);
             if (!ok) bwd_report(p, abort_flag, ST_BWD_DRAIN_WAIT);
         }
-    } else if (warp == 5) {
+    } else if (warp == kBwdMmaWarp) {
         // ================================================================ MMA issuer
         // The warp runs converged; one elected lane issues each MMA and commit.
         if (steps > 0) {
@@ -360,12 +367,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 ok = wait(ds_full, j & 1);
                 if (!ok || __any_sync(0xffffffffu, *abort_flag != 0)) break;
                 tc_fence_after_sync();
-                // dV += Pᵀ dO (Pᵀ bf16 in the Sᵀ columns) and dK += dSᵀ Q (M = kv rows, N = D, K = query rows)
+                // dV += Pᵀ dO and dK += dSᵀ Q (M = kv rows, N = D, K = query rows);
+                // Pᵀ bf16 pairs: query columns 64h .. 64h+63 packed in Sᵀ columns 64h .. 64h+31
 #pragma unroll
                 for (int kk = 0; kk < kBwdTile / 16; kk++) {
                     if (elect_one())
-                        mma_ts(tmem + C::kColdV, tmem + C::kColS + kk * 8, desc_from_halves(o_mn + bo + mn(kk), hi),
-                               id_kv, (j > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts(tmem + C::kColdV, tmem + C::kColS + (kk / 4) * 64 + (kk % 4) * 8,
+                               desc_from_halves(o_mn + bo + mn(kk), hi), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
                     __syncwarp();
                 }
 #pragma unroll
@@ -392,14 +400,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!wait(drain, 0) && lane == 0) bwd_report(p, abort_flag, ST_BWD_DRAIN_WAIT);
         }
     } else {
-        // ================================================================ element-wise warps 0-3
+        // ================================================================ element-wise warps 0-7
+        // Warp w serves tensor-memory lanes 32 (w % 4) .. +31 (kv rows of Sᵀ,
+        // dPᵀ, dK, dV; query rows of dQ) and column half h = w / 4: query
+        // columns 64h .. 64h+63 of Sᵀ / dPᵀ, columns h D/2 .. of dQ, dK, dV.
         // Each warp decides to leave its loop as a whole (every test goes
-        // through a vote); the four warps never wait on one another except
-        // through bounded mbarrier waits.
-        const int t = threadIdx.x;  // kv row of Sᵀ / dPᵀ / dK / dV, query row of dQ (tensor-memory lane)
-        const uint32_t lanes = static_cast<uint32_t>(warp * 32) << 16;
+        // through a vote); the warps never wait on one another except through
+        // bounded mbarrier waits.
+        const int quarter = warp % 4;
+        const int half = warp / 4;
+        const int t = quarter * 32 + lane;  // kv row (and query row of dQ) of this thread
+        const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
         const int kv = c * kBwdTile + t;
         const bool kv_ragged = (c + 1) * kBwdTile > p.N;
+        constexpr int kHalfD = D / 2;
+        // this warp's rows of dSᵀ panel `half`: free between a step's dq_full and
+        // the next step's element-wise pass, used to stage dQ for coalesced reductions
+        uint8_t* stage = sdS + half * C::kPanel + quarter * 32 * 128;
         bool ok = true;
         for (int j = 0; j < steps; j++) {
             int hq, r;
@@ -407,11 +424,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             step_of(j, hq, r, full);
             const int q0 = r * kBwdTile;
             const int64_t qrow0 = (int64_t(b) * p.Hq + hq) * p.N;
-            // LSE₂ and Δ of query column 32cc + lane, handed to the other lanes by shuffles
-            float lse_r[4], dl_r[4];
+            // LSE₂ and Δ of query column 64 half + 32 cc + lane, handed to the other lanes by shuffles
+            float lse_r[2], dl_r[2];
 #pragma unroll
-            for (int cc = 0; cc < 4; cc++) {
-                const int q = q0 + cc * 32 + lane;
+            for (int cc = 0; cc < 2; cc++) {
+                const int q = q0 + half * 64 + cc * 32 + lane;
                 lse_r[cc] = q < p.N ? __ldg(&p.lse2[qrow0 + q]) : INFINITY;
                 dl_r[cc] = q < p.N ? __ldg(&p.delta[qrow0 + q]) : 0.f;
             }
@@ -420,13 +437,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after_sync();
             const bool masked = !full || kv_ragged || q0 + kBwdTile > p.N;
 #pragma unroll 1
-            for (int cc = 0; cc < kBwdTile / 32; cc++) {
+            for (int cc = 0; cc < 2; cc++) {
+                const int col = half * 64 + cc * 32;  // first query column of the chunk
                 uint32_t s[32], d[32];
-                tmem_ld_32x32b_x32(tmem + lanes + C::kColS + cc * 32, s);
-                tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + cc * 32, d);
-                const float lse_c = cc == 0 ? lse_r[0] : cc == 1 ? lse_r[1] : cc == 2 ? lse_r[2] : lse_r[3];
-                const float dl_c = cc == 0 ? dl_r[0] : cc == 1 ? dl_r[1] : cc == 2 ? dl_r[2] : dl_r[3];
-                const uint32_t allow = masked ? bwd_allow_word(p, q0 + cc * 32, kv) : 0xffffffffu;
+                tmem_ld_32x32b_x32(tmem + lanes + C::kColS + col, s);
+                tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + col, d);
+                const float lse_c = cc == 0 ? lse_r[0] : lse_r[1];
+                const float dl_c = cc == 0 ? dl_r[0] : dl_r[1];
+                const uint32_t allow = masked ? bwd_allow_word(p, q0 + col, kv) : 0xffffffffu;
                 tmem_wait_ld();
                 reg_fence(s);
                 reg_fence(d);
@@ -446,13 +464,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     pk[i / 2] = pack_bf16x2(p0, p1);
                     gk[i / 2] = pack_bf16x2(g0, g1);
                 }
-                // Pᵀ (bf16 pairs) over Sᵀ columns already read
-                tmem_st_32x32b_x16(tmem + lanes + C::kColS + cc * 16, pk);
-                // dSᵀ row t, query columns 32cc..32cc+31: four 16-byte units of panel cc / 2
-                uint8_t* rowp = sdS + (cc / 2) * C::kPanel + t * 128;
+                // Pᵀ (bf16 pairs) over Sᵀ columns this warp has already read:
+                // query columns col .. col+31 go to packed columns 64 half + 16 cc
+                // .. +15, inside the half's own 64 columns (the other half's warps
+                // may still be reading theirs)
+                tmem_st_32x32b_x16(tmem + lanes + C::kColS + half * 64 + cc * 16, pk);
+                // dSᵀ row t, query columns col .. col+31: four 16-byte units of panel `half`
+                uint8_t* rowp = sdS + half * C::kPanel + t * 128;
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
-                    const int u = (cc % 2) * 4 + k;
+                    const int u = cc * 4 + k;
                     *reinterpret_cast<uint4*>(rowp + ((u ^ (t & 7)) << 4)) =
                         make_uint4(gk[4 * k], gk[4 * k + 1], gk[4 * k + 2], gk[4 * k + 3]);
                 }
@@ -464,55 +485,72 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(dq_full, j & 1, lim) && !*abort_flag);
             if (!ok) break;
             tc_fence_after_sync();
-            // dQ row q0 + t of head hq into the fp32 accumulator
-            {
-                const int q = q0 + t;
-                float* dst = p.dq_acc + (qrow0 + q) * D;
-#pragma unroll 1
-                for (int k = 0; k < D / 32; k++) {
-                    uint32_t g[32];
-                    tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + k * 32, g);
-                    tmem_wait_ld();
-                    reg_fence(g);
-                    if (q < p.N) {
+            // dQ rows of this warp, columns half * D/2 .. +D/2: all of it out of
+            // tensor memory first, so the next step's MMAs may start
+            uint32_t g[kHalfD];
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            red_add_v4(dst + k * 32 + i, __uint_as_float(g[i]), __uint_as_float(g[i + 1]),
-                                       __uint_as_float(g[i + 2]), __uint_as_float(g[i + 3]));
-                    }
-                }
+            for (int k = 0; k < kHalfD / 32; k++) {
+                uint32_t (&gc)[32] = *reinterpret_cast<uint32_t(*)[32]>(&g[32 * k]);
+                tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + half * kHalfD + k * 32, gc);
             }
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < kHalfD / 32; k++) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&g[32 * k]));
             tc_fence_before_sync();
             mbar_arrive(dq_empty);
+            // through shared memory: lane l holds row l of a 32 x 32 block; after
+            // the exchange each instruction adds 4 rows x 128 contiguous bytes
+#pragma unroll
+            for (int k = 0; k < kHalfD / 32; k++) {
+                __syncwarp();
+#pragma unroll
+                for (int u = 0; u < 8; u++)
+                    *reinterpret_cast<uint4*>(stage + lane * 128 + ((u ^ (lane & 7)) << 4)) =
+                        make_uint4(g[32 * k + 4 * u], g[32 * k + 4 * u + 1], g[32 * k + 4 * u + 2],
+                                   g[32 * k + 4 * u + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const int rr = 4 * i + lane / 8;  // row within the warp's 32
+                    const int u = lane % 8;
+                    const float4 v = *reinterpret_cast<const float4*>(stage + rr * 128 + ((u ^ (rr & 7)) << 4));
+                    const int q = q0 + quarter * 32 + rr;
+                    if (q < p.N)
+                        red_add_v4(p.dq_acc + (qrow0 + q) * D + half * kHalfD + k * 32 + 4 * u, v.x, v.y, v.z,
+                                   v.w);
+                }
+            }
+            __syncwarp();
         }
         if (!ok && lane == 0) bwd_report(p, abort_flag, ST_BWD_ELEM_WAIT);
-        // dK and dV rows of this kv tile (zeros when no query attends to it);
-        // the tensor-memory loads are warp-collective, the stores per row
+        // dK and dV rows of this kv tile, this warp's column half (zeros when no
+        // query attends to it); the tensor-memory loads are warp-collective,
+        // the stores per row
         if (ok) {
             const int64_t orow = (int64_t(b) * p.Hkv + hkv) * p.N + kv;
 #pragma unroll 1
             for (int which = 0; which < 2; which++) {
-                uint4* dst = reinterpret_cast<uint4*>((which == 0 ? p.dV : p.dK) + orow * D);
-                const uint32_t col = which == 0 ? C::kColdV : C::kColdK;
+                uint4* dst = reinterpret_cast<uint4*>((which == 0 ? p.dV : p.dK) + orow * D + half * kHalfD);
+                const uint32_t col = (which == 0 ? C::kColdV : C::kColdK) + half * kHalfD;
 #pragma unroll 1
-                for (int k = 0; k < D / 32; k++) {
-                    uint32_t g[32];
+                for (int k = 0; k < kHalfD / 32; k++) {
+                    uint32_t gg[32];
                     if (steps > 0) {
-                        tmem_ld_32x32b_x32(tmem + lanes + col + k * 32, g);
+                        tmem_ld_32x32b_x32(tmem + lanes + col + k * 32, gg);
                         tmem_wait_ld();
-                        reg_fence(g);
+                        reg_fence(gg);
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 32; i++) g[i] = 0u;
+                        for (int i = 0; i < 32; i++) gg[i] = 0u;
                     }
                     if (kv < p.N) {
 #pragma unroll
                         for (int i = 0; i < 32; i += 8)
                             dst[(k * 32 + i) / 8] = make_uint4(
-                                pack_bf16x2(__uint_as_float(g[i]), __uint_as_float(g[i + 1])),
-                                pack_bf16x2(__uint_as_float(g[i + 2]), __uint_as_float(g[i + 3])),
-                                pack_bf16x2(__uint_as_float(g[i + 4]), __uint_as_float(g[i + 5])),
-                                pack_bf16x2(__uint_as_float(g[i + 6]), __uint_as_float(g[i + 7])));
+                                pack_bf16x2(__uint_as_float(gg[i]), __uint_as_float(gg[i + 1])),
+                                pack_bf16x2(__uint_as_float(gg[i + 2]), __uint_as_float(gg[i + 3])),
+                                pack_bf16x2(__uint_as_float(gg[i + 4]), __uint_as_float(gg[i + 5])),
+                                pack_bf16x2(__uint_as_float(gg[i + 6]), __uint_as_float(gg[i + 7])));
                     }
                 }
             }
@@ -521,7 +559,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kBwdMmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, C::kTmemCols);
     }
