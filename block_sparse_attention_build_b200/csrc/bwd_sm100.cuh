@@ -27,15 +27,17 @@
 // MMA-issuing lane.  Per step (one query
 // tile of one head):
 //   Sᵀ = K Qᵀ, dPᵀ = V dOᵀ                 tcgen05 SS, fp32 in tensor memory
-//   Pᵀ = exp2(Sᵀ·scale·log2e − LSE₂)      masked on partial tiles; bf16 back
-//                                           into the Sᵀ columns
-//   dSᵀ = Pᵀ ∘ (dPᵀ − Δ) · scale           bf16 into shared memory
-//   dV += Pᵀ dO  (TS: Pᵀ from tensor memory), dK += dSᵀ Q  (SS)
-//   dQ  = dS K   (SS, dS read MN-major from the same shared tile) into the dPᵀ
-//                columns, then read out (releasing tensor memory for the next
-//                step's MMAs) and reduced into global memory through a
-//                shared-memory transpose, so that each reduction instruction
-//                covers whole 128-byte lines.
+//   Pᵀ = exp2(Sᵀ·scale·log2e − LSE₂)      masked on partial tiles
+//   dSᵀ = Pᵀ ∘ (dPᵀ − Δ) · scale           both bf16 back into the Sᵀ columns of
+//                                           tensor memory; dSᵀ also to shared memory
+//   dV += Pᵀ dO, dK += dSᵀ Q               TS: A from tensor memory
+//   dQᵀ = Kᵀ dSᵀ                            SS, both operands MN-major, into the dPᵀ
+//                columns with lanes = features; read out (releasing tensor
+//                memory for the next step's MMAs) and reduced into global
+//                memory, each warp instruction adding one query row's 32
+//                consecutive features (one 128-byte line).
+// Shared memory carries only the SS operands, the TMA fills and the dSᵀ tile:
+// its bandwidth, not the tensor pipe, is what bounds a step of this design.
 // Every wait is bounded; on expiry a role sets a status bit, raises an abort
 // flag and leaves its loop; the MMA lane drains its MMAs and the producer its
 // copies before tensor memory is freed.
@@ -93,8 +95,8 @@ struct BwdCfg {
     static constexpr int kNumBars = 10;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tensor-memory base, abort flag
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
-    static constexpr uint32_t kColS = 0;         // Sᵀ (fp32), then Pᵀ (bf16 pairs) in columns 0-31 and 64-95
-    static constexpr uint32_t kColdP = 128;      // dPᵀ (fp32), then the step's dQ tile
+    static constexpr uint32_t kColS = 0;         // Sᵀ (fp32), then Pᵀ and dSᵀ (bf16 pairs), 16 columns each per 32
+    static constexpr uint32_t kColdP = 128;      // dPᵀ (fp32), then the step's dQᵀ tile (lanes = features)
     static constexpr uint32_t kColdV = 256;
     static constexpr uint32_t kColdK = 256 + D;
     static constexpr uint32_t kTmemCols = 512;
@@ -137,10 +139,9 @@ __device__ __forceinline__ uint32_t bwd_allow_word(const BwdParams& p, int qb, i
     return m & in_range;
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d)
+__device__ __forceinline__ void red_add_f32(float* addr, float a)
 {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
 }
 
 // One warp per query row: Δ = Σ_d dO·O (fp32 from the bf16 tensors), LSE₂ =
@@ -318,7 +319,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (steps > 0) {
             constexpr uint32_t id_s = idesc_bf16_f32(kBwdTile, kBwdTile, false, false);
             constexpr uint32_t id_kv = idesc_bf16_f32(kBwdTile, D, false, true);
-            constexpr uint32_t id_q = idesc_bf16_f32(kBwdTile, D, true, true);
+            // dQᵀ = Kᵀ dSᵀ: M = 128 feature rows (at D = 64 the upper 64 read the V tile
+            // and are never used), N = 128 query rows, both operands MN-major
+            constexpr uint32_t id_q = idesc_bf16_f32(kBwdTile, kBwdTile, true, true);
             constexpr uint32_t kTileU = C::kTileBytes >> 4;  // descriptor units (16 bytes)
             const uint64_t d0 = smem_desc_sw128(smem_addr(sK), 16, 1024);
             const uint32_t hi = static_cast<uint32_t>(d0 >> 32);
@@ -329,7 +332,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint32_t q_mn = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sQ), C::kPanel, 1024));
             const uint32_t o_km = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sdO), 16, 1024));
             const uint32_t o_mn = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sdO), C::kPanel, 1024));
-            const uint32_t s_km = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sdS), 16, 1024));
             const uint32_t s_mn = static_cast<uint32_t>(smem_desc_sw128(smem_addr(sdS), C::kPanel, 1024));
             // k-step offsets (16 elements of the contraction), in descriptor units
             auto km = [](int kk) { return static_cast<uint32_t>(((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4); };
@@ -367,29 +369,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 ok = wait(ds_full, j & 1);
                 if (!ok || __any_sync(0xffffffffu, *abort_flag != 0)) break;
                 tc_fence_after_sync();
-                // dV += Pᵀ dO and dK += dSᵀ Q (M = kv rows, N = D, K = query rows);
-                // Pᵀ bf16 pairs: query columns 64h .. 64h+63 packed in Sᵀ columns 64h .. 64h+31
+                // dV += Pᵀ dO and dK += dSᵀ Q (M = kv rows, N = D, K = query rows), A
+                // from tensor memory: query columns 32c .. 32c+31 (c = kk / 2) hold
+                // Pᵀ in packed columns 32c .. 32c+15 and dSᵀ in 32c+16 .. 32c+31
 #pragma unroll
                 for (int kk = 0; kk < kBwdTile / 16; kk++) {
                     if (elect_one())
-                        mma_ts(tmem + C::kColdV, tmem + C::kColS + (kk / 4) * 64 + (kk % 4) * 8,
+                        mma_ts(tmem + C::kColdV, tmem + C::kColS + (kk / 2) * 32 + (kk % 2) * 8,
                                desc_from_halves(o_mn + bo + mn(kk), hi), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
                     __syncwarp();
                 }
 #pragma unroll
                 for (int kk = 0; kk < kBwdTile / 16; kk++) {
                     if (elect_one())
-                        mma_ss(tmem + C::kColdK, desc_from_halves(s_km + km(kk), hi),
+                        mma_ts(tmem + C::kColdK, tmem + C::kColS + (kk / 2) * 32 + 16 + (kk % 2) * 8,
                                desc_from_halves(q_mn + bo + mn(kk), hi), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
                     __syncwarp();
                 }
                 commit(&qd_empty[buf]);
-                // dQ = dS K (M = query rows, N = D, K = kv rows), into the dPᵀ columns
+                // dQᵀ = Kᵀ dSᵀ (M = feature rows, N = query rows, K = kv rows), into the dPᵀ columns
 #pragma unroll
                 for (int kk = 0; kk < kBwdTile / 16; kk++) {
                     if (elect_one())
-                        mma_ss(tmem + C::kColdP, desc_from_halves(s_mn + mn(kk), hi),
-                               desc_from_halves(k_mn + mn(kk), hi), id_q, kk > 0 ? 1u : 0u);
+                        mma_ss(tmem + C::kColdP, desc_from_halves(k_mn + mn(kk), hi),
+                               desc_from_halves(s_mn + mn(kk), hi), id_q, kk > 0 ? 1u : 0u);
                     __syncwarp();
                 }
                 commit(dq_full);
@@ -414,9 +417,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int kv = c * kBwdTile + t;
         const bool kv_ragged = (c + 1) * kBwdTile > p.N;
         constexpr int kHalfD = D / 2;
-        // this warp's rows of dSᵀ panel `half`: free between a step's dq_full and
-        // the next step's element-wise pass, used to stage dQ for coalesced reductions
-        uint8_t* stage = sdS + half * C::kPanel + quarter * 32 * 128;
         bool ok = true;
         for (int j = 0; j < steps; j++) {
             int hq, r;
@@ -464,11 +464,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     pk[i / 2] = pack_bf16x2(p0, p1);
                     gk[i / 2] = pack_bf16x2(g0, g1);
                 }
-                // Pᵀ (bf16 pairs) over Sᵀ columns this warp has already read:
-                // query columns col .. col+31 go to packed columns 64 half + 16 cc
-                // .. +15, inside the half's own 64 columns (the other half's warps
-                // may still be reading theirs)
-                tmem_st_32x32b_x16(tmem + lanes + C::kColS + half * 64 + cc * 16, pk);
+                // Pᵀ and dSᵀ (bf16 pairs) over the 32 Sᵀ columns of this chunk, just
+                // read by this thread: Pᵀ in col .. col+15, dSᵀ in col+16 .. col+31
+                tmem_st_32x32b_x16(tmem + lanes + C::kColS + col, pk);
+                tmem_st_32x32b_x16(tmem + lanes + C::kColS + col + 16, gk);
                 // dSᵀ row t, query columns col .. col+31: four 16-byte units of panel `half`
                 uint8_t* rowp = sdS + half * C::kPanel + t * 128;
 #pragma unroll
@@ -485,42 +484,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(dq_full, j & 1, lim) && !*abort_flag);
             if (!ok) break;
             tc_fence_after_sync();
-            // dQ rows of this warp, columns half * D/2 .. +D/2: all of it out of
-            // tensor memory first, so the next step's MMAs may start
-            uint32_t g[kHalfD];
-#pragma unroll
-            for (int k = 0; k < kHalfD / 32; k++) {
-                uint32_t (&gc)[32] = *reinterpret_cast<uint32_t(*)[32]>(&g[32 * k]);
-                tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + half * kHalfD + k * 32, gc);
-            }
+            // dQᵀ: lane = feature d = 32 quarter + lane, columns = query rows 64 half
+            // .. +63.  All of it out of tensor memory first, so the next step's
+            // MMAs may start; then each reduction instruction adds one query
+            // row's 32 consecutive features: 128 contiguous bytes per warp.
+            uint32_t g[64];
+            tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+            tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
             tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < kHalfD / 32; k++) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&g[32 * k]));
+            reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+            reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&g[32]));
             tc_fence_before_sync();
             mbar_arrive(dq_empty);
-            // through shared memory: lane l holds row l of a 32 x 32 block; after
-            // the exchange each instruction adds 4 rows x 128 contiguous bytes
+            const int dcol = quarter * 32 + lane;
+            if (dcol < D) {  // warp-uniform: at D = 64 warps of quarters 2, 3 hold no feature
+                float* dst = p.dq_acc + (qrow0 + q0 + half * 64) * D + dcol;
+                const int nq = min(64, p.N - (q0 + half * 64));
 #pragma unroll
-            for (int k = 0; k < kHalfD / 32; k++) {
-                __syncwarp();
-#pragma unroll
-                for (int u = 0; u < 8; u++)
-                    *reinterpret_cast<uint4*>(stage + lane * 128 + ((u ^ (lane & 7)) << 4)) =
-                        make_uint4(g[32 * k + 4 * u], g[32 * k + 4 * u + 1], g[32 * k + 4 * u + 2],
-                                   g[32 * k + 4 * u + 3]);
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const int rr = 4 * i + lane / 8;  // row within the warp's 32
-                    const int u = lane % 8;
-                    const float4 v = *reinterpret_cast<const float4*>(stage + rr * 128 + ((u ^ (rr & 7)) << 4));
-                    const int q = q0 + quarter * 32 + rr;
-                    if (q < p.N)
-                        red_add_v4(p.dq_acc + (qrow0 + q) * D + half * kHalfD + k * 32 + 4 * u, v.x, v.y, v.z,
-                                   v.w);
-                }
+                for (int i = 0; i < 64; i++)
+                    if (i < nq) red_add_f32(dst + int64_t(i) * D, __uint_as_float(g[i]));
             }
-            __syncwarp();
         }
         if (!ok && lane == 0) bwd_report(p, abort_flag, ST_BWD_ELEM_WAIT);
         // dK and dV rows of this kv tile, this warp's column half (zeros when no
