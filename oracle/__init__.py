@@ -30,14 +30,16 @@ class OraclePattern(ctypes.Structure):
         ("stride", ctypes.c_int32),
         ("n_global", ctypes.c_int32),
         ("global_rows_see_all", ctypes.c_int32),
+        ("area", ctypes.c_int32),
     ]
 
 
 @dataclass(frozen=True)
 class Pattern:
-    """A fixed sparsity pattern: causal band of width ``window`` (inclusive,
-    -1 for none), ``sinks`` leading key tokens, every ``stride``-th prior token
-    (0 for none) and ``n_global`` global tokens."""
+    """A fixed sparsity pattern: band of width ``window`` (inclusive, -1 for
+    none; two-sided without causality), ``sinks`` leading key tokens, every
+    ``stride``-th prior token (0 for none), ``n_global`` global tokens and, if
+    ``area`` > 0, the pairs inside one stripe of ``area`` tokens."""
 
     window: int = -1
     sinks: int = 0
@@ -45,10 +47,11 @@ class Pattern:
     n_global: int = 0
     causal: int = 1
     global_rows_see_all: int = 0
+    area: int = 0
 
     def c(self) -> OraclePattern:
         return OraclePattern(self.causal, self.window, self.sinks, self.stride,
-                             self.n_global, self.global_rows_see_all)
+                             self.n_global, self.global_rows_see_all, self.area)
 
 
 def build(force: bool = False) -> str:

@@ -19,6 +19,12 @@
  *    where the pages leave a choice: the stride is relative ((q - kv) mod s ==
  *    0); causality is applied to the global rows and columns too, unless
  *    `global_rows_see_all` selects the other reading.
+ *    Without causality (causal = 0) the window is two-sided, |q - kv| <= window
+ *    (the sliding window of "Основные шаблоны разреженности": w neighbours on
+ *    the left and on the right), and `area` > 0 admits the pairs of one stripe
+ *    of `area` consecutive tokens (the Area Attention of the "Sparse Attention"
+ *    glossary page, section "Anwendungen": a 40 x 40 feature map cut into four
+ *    stripes of 400 tokens, attention only inside each stripe).
  *
  *  - oracle_block_mask: brute force.  For every (q-tile, kv-tile) pair count
  *    the allowed (q, kv) pairs one by one; zero means empty, all of them means
@@ -59,24 +65,28 @@ typedef struct {
     int32_t stride;              /* > 0: pairs with (q - kv) mod stride == 0 */
     int32_t n_global;            /* keys kv < n_global and queries q < n_global */
     int32_t global_rows_see_all; /* 1: rows q < n_global ignore causality (alternative reading) */
+    int32_t area;                /* > 0: pairs in the same stripe, floor(q / area) == floor(kv / area) */
 } oracle_pattern;
 
 int oracle_allowed(const oracle_pattern *p, int64_t q, int64_t kv)
 {
     int64_t delta = q - kv;
+    int64_t dist = delta < 0 ? -delta : delta;
     if (p->global_rows_see_all && q < p->n_global)
         return 1;
     if (p->causal && delta < 0)
         return 0;
-    if (!p->causal)
-        return -1; /* only causal patterns are defined here */
-    if (p->window >= 0 && delta <= p->window)
+    if (!p->causal && p->stride > 0)
+        return -1; /* a stride without causality is not defined here */
+    if (p->window >= 0 && dist <= p->window)
         return 1;
     if (kv < p->sinks)
         return 1;
     if (p->stride > 0 && delta % p->stride == 0)
         return 1;
     if (kv < p->n_global || q < p->n_global)
+        return 1;
+    if (p->area > 0 && q / p->area == kv / p->area)
         return 1;
     return 0;
 }

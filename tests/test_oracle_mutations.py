@@ -19,7 +19,7 @@ from test_oracle import (closed_live_window_sinks, closed_pairs_window_sinks,
 from test_oracle_bwd import FD_CASES, autograd_pin_holds, fd_pin_holds
 
 MUTANTS = {
-    "window_exclusive": ("delta <= p->window", "delta < p->window"),
+    "window_exclusive": ("dist <= p->window", "dist < p->window"),
     "sinks_inclusive": ("if (kv < p->sinks)", "if (kv <= p->sinks)"),
     "stride_absolute": ("delta % p->stride == 0", "kv % p->stride == 0"),
     "lse_base2": ("*lse = m + log(l);", "*lse = m + log2(l);"),
@@ -89,6 +89,40 @@ def test_mutant_is_caught(name, tmp_path):
     assert src.count(old) == 1, f"mutation site for {name} not found"
     path = oracle.compile_source(src.replace(old, new), str(tmp_path / f"lib_{name}.so"))
     assert not pins_hold(oracle.Oracle(path))
+
+
+NONCAUSAL_MUTANTS = {
+    "window_one_sided": ("int64_t dist = delta < 0 ? -delta : delta;", "int64_t dist = delta;"),
+    "area_stripe_shifted": ("q / p->area == kv / p->area", "(q + 1) / p->area == kv / p->area"),
+    "area_ignored": ("if (p->area > 0 && q / p->area", "if (p->area < 0 && q / p->area"),
+}
+
+
+def noncausal_pins_hold(o: oracle.Oracle) -> bool:
+    from test_oracle_noncausal import nc_sets
+    if o.count_pairs(Pattern(window=-1, causal=0, area=400), 1600) != 640000:
+        return False
+    if o.count_pairs(Pattern(window=37, causal=0), 1000) != sum(min(q, 37) + min(999 - q, 37) + 1 for q in range(1000)):
+        return False
+    for p, N in [(Pattern(window=2, sinks=3, causal=0, area=7), 33), (Pattern(window=-1, causal=1, area=6), 31)]:
+        for q in range(N):
+            for kv in range(N):
+                if o.allowed(p, q, kv) != (kv in nc_sets(N, q, p)):
+                    return False
+    return True
+
+
+def test_unmutated_oracle_passes_noncausal_pins():
+    assert noncausal_pins_hold(oracle.default())
+
+
+@pytest.mark.parametrize("name", sorted(NONCAUSAL_MUTANTS))
+def test_noncausal_mutant_is_caught(name, tmp_path):
+    old, new = NONCAUSAL_MUTANTS[name]
+    src = oracle.source()
+    assert src.count(old) == 1, f"mutation site for {name} not found"
+    path = oracle.compile_source(src.replace(old, new), str(tmp_path / f"lib_{name}.so"))
+    assert not noncausal_pins_hold(oracle.Oracle(path))
 
 
 BWD_MUTANTS = {
