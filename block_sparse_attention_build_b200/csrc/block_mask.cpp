@@ -1,6 +1,10 @@
-// Pattern compiler: classify every (q-tile, kv-tile) of the causal score
-// matrix as empty, partial or full from interval arithmetic on the pattern,
-// and count allowed pairs in closed form per query row.
+// Pattern compiler: classify every (q-tile, kv-tile) of the score matrix as
+// empty, partial or full, and count allowed pairs per query row.  Causal
+// patterns without stripes: interval arithmetic on each tile.  Patterns
+// without causality or with stripes (Area Attention, "Sparse Attention"
+// glossary page, section "Anwendungen"): each row's allowed keys are a union
+// of at most four intervals (two-sided band, sink/global columns, stripe, or
+// the whole row for a global query), counted over each tile's columns.
 //
 // "Sparse Attention" glossary page, section "Ein Muster in Einsparungen
 // verwandeln": a mask is split into 128 x 128 blocks so that kernels can skip
@@ -61,9 +65,67 @@ bool all_allowed(const sa_pattern& p, const Rect& r)
     return lo == hi && lo % p.stride == 0;
 }
 
-bool pattern_ok(const sa_pattern* p)
+// Status of a pattern: SA_OK, SA_ERR_INVALID_ARG for negative fields, or
+// SA_ERR_UNSUPPORTED for a form the library does not build.
+int pattern_status(const sa_pattern* p)
 {
-    return p && p->causal == 1 && p->window >= -1 && p->sinks >= 0 && p->stride >= 0 && p->n_global >= 0;
+    if (!p) return SA_ERR_INVALID_ARG;
+    if (p->window < -1 || p->sinks < 0 || p->stride < 0 || p->n_global < 0 || p->area < 0) return SA_ERR_INVALID_ARG;
+    if (p->causal != 0 && p->causal != 1) return SA_ERR_UNSUPPORTED;
+    if (p->stride > 0 && (p->causal == 0 || p->area > 0)) return SA_ERR_UNSUPPORTED;
+    return SA_OK;
+}
+
+// The causal forms without stripes take the analytic per-tile classifier;
+// the others the per-row interval count.
+bool general_form(const sa_pattern& p) { return p.causal == 0 || p.area > 0; }
+
+// Allowed keys of row q as a union of closed intervals (no stride), clipped
+// to [lo, hi]; returns how many keys of [lo, hi] it holds.
+int64_t row_keys_in(const sa_pattern& p, int64_t N, int64_t q, int64_t lo, int64_t hi)
+{
+    if (p.causal) hi = std::min(hi, q);
+    hi = std::min(hi, N - 1);
+    lo = std::max<int64_t>(lo, 0);
+    if (lo > hi) return 0;
+    if (q < p.n_global) return hi - lo + 1;  // a global row sees every key (up to q when causal)
+    int64_t a[4], b[4];
+    int n = 0;
+    auto add = [&](int64_t x, int64_t y) {
+        x = std::max(x, lo);
+        y = std::min(y, hi);
+        if (x <= y) {
+            a[n] = x;
+            b[n] = y;
+            n++;
+        }
+    };
+    if (p.window >= 0) add(q - p.window, q + p.window);
+    const int64_t cols = std::max(p.sinks, p.n_global);
+    if (cols > 0) add(0, cols - 1);
+    if (p.area > 0) {
+        const int64_t a0 = (q / p.area) * p.area;
+        add(a0, a0 + p.area - 1);
+    }
+    // sort (at most three intervals) and merge
+    for (int i = 0; i < n; i++)
+        for (int j = i + 1; j < n; j++)
+            if (a[j] < a[i]) {
+                std::swap(a[i], a[j]);
+                std::swap(b[i], b[j]);
+            }
+    int64_t total = 0, cur_a = 0, cur_b = -1;
+    for (int i = 0; i < n; i++) {
+        if (a[i] > cur_b + 1 || cur_b < cur_a) {
+            if (cur_b >= cur_a) total += cur_b - cur_a + 1;
+            cur_a = a[i];
+            cur_b = b[i];
+        } else {
+            cur_b = std::max(cur_b, b[i]);
+        }
+    }
+    if (cur_b >= cur_a) total += cur_b - cur_a + 1;
+    return total;
 }
 
 }  // namespace
@@ -104,8 +166,7 @@ extern "C" int32_t sparse_attn_num_tiles(int64_t N, int32_t block)
 extern "C" int sparse_attn_build_block_mask(const sa_pattern* pattern, int64_t N, int32_t block, sa_block_mask* out)
 {
     if (!out || N < 0) return SA_ERR_INVALID_ARG;
-    if (!pattern) return SA_ERR_INVALID_ARG;
-    if (!sa::pattern_ok(pattern)) return pattern->causal != 1 ? SA_ERR_UNSUPPORTED : SA_ERR_INVALID_ARG;
+    if (int rc = sa::pattern_status(pattern)) return rc;
     if (block != 64 && block != 128) return SA_ERR_UNSUPPORTED;
     const int64_t T64 = (N + block - 1) / block;
     if (T64 > (1 << 20)) return SA_ERR_UNSUPPORTED;
@@ -115,6 +176,40 @@ extern "C" int sparse_attn_build_block_mask(const sa_pattern* pattern, int64_t N
 
     int32_t max_row = 0;
     int64_t live = 0, nfull = 0;
+    if (sa::general_form(*pattern)) {
+        // per tile, the allowed keys of each of its rows within the tile's columns
+        for (int32_t i = 0; i < T; i++) {
+            const int64_t q0 = int64_t(i) * block, q1 = std::min<int64_t>(N, q0 + block) - 1;
+            int32_t* idx = out->kv_index + int64_t(i) * T;
+            uint8_t* full = out->kv_full + int64_t(i) * T;
+            int32_t c = 0;
+            const int32_t j_end = pattern->causal ? i : T - 1;
+            for (int32_t j = 0; j <= j_end; j++) {
+                const int64_t k0 = int64_t(j) * block, k1 = std::min<int64_t>(N, k0 + block) - 1;
+                int64_t n = 0;
+                for (int64_t q = q0; q <= q1; q++) n += sa::row_keys_in(*pattern, N, q, k0, k1);
+                if (n == 0) continue;
+                idx[c] = j;
+                full[c] = n == (q1 - q0 + 1) * (k1 - k0 + 1) ? 1 : 0;
+                nfull += full[c];
+                c++;
+            }
+            for (int32_t t = c; t < T; t++) {
+                idx[t] = -1;
+                full[t] = 0;
+            }
+            out->kv_count[i] = c;
+            live += c;
+            max_row = std::max(max_row, c);
+        }
+        out->n_q_tiles = T;
+        out->n_kv_tiles = T;
+        out->block = block;
+        out->max_per_row = max_row;
+        out->n_live = live;
+        out->n_full = nfull;
+        return SA_OK;
+    }
     for (int32_t i = 0; i < T; i++) {
         sa::Rect r;
         r.q0 = int64_t(i) * block;
@@ -151,9 +246,13 @@ extern "C" int sparse_attn_build_block_mask(const sa_pattern* pattern, int64_t N
 extern "C" int sparse_attn_count_pairs(const sa_pattern* pattern, int64_t N, int64_t* pairs)
 {
     if (!pattern || !pairs || N < 0) return SA_ERR_INVALID_ARG;
-    if (!sa::pattern_ok(pattern)) return pattern->causal != 1 ? SA_ERR_UNSUPPORTED : SA_ERR_INVALID_ARG;
+    if (int rc = sa::pattern_status(pattern)) return rc;
     int64_t total = 0;
-    for (int64_t q = 0; q < N; q++) total += sa::row_pairs(*pattern, q);
+    if (sa::general_form(*pattern)) {
+        for (int64_t q = 0; q < N; q++) total += sa::row_keys_in(*pattern, N, q, 0, N - 1);
+    } else {
+        for (int64_t q = 0; q < N; q++) total += sa::row_pairs(*pattern, q);
+    }
     *pairs = total;
     return SA_OK;
 }

@@ -77,7 +77,7 @@ struct BwdParams {
     int32_t* status;
     long long timeout;       // SM cycles per bounded wait
     int32_t T, N, B, Hq, Hkv, group;
-    int32_t window, sinks, stride, n_global;
+    int32_t window, sinks, stride, n_global, causal, area;  // window and area clipped to N
     float scale_log2;        // scale * log2(e)
     float scale;
 };
@@ -121,16 +121,20 @@ __device__ __forceinline__ uint32_t bwd_bits(int lo, int hi)
 }
 
 // Allowed pairs (q, kv) for q = qb + i, i in [0, 32), as bits: the pattern's
-// rule (band, sink and global columns, global rows, stride) under causality
-// and the sequence bound.
+// rule (two-sided band, sink and global columns, global rows, stripe, stride)
+// under causality (if set) and the sequence bound.
 __device__ __forceinline__ uint32_t bwd_allow_word(const BwdParams& p, int qb, int kv)
 {
     if (kv >= p.N) return 0u;
-    const uint32_t in_range = bwd_bits(kv - qb, p.N - 1 - qb);  // kv <= q < N
+    const uint32_t in_range = bwd_bits((p.causal ? kv : 0) - qb, p.N - 1 - qb);  // (kv <=) q < N
     if (kv < max(p.sinks, p.n_global)) return in_range;
     uint32_t m = 0u;
-    if (p.window >= 0) m |= bwd_bits(kv - qb, kv + p.window - qb);
+    if (p.window >= 0) m |= bwd_bits(kv - p.window - qb, kv + p.window - qb);
     if (p.n_global > 0) m |= bwd_bits(0, p.n_global - 1 - qb);
+    if (p.area > 0) {
+        const int a0 = (kv / p.area) * p.area;
+        m |= bwd_bits(a0 - qb, a0 + p.area - 1 - qb);
+    }
     if (p.stride > 0) {
         int i = (kv - qb) % p.stride;
         if (i < 0) i += p.stride;

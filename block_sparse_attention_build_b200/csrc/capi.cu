@@ -86,10 +86,24 @@ int launch_any(int D, int block, const CUtensorMap& mq, const CUtensorMap& mk, c
     return launch<64, 64, MULTI>(mq, mk, mv, mo, p, hp, g, st);
 }
 
-bool pattern_ok(const sa_pattern& pt)
+// SA_OK, SA_ERR_INVALID_ARG (a negative field) or SA_ERR_UNSUPPORTED (a form
+// the library does not build: causal not 0 or 1, a stride without causality
+// or with stripes).
+int pattern_status(const sa_pattern& pt)
 {
-    return pt.window >= -1 && pt.sinks >= 0 && pt.stride >= 0 && pt.n_global >= 0;
+    if (pt.window < -1 || pt.sinks < 0 || pt.stride < 0 || pt.n_global < 0 || pt.area < 0) return SA_ERR_INVALID_ARG;
+    if (pt.causal != 0 && pt.causal != 1) return SA_ERR_UNSUPPORTED;
+    if (pt.stride > 0 && (pt.causal == 0 || pt.area > 0)) return SA_ERR_UNSUPPORTED;
+    return SA_OK;
 }
+
+// Forms beyond the causal band / sinks / stride / global rules: the kernel
+// instantiation with a pattern table masks them.
+bool general_form(const sa_pattern& pt) { return pt.causal == 0 || pt.area > 0; }
+
+// Window and stripe clipped to the sequence (same allowed set), so that the
+// kernels' q - kv +- window and stripe bounds stay inside int32.
+int32_t clip_to(int32_t v, int32_t N) { return v > N ? N : v; }
 
 // The forward pass behind sparse_attn_fwd (one pattern: n_patterns = 1,
 // head_pattern = null) and sparse_attn_fwd_heads (a pattern per query head).
@@ -98,23 +112,23 @@ int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* m
              void* stream)
 {
     if (!masks || !patterns || !shape) return SA_ERR_INVALID_ARG;
-    const bool multi = head_pattern != nullptr;
-    if (n_patterns < 1 || n_patterns > (multi ? kMaxPatterns : 1)) return SA_ERR_INVALID_ARG;
+    const bool per_head = head_pattern != nullptr;
+    if (n_patterns < 1 || n_patterns > (per_head ? kMaxPatterns : 1)) return SA_ERR_INVALID_ARG;
+    bool multi = per_head;  // general forms also take the pattern-table kernel
+    for (int i = 0; i < n_patterns; i++) multi = multi || general_form(patterns[i]);
     const sa_block_mask* mask = &masks[0];
     const sa_pattern* pattern = &patterns[0];
     const sa_shape s = *shape;
     if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
-    for (int i = 0; i < n_patterns; i++) {
-        if (patterns[i].causal != 1) return SA_ERR_UNSUPPORTED;
-        if (!pattern_ok(patterns[i])) return SA_ERR_INVALID_ARG;
-    }
+    for (int i = 0; i < n_patterns; i++)
+        if (int rc = pattern_status(patterns[i])) return rc;
     if (s.D != 64 && s.D != 128) return SA_ERR_UNSUPPORTED;
     if (mask->block != 64 && mask->block != 128) return SA_ERR_UNSUPPORTED;
     for (int i = 1; i < n_patterns; i++)
         if (masks[i].block != mask->block) return SA_ERR_MASK_MISMATCH;
     if (multi && s.Hq > kMaxHeadsMulti) return SA_ERR_UNSUPPORTED;
-    if (multi)
+    if (per_head)
         for (int h = 0; h < s.Hq; h++)
             if (head_pattern[h] < 0 || head_pattern[h] >= n_patterns) return SA_ERR_INVALID_ARG;
     if (s.B == 0 || s.Hq == 0 || s.N == 0) return SA_OK;  // nothing to compute
@@ -175,7 +189,7 @@ int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* m
     p.n_whole = static_cast<int32_t>(n_whole);
     p.n_items = static_cast<int32_t>(n_items);
     p.pairs = static_cast<int32_t>(pairs);
-    p.window = pattern->window;
+    p.window = clip_to(pattern->window, s.N);
     p.sinks = pattern->sinks;
     p.stride = pattern->stride;
     p.n_global = pattern->n_global;
@@ -193,12 +207,14 @@ int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* m
         hp.pat[i].kv_count = masks[i].kv_count;
         hp.pat[i].kv_index = masks[i].kv_index;
         hp.pat[i].kv_full = masks[i].kv_full;
-        hp.pat[i].window = patterns[i].window;
+        hp.pat[i].window = clip_to(patterns[i].window, s.N);
         hp.pat[i].sinks = patterns[i].sinks;
         hp.pat[i].stride = patterns[i].stride;
         hp.pat[i].n_global = patterns[i].n_global;
+        hp.pat[i].causal = patterns[i].causal;
+        hp.pat[i].area = clip_to(patterns[i].area, s.N);
     }
-    for (int h = 0; h < s.Hq; h++) hp.head[h] = static_cast<uint8_t>(head_pattern[h]);
+    for (int h = 0; h < s.Hq; h++) hp.head[h] = per_head ? static_cast<uint8_t>(head_pattern[h]) : 0;
     return launch_any<true>(s.D, mask->block, mq, mk, mv, mo, p, hp, g, st);
 }
 
@@ -319,4 +335,4 @@ extern "C" const char* sparse_attn_status_string(int status)
     }
 }
 
-extern "C" int32_t sparse_attn_version(void) { return 100; }
+extern "C" int32_t sparse_attn_version(void) { return 200; }

@@ -85,7 +85,8 @@ extern "C" int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void*
     const sa_shape s = *shape;
     if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
-    if (pattern->causal != 1) return SA_ERR_UNSUPPORTED;
+    // the causal band / sinks / stride / global forms only (no pattern table here)
+    if (pattern->causal != 1 || pattern->area != 0) return SA_ERR_UNSUPPORTED;
     if (pattern->window < -1 || pattern->sinks < 0 || pattern->stride < 0 || pattern->n_global < 0)
         return SA_ERR_INVALID_ARG;
     if (s.D != 64 && s.D != 128) return SA_ERR_UNSUPPORTED;
@@ -157,7 +158,7 @@ extern "C" int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void*
     p.n_whole = static_cast<int32_t>(n_whole);
     p.n_items = static_cast<int32_t>(n_items);
     p.pairs = static_cast<int32_t>(pairs);
-    p.window = pattern->window;
+    p.window = pattern->window > s.N ? s.N : pattern->window;  // same allowed set, no int32 overflow in the kernel
     p.sinks = pattern->sinks;
     p.stride = pattern->stride;
     p.n_global = pattern->n_global;

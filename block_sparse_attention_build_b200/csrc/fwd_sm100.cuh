@@ -97,14 +97,17 @@ struct FwdParams {
 // compiled patterns (its block mask and the rule parameters its partial tiles
 // are masked with).  Different heads of a layer may carry different patterns
 // ("Sparse-трансформеры" page, section "Комбинация — норма, а не
-// исключение").  Used by the kernels instantiated with MULTI = true.
+// исключение").  Used by the kernels instantiated with MULTI = true, which
+// also take the pattern forms beyond causal band / sinks / stride / global:
+// no causality (two-sided band) and stripes (Area Attention, "Sparse
+// Attention" glossary page, section "Anwendungen").
 constexpr int kMaxPatterns = 8;
 constexpr int kMaxHeadsMulti = 256;
 struct PatternRef {
     const int32_t* kv_count;  // [T]
     const int32_t* kv_index;  // [T * T]
     const uint8_t* kv_full;   // [T * T]
-    int32_t window, sinks, stride, n_global;
+    int32_t window, sinks, stride, n_global, causal, area;
 };
 struct HeadPatterns {
     PatternRef pat[kMaxPatterns];
@@ -901,6 +904,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t col_o = static_cast<uint32_t>(2 * BN + x * D);
         int cols = max(p.sinks, p.n_global);
         int pw = p.window, ps = p.stride, pg = p.n_global;  // this slot's pattern (per unit when MULTI)
+        int qlim = 0, a_lo = 0, a_hi = -1;                   // MULTI: last allowed key (causal bound), stripe
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
         int steps = 0, units = 0;
         int units_b = 0;   // slot A only: completed phases of o_full[1] (slot B's last PV of a unit)
@@ -926,6 +930,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ps = pr.stride;
                 pg = pr.n_global;
                 cols = max(pr.sinks, pr.n_global);
+                qlim = pr.causal ? q : p.N - 1;
+                if (pr.area > 0) {
+                    a_lo = (q / pr.area) * pr.area;
+                    a_hi = a_lo + pr.area - 1;
+                } else {
+                    a_lo = 0;
+                    a_hi = -1;
+                }
             }
             const bool row_all = q < pg;
             float m_ref = -INFINITY;  // running max, log2 units of the scaled score
@@ -945,12 +957,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t allow[BN / 32];
                 if (masked) {
                     const int dq = q - kv0;
-                    const int c_max = min(dq, p.N - 1 - kv0);
+                    // MULTI: causal or not (qlim), two-sided band, stripe [a_lo, a_hi]
+                    const int c_max = MULTI ? min(qlim, p.N - 1) - kv0 : min(dq, p.N - 1 - kv0);
 #pragma unroll
                     for (int w = 0; w < BN / 32; w++) {
                         const int base = 32 * w;
                         uint32_t m = bits_between(0, cols - 1 - kv0 - base);
-                        if (pw >= 0) m |= bits_between(dq - pw - base, 31);
+                        if (pw >= 0) m |= bits_between(dq - pw - base, MULTI ? dq + pw - base : 31);
+                        if constexpr (MULTI) m |= bits_between(a_lo - kv0 - base, a_hi - kv0 - base);
                         if (ps > 0) {
                             int r0 = dq % ps;
                             if (r0 < 0) r0 += ps;

@@ -1,5 +1,5 @@
 /*
- * sparse_attn — block-sparse causal attention forward for NVIDIA B200 (sm_100a).
+ * sparse_attn — block-sparse attention, forward and backward, for NVIDIA B200 (sm_100a).
  *
  * C ABI.  Plain pointers and sizes only; no C++ or framework types cross it.
  * Every call returns an int status (SA_OK or a negative SA_ERR_* code); no
@@ -37,7 +37,7 @@ extern "C" {
 /* ---- status codes ------------------------------------------------------- */
 #define SA_OK 0
 #define SA_ERR_INVALID_ARG (-1)      /* null pointer, negative size, bad scale */
-#define SA_ERR_UNSUPPORTED (-2)      /* D not in {64, 128}, block not in {64, 128}, causal != 1, Hq % Hkv != 0 */
+#define SA_ERR_UNSUPPORTED (-2)      /* D not in {64, 128}, block not in {64, 128}, Hq % Hkv != 0, a pattern form not built */
 #define SA_ERR_MISALIGNED (-3)       /* a tensor pointer is not 16-byte aligned */
 #define SA_ERR_BUFFER_TOO_SMALL (-4) /* output arrays smaller than the tile count */
 #define SA_ERR_CUDA (-5)             /* a CUDA runtime call or kernel launch failed */
@@ -47,14 +47,21 @@ extern "C" {
 
 /*
  * A fixed sparsity pattern.  A pair (q, kv) is allowed when
- *     q >= kv  and  ( (window >= 0 and q - kv <= window)
- *                     or kv < sinks
- *                     or (stride > 0 and (q - kv) mod stride == 0)
- *                     or kv < n_global or q < n_global ).
+ *     (causal == 0 or q >= kv)
+ *     and ( (window >= 0 and |q - kv| <= window)
+ *           or kv < sinks
+ *           or (stride > 0 and (q - kv) mod stride == 0)
+ *           or kv < n_global or q < n_global
+ *           or (area > 0 and floor(q / area) == floor(kv / area)) ).
  * Pages: "Sparse Attention", sections "Gängige Sparsity-Muster" and "Ein
- * Muster in Einsparungen verwandeln" (window inclusive, as in local_plus_sinks).
- * The stride counts back from the query (every s-th prior token); the global
- * rows and columns stay causal.  causal must be 1.
+ * Muster in Einsparungen verwandeln" (window inclusive, as in local_plus_sinks),
+ * and section "Anwendungen" (Area Attention: attention only inside stripes of
+ * consecutive tokens); "Sparse-трансформеры", section "Основные шаблоны
+ * разреженности" (without causality the window reaches w tokens on both
+ * sides).  The stride counts back from the query (every s-th prior token) and
+ * needs causal == 1; with causal == 1 the global rows and columns stay causal.
+ * Supported forms: causal == 1 with any of the rules; causal == 0 with window,
+ * sinks, n_global and area (stride > 0 gives SA_ERR_UNSUPPORTED).
  */
 typedef struct {
     int32_t causal;
@@ -62,6 +69,7 @@ typedef struct {
     int32_t sinks;
     int32_t stride;
     int32_t n_global;
+    int32_t area;  /* stripe length; 0 for none */
 } sa_pattern;
 
 /*
@@ -96,9 +104,11 @@ typedef struct {
 int32_t sparse_attn_num_tiles(int64_t N, int32_t block);
 
 /*
- * Classify every (q-tile, kv-tile) pair of an N x N causal score matrix as
- * empty, partial or full, analytically from the pattern (no per-pair loop),
- * and write the lists described at sa_block_mask.  Host-only; `out` holds
+ * Classify every (q-tile, kv-tile) pair of an N x N score matrix as empty,
+ * partial or full and write the lists described at sa_block_mask: for causal
+ * patterns without stripes analytically per tile (no per-pair or per-row
+ * loop); for the others (causal == 0, or area > 0) from each row's allowed
+ * keys, a union of at most four intervals, counted per tile.  Host-only; `out` holds
  * caller-owned host arrays with capacity out->n_q_tiles rows of
  * out->n_kv_tiles entries, both at least T (else SA_ERR_BUFFER_TOO_SMALL).
  * block is 64 or 128; N >= 0 (N = 0 gives T = 0).
@@ -107,7 +117,8 @@ int sparse_attn_build_block_mask(const sa_pattern* pattern, int64_t N, int32_t b
 
 /*
  * Number of allowed (q, kv) pairs of one head, 0 <= q, kv < N, in closed form
- * per query row.  4 * D * pairs is the useful work of one (batch, head).
+ * per query row (interval unions for the forms without a stride).  4 * D *
+ * pairs is the useful work of one (batch, head).
  */
 int sparse_attn_count_pairs(const sa_pattern* pattern, int64_t N, int64_t* pairs);
 
@@ -120,8 +131,11 @@ int sparse_attn_count_pairs(const sa_pattern* pattern, int64_t N, int64_t* pairs
  * legacy default stream).  Asynchronous: returns once the kernel is queued;
  * launch errors come back as SA_ERR_CUDA, a device-side timeout through
  * sparse_attn_check_device.  Rows with no allowed key get O = 0, LSE = -inf.
- * Supported: D in {64, 128}, mask block in {64, 128}, Hq % Hkv == 0, causal,
- * at most 4096 tiles per side (N <= 4096 * block); else SA_ERR_UNSUPPORTED.
+ * Supported: D in {64, 128}, mask block in {64, 128}, Hq % Hkv == 0, the
+ * pattern forms listed at sa_pattern, at most 4096 tiles per side (N <= 4096 *
+ * block); else SA_ERR_UNSUPPORTED.  Patterns with causal == 0 or area > 0 run
+ * on the kernel instantiation that takes a pattern table (as
+ * sparse_attn_fwd_heads), which limits them to Hq <= 256.
  */
 int sparse_attn_fwd(const void* Q, const void* K, const void* V, const sa_block_mask* mask,
                     const sa_pattern* pattern, const sa_shape* shape, float scale, void* O, float* LSE,

@@ -25,13 +25,16 @@ class Workload:
     n_global: int
     block: int
     seed: int = 0
+    causal: int = 1
+    area: int = 0
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.D)
 
     def pattern_args(self) -> dict:
-        return dict(window=self.window, sinks=self.sinks, stride=self.stride, n_global=self.n_global)
+        return dict(window=self.window, sinks=self.sinks, stride=self.stride, n_global=self.n_global,
+                    causal=self.causal, area=self.area)
 
 
 WORKLOADS = {
@@ -45,6 +48,9 @@ WORKLOADS = {
     "w128_s4_h64_n16384": Workload("w128_s4_h64_n16384", 2, 64, 8, 16384, 64, 128, 4, 0, 0, 128),
     # local 128 + every 128th prior token + 16 global tokens
     "strided_global_n16384": Workload("strided_global_n16384", 1, 16, 16, 16384, 128, 128, 0, 128, 16, 128),
+    # Area Attention: 1,600 tokens (a 40 x 40 feature map) in four stripes of 400, no causality;
+    # heads, head size and batch are not on the pages (8 heads of 64, a batch of 16 images)
+    "area_n1600": Workload("area_n1600", 16, 8, 8, 1600, 64, -1, 0, 0, 0, 128, causal=0, area=400),
 }
 
 # The workload the throughput metric is quoted on.

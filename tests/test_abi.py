@@ -41,7 +41,8 @@ def test_version_and_status_strings():
 
 
 def opattern(p: sa.Pattern):
-    return oracle.Pattern(window=p.window, sinks=p.sinks, stride=p.stride, n_global=p.n_global)
+    return oracle.Pattern(window=p.window, sinks=p.sinks, stride=p.stride, n_global=p.n_global, causal=p.causal,
+                          area=p.area)
 
 
 SWEEP = [
@@ -90,7 +91,7 @@ def test_builder_errors():
         sa.build_block_mask(sa.Pattern(window=4), 100, 32)
     assert e.value.status == sa.SA_ERR_UNSUPPORTED
     with pytest.raises(sa.SparseAttnError) as e:
-        sa.build_block_mask(sa.Pattern(window=4, causal=0), 100, 64)
+        sa.build_block_mask(sa.Pattern(window=4, stride=2, causal=0), 100, 64)
     assert e.value.status == sa.SA_ERR_UNSUPPORTED
     with pytest.raises(sa.SparseAttnError) as e:
         sa.build_block_mask(sa.Pattern(window=-2), 100, 64)
@@ -120,7 +121,7 @@ def test_fwd_argument_errors_without_gpu():
     assert call((1, 2, 2, 100, 128), ptr=fake + 8) == sa.SA_ERR_MISALIGNED
     assert call((0, 2, 2, 100, 128)) == sa.SA_OK                      # nothing to compute
     assert call((1, 2, 2, 0, 128)) == sa.SA_OK
-    bad = sa.Pattern(window=8, causal=0)._c()
+    bad = sa.Pattern(window=8, stride=4, causal=0)._c()
     assert call((1, 2, 2, 100, 128), pat=bad) == sa.SA_ERR_UNSUPPORTED
     ws = ctypes.c_size_t(0)
     assert sa.lib.sparse_attn_fwd_host_workspace(ctypes.byref(sa._Shape(1, 2, 1, 100, 64)), ctypes.byref(ws)) == 0
@@ -149,7 +150,7 @@ def test_fwd_heads_argument_errors_without_gpu():
     assert call((1, 2, 2, 100, 128), [0, -1]) == sa.SA_ERR_INVALID_ARG
     assert call((1, 2, 2, 100, 128), [0, 1], masks=(m, m64)) == sa.SA_ERR_MASK_MISMATCH  # blocks differ
     assert call((1, 300, 300, 100, 128), [0] * 300) == sa.SA_ERR_UNSUPPORTED         # more than 256 heads
-    bad = sa.Pattern(window=8, causal=0)._c()
+    bad = sa.Pattern(window=8, stride=4, causal=0)._c()
     assert call((1, 2, 2, 100, 128), [0, 1], pats=(p, bad)) == sa.SA_ERR_UNSUPPORTED
     assert call((1, 2, 2, 100, 128), [0, 1], ptr=fake + 8) == sa.SA_ERR_MISALIGNED
     assert call((0, 2, 2, 100, 128), [0, 1]) == sa.SA_OK                             # nothing to compute
@@ -216,7 +217,60 @@ def test_bwd_argument_errors_without_gpu():
     assert call((1, 2, 2, 100, 128), ws=fake + 16) == sa.SA_ERR_MISALIGNED         # workspace 256-aligned
     assert call((1, 2, 2, 100, 128), ws_bytes=ws_ok - 1) == sa.SA_ERR_BUFFER_TOO_SMALL
     assert call((0, 2, 2, 100, 128)) == sa.SA_OK
-    bad = sa.Pattern(window=8, causal=0)._c()
+    bad = sa.Pattern(window=8, stride=4, causal=0)._c()
     assert call((1, 2, 2, 100, 128), pat=bad) == sa.SA_ERR_UNSUPPORTED
     rows = 1 * 2 * 100
     assert ws_ok >= 2 * rows * 4 + rows * 128 * 4
+
+
+GENERAL = [
+    (sa.Pattern(window=w, sinks=s, n_global=g, causal=c, area=a), N, b)
+    for (w, s, g, c, a) in [(37, 0, 0, 0, 0), (-1, 0, 0, 0, 400), (-1, 0, 0, 0, 100), (5, 3, 0, 0, 0),
+                            (2, 0, 4, 0, 0), (-1, 2, 0, 0, 77), (20, 0, 0, 1, 64), (-1, 0, 0, 1, 400),
+                            (300, 1, 2, 0, 130), (0, 0, 0, 0, 1), (-1, 0, 0, 0, 0), (5000, 0, 0, 0, 0)]
+    for N in (1, 100, 500, 1000, 1600)
+    for b in (64, 128)
+]
+
+
+@pytest.mark.parametrize("p,N,b", GENERAL)
+def test_general_block_mask_matches_oracle(p, N, b):
+    m = sa.build_block_mask(p, N, b)
+    c, i, f = oracle.block_mask(opattern(p), N, b)
+    assert np.array_equal(m.counts, c) and np.array_equal(m.index, i) and np.array_equal(m.full, f)
+    assert sa.count_pairs(p, N) == oracle.count_pairs(opattern(p), N)
+    t = sa.transpose_block_mask(m)
+    tc, ti, tf = transpose_of_oracle(p, N, b)
+    assert np.array_equal(t.counts, tc) and np.array_equal(t.index, ti) and np.array_equal(t.full, tf)
+
+
+def test_area_attention_printed_pair_count():
+    assert sa.count_pairs(sa.Pattern(window=-1, causal=0, area=400), 1600) == 640000
+
+
+def test_general_pattern_errors():
+    for p, rc in [(sa.Pattern(window=4, stride=8, causal=0), sa.SA_ERR_UNSUPPORTED),
+                  (sa.Pattern(window=4, stride=8, area=64), sa.SA_ERR_UNSUPPORTED),
+                  (sa.Pattern(window=4, causal=2), sa.SA_ERR_UNSUPPORTED),
+                  (sa.Pattern(window=4, area=-1), sa.SA_ERR_INVALID_ARG)]:
+        with pytest.raises(sa.SparseAttnError) as e:
+            sa.build_block_mask(p, 100, 64)
+        assert e.value.status == rc
+        with pytest.raises(sa.SparseAttnError) as e:
+            sa.count_pairs(p, 100)
+        assert e.value.status == rc
+    # the forward and backward entry points check the same before any CUDA call
+    m = sa._BlockMask(1, 1, 128, 1, 1, 0, 16, 16, 16)
+    fake = 1 << 20
+    bad = sa.Pattern(window=4, stride=8, causal=0)._c()
+    shape = sa._Shape(1, 2, 2, 100, 128)
+    assert sa.lib.sparse_attn_fwd(fake, fake, fake, ctypes.byref(m), ctypes.byref(bad), ctypes.byref(shape), 0.1,
+                                  fake, fake, None) == sa.SA_ERR_UNSUPPORTED
+    assert sa.lib.sparse_attn_bwd(fake, fake, fake, fake, fake, fake, ctypes.byref(m), ctypes.byref(bad),
+                                  ctypes.byref(shape), 0.1, fake, fake, fake, fake, 1 << 30, None) == sa.SA_ERR_UNSUPPORTED
+    area = sa.Pattern(window=-1, causal=0, area=64)._c()
+    assert sa.lib.sparse_attn_fwd_noalloc(fake, fake, fake, ctypes.byref(m), ctypes.byref(area), ctypes.byref(shape),
+                                          0.1, fake, fake, None) == sa.SA_ERR_UNSUPPORTED
+    big = sa._Shape(1, 300, 300, 100, 128)  # general forms use the pattern-table kernel: Hq <= 256
+    assert sa.lib.sparse_attn_fwd(fake, fake, fake, ctypes.byref(m), ctypes.byref(area), ctypes.byref(big), 0.1,
+                                  fake, fake, None) == sa.SA_ERR_UNSUPPORTED

@@ -31,7 +31,8 @@ def to_dev(bits: np.ndarray) -> torch.Tensor:
 
 
 def opattern(p: sa.Pattern):
-    return oracle.Pattern(window=p.window, sinks=p.sinks, stride=p.stride, n_global=p.n_global)
+    return oracle.Pattern(window=p.window, sinks=p.sinks, stride=p.stride, n_global=p.n_global, causal=p.causal,
+                          area=p.area)
 
 
 def inputs(B, Hq, Hkv, N, D, seed):
@@ -79,6 +80,10 @@ CASES = [
     (1, 1, 1, 100, 128, sa.Pattern(window=30, sinks=2)),               # one partial tile
     (1, 1, 1, 1, 64, sa.Pattern(window=5)),                            # N = 1
     (1, 2, 2, 1100, 128, sa.Pattern(window=257, sinks=130)),           # sinks wider than a tile
+    (1, 2, 2, 1600, 64, sa.Pattern(window=-1, causal=0, area=400)),    # Area Attention, 4 x 400
+    (2, 2, 1, 1000, 128, sa.Pattern(window=100, causal=0)),            # two-sided window, GQA
+    (1, 2, 2, 900, 128, sa.Pattern(window=-1, sinks=4, n_global=3, causal=0, area=200)),
+    (1, 2, 2, 1100, 64, sa.Pattern(window=20, causal=1, area=300)),    # block-causal stripes + band
 ]
 
 

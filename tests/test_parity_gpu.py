@@ -50,7 +50,8 @@ def compare(O, LSE, Oref, LSEref):
 
 
 def opattern(p: sa.Pattern):
-    return oracle.Pattern(window=p.window, sinks=p.sinks, stride=p.stride, n_global=p.n_global)
+    return oracle.Pattern(window=p.window, sinks=p.sinks, stride=p.stride, n_global=p.n_global, causal=p.causal,
+                          area=p.area)
 
 
 SMALL = [
@@ -244,3 +245,41 @@ def test_per_head_entry_with_one_pattern_equals_fwd():
     O1, L1 = run_heads(q, k, v, [p], [0] * Hq, 128, scale)
     O2, L2 = run_gpu(q, k, v, p, 128, scale)
     assert np.array_equal(O1, O2) and np.array_equal(L1, L2)
+
+
+GENERAL_CASES = [
+    # (B, Hq, Hkv, N, D, pattern, block): without causality, and stripes
+    (1, 2, 2, 1600, 64, sa.Pattern(window=-1, causal=0, area=400), 128),      # Area Attention, 4 x 400
+    (2, 2, 1, 1000, 128, sa.Pattern(window=100, causal=0), 128),              # two-sided window, GQA
+    (1, 2, 2, 700, 64, sa.Pattern(window=700, causal=0), 64),                 # dense, no causality
+    (1, 3, 3, 900, 128, sa.Pattern(window=-1, sinks=4, n_global=3, causal=0, area=200), 128),
+    (1, 2, 2, 1100, 64, sa.Pattern(window=20, causal=1, area=300), 64),       # block-causal stripes + band
+    (1, 1, 1, 333, 128, sa.Pattern(window=10, causal=0, area=50), 128),       # ragged, stripes inside a tile
+]
+
+
+@pytest.mark.parametrize("split", [False, True], ids=["whole", "split"])
+@pytest.mark.parametrize("case", GENERAL_CASES, ids=lambda c: f"B{c[0]}H{c[1]}/{c[2]}N{c[3]}D{c[4]}b{c[6]}-{c[5]}")
+def test_general_pattern_parity(case, split):
+    B, Hq, Hkv, N, D, p, block = case
+    q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=N + 11)
+    scale = 1 / math.sqrt(D)
+    if split:
+        sa.set_debug(sa.DEBUG_SPLIT_ALL)
+    try:
+        O, LSE = run_gpu(q, k, v, p, block, scale)
+    finally:
+        sa.set_debug(0)
+    Oref, LSEref = oracle.attention(q, k, v, opattern(p), scale)
+    compare(O, LSE, Oref, LSEref)
+
+
+def test_per_head_mix_of_causal_and_area():
+    B, Hq, Hkv, N, D, block = 1, 4, 2, 1600, 64, 128
+    patterns = [sa.Pattern(window=256, sinks=4), sa.Pattern(window=-1, causal=0, area=400)]
+    heads = [0, 1, 1, 0]
+    q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=21)
+    scale = 1 / math.sqrt(D)
+    O, LSE = run_heads(q, k, v, patterns, heads, block, scale)
+    Oref, LSEref = oracle_heads(q, k, v, patterns, heads, scale)
+    compare(O, LSE, Oref, LSEref)
