@@ -31,6 +31,7 @@ class OraclePattern(ctypes.Structure):
         ("n_global", ctypes.c_int32),
         ("global_rows_see_all", ctypes.c_int32),
         ("area", ctypes.c_int32),
+        ("summary", ctypes.c_int32),
     ]
 
 
@@ -39,7 +40,8 @@ class Pattern:
     """A fixed sparsity pattern: band of width ``window`` (inclusive, -1 for
     none; two-sided without causality), ``sinks`` leading key tokens, every
     ``stride``-th prior token (0 for none), ``n_global`` global tokens and, if
-    ``area`` > 0, the pairs inside one stripe of ``area`` tokens."""
+    ``area`` > 0, the pairs inside one stripe of ``area`` tokens, plus (``summary``
+    > 0) keys in the last ``summary`` positions of any stripe."""
 
     window: int = -1
     sinks: int = 0
@@ -48,10 +50,11 @@ class Pattern:
     causal: int = 1
     global_rows_see_all: int = 0
     area: int = 0
+    summary: int = 0
 
     def c(self) -> OraclePattern:
         return OraclePattern(self.causal, self.window, self.sinks, self.stride,
-                             self.n_global, self.global_rows_see_all, self.area)
+                             self.n_global, self.global_rows_see_all, self.area, self.summary)
 
 
 def build(force: bool = False) -> str:

@@ -24,7 +24,11 @@
  *    the left and on the right), and `area` > 0 admits the pairs of one stripe
  *    of `area` consecutive tokens (the Area Attention of the "Sparse Attention"
  *    glossary page, section "Anwendungen": a 40 x 40 feature map cut into four
- *    stripes of 400 tokens, attention only inside each stripe).
+ *    stripes of 400 tokens, attention only inside each stripe).  With `area`
+ *    and `summary` > 0 this is the "fixed" pattern of "Основные шаблоны
+ *    разреженности": blocks with local attention inside, linked through
+ *    dedicated summary positions, read here as the last `summary` positions
+ *    of every block, which every (causally later) query may attend to.
  *
  *  - oracle_block_mask: brute force.  For every (q-tile, kv-tile) pair count
  *    the allowed (q, kv) pairs one by one; zero means empty, all of them means
@@ -66,6 +70,7 @@ typedef struct {
     int32_t n_global;            /* keys kv < n_global and queries q < n_global */
     int32_t global_rows_see_all; /* 1: rows q < n_global ignore causality (alternative reading) */
     int32_t area;                /* > 0: pairs in the same stripe, floor(q / area) == floor(kv / area) */
+    int32_t summary;             /* with area > 0: keys in the last `summary` positions of any stripe */
 } oracle_pattern;
 
 int oracle_allowed(const oracle_pattern *p, int64_t q, int64_t kv)
@@ -87,6 +92,8 @@ int oracle_allowed(const oracle_pattern *p, int64_t q, int64_t kv)
     if (kv < p->n_global || q < p->n_global)
         return 1;
     if (p->area > 0 && q / p->area == kv / p->area)
+        return 1;
+    if (p->area > 0 && p->summary > 0 && kv % p->area >= p->area - p->summary)
         return 1;
     return 0;
 }

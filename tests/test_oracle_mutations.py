@@ -95,14 +95,23 @@ NONCAUSAL_MUTANTS = {
     "window_one_sided": ("int64_t dist = delta < 0 ? -delta : delta;", "int64_t dist = delta;"),
     "area_stripe_shifted": ("q / p->area == kv / p->area", "(q + 1) / p->area == kv / p->area"),
     "area_ignored": ("if (p->area > 0 && q / p->area", "if (p->area < 0 && q / p->area"),
+    "summary_first_positions": ("kv % p->area >= p->area - p->summary", "kv % p->area < p->summary"),
 }
 
 
 def noncausal_pins_hold(o: oracle.Oracle) -> bool:
-    from test_oracle_noncausal import nc_sets
+    from test_oracle_noncausal import fixed_sets, nc_sets
+    N = 37
+    for q in range(N):
+        for kv in range(N):
+            if o.allowed(Pattern(window=-1, causal=1, area=8, summary=2), q, kv) != (kv in fixed_sets(N, q, 8, 2)):
+                return False
     if o.count_pairs(Pattern(window=-1, causal=0, area=400), 1600) != 640000:
         return False
     if o.count_pairs(Pattern(window=37, causal=0), 1000) != sum(min(q, 37) + min(999 - q, 37) + 1 for q in range(1000)):
+        return False
+    if o.count_pairs(Pattern(window=-1, causal=1, area=128, summary=16), 1024) != sum(
+            q % 128 + 1 + (q // 128) * 16 for q in range(1024)):
         return False
     for p, N in [(Pattern(window=2, sinks=3, causal=0, area=7), 33), (Pattern(window=-1, causal=1, area=6), 31)]:
         for q in range(N):

@@ -154,3 +154,61 @@ def test_noncausal_gradients_equal_autograd():
     rO, rq, rk, rv = torch_grads(q, k, v, do, 0.3, mask=mask)
     for a, b in ((O, rO), (dQ, rq), (dK, rk), (dV, rv)):
         assert np.abs(a - b).max() <= 1e-10
+
+
+# ----------------------------------------------------------------------------
+# The "fixed" pattern ("Sparse-трансформеры" page, section "Основные шаблоны
+# разреженности"): local attention inside blocks of `area` tokens, plus the
+# last `summary` positions of every block as keys for all later queries.
+
+def fixed_sets(N, q, A, c, causal=1):
+    s = set(range((q // A) * A, min(N, (q // A) * A + A)))
+    s |= {kv for kv in range(N) if kv % A >= A - c}
+    if causal:
+        s &= set(range(q + 1))
+    return s
+
+
+@pytest.mark.parametrize("N,A,c", [(1024, 128, 16), (1000, 100, 10), (333, 64, 1), (257, 32, 32)])
+def test_fixed_pattern_pair_count_closed_form(N, A, c):
+    # causal: q mod A + 1 keys of its own block, plus c summary keys in each earlier block
+    p = Pattern(window=-1, causal=1, area=A, summary=c)
+    closed = sum(q % A + 1 + (q // A) * min(c, A) for q in range(N))
+    if c >= A:
+        closed = N * (N + 1) // 2  # every key is a summary key: dense causal
+    assert oracle.count_pairs(p, N) == closed
+
+
+@pytest.mark.parametrize("p,N", [(Pattern(window=-1, causal=1, area=8, summary=2), 37),
+                                 (Pattern(window=1, causal=0, area=6, summary=1), 29),
+                                 (Pattern(window=-1, sinks=2, causal=1, area=10, summary=3), 41)])
+def test_fixed_pattern_brute_force_and_sdpa(p, N):
+    def sets(q):
+        s = fixed_sets(N, q, p.area, p.summary, p.causal) | nc_sets(N, q, Pattern(
+            window=p.window, sinks=p.sinks, n_global=p.n_global, causal=p.causal, area=p.area))
+        return s
+    for q in range(N):
+        for kv in range(N):
+            assert oracle.allowed(p, q, kv) == (kv in sets(q))
+    B, Hq, Hkv, D = 1, 2, 1, 8
+    qq, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=N + 1)
+    O, _ = oracle.attention(qq, k, v, p, 0.4)
+    mask = torch.zeros(N, N, dtype=torch.bool)
+    for qi in range(N):
+        mask[qi, sorted(sets(qi))] = True
+    kt, vt = to_f64(k).repeat_interleave(2, 1), to_f64(v).repeat_interleave(2, 1)
+    ref = torch.nn.functional.scaled_dot_product_attention(to_f64(qq), kt, vt, attn_mask=mask, scale=0.4)
+    assert np.abs(O - ref.numpy()).max() < 1e-12
+
+
+def test_fixed_pattern_zero_query_lse():
+    N, D, A, c = 1024, 8, 128, 16
+    q = np.zeros((1, 1, N, D), dtype=np.uint16)
+    _, k, v = synth.qkv(1, 1, 1, N, D, seed=3)
+    _, LSE = oracle.attention(q, k, v, Pattern(window=-1, causal=1, area=A, summary=c), 0.5)
+    cnt = np.array([r % A + 1 + (r // A) * c for r in range(N)])
+    assert np.abs(LSE[0, 0] - np.log(cnt)).max() < 1e-12
+
+
+def test_fixed_pattern_gradients_match_finite_differences():
+    assert fd_pin_holds(oracle.default(), (1, 1, 1, 12, 2, Pattern(window=-1, causal=1, area=4, summary=1)))
