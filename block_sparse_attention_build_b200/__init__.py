@@ -53,7 +53,8 @@ class SparseAttnError(RuntimeError):
 
 class _Pattern(ctypes.Structure):
     _fields_ = [("causal", ctypes.c_int32), ("window", ctypes.c_int32), ("sinks", ctypes.c_int32),
-                ("stride", ctypes.c_int32), ("n_global", ctypes.c_int32), ("area", ctypes.c_int32)]
+                ("stride", ctypes.c_int32), ("n_global", ctypes.c_int32), ("area", ctypes.c_int32),
+                ("summary", ctypes.c_int32)]
 
 
 class _BlockMask(ctypes.Structure):
@@ -118,7 +119,8 @@ def _check(status: int, where: str) -> None:
 class Pattern:
     """allowed(q, kv) = (not causal or q >= kv) and ((window >= 0 and |q - kv| <= window)
     or kv < sinks or (stride > 0 and (q - kv) % stride == 0) or kv < n_global or q < n_global
-    or (area > 0 and q // area == kv // area)).  A stride needs causal = 1."""
+    or (area > 0 and q // area == kv // area)
+    or (area > 0 and summary > 0 and kv % area >= area - summary)).  A stride needs causal = 1."""
 
     window: int = -1
     sinks: int = 0
@@ -126,9 +128,10 @@ class Pattern:
     n_global: int = 0
     causal: int = 1
     area: int = 0
+    summary: int = 0
 
     def _c(self) -> _Pattern:
-        return _Pattern(self.causal, self.window, self.sinks, self.stride, self.n_global, self.area)
+        return _Pattern(self.causal, self.window, self.sinks, self.stride, self.n_global, self.area, self.summary)
 
 
 class BlockMask:

@@ -70,7 +70,9 @@ bool all_allowed(const sa_pattern& p, const Rect& r)
 int pattern_status(const sa_pattern* p)
 {
     if (!p) return SA_ERR_INVALID_ARG;
-    if (p->window < -1 || p->sinks < 0 || p->stride < 0 || p->n_global < 0 || p->area < 0) return SA_ERR_INVALID_ARG;
+    if (p->window < -1 || p->sinks < 0 || p->stride < 0 || p->n_global < 0 || p->area < 0 || p->summary < 0)
+        return SA_ERR_INVALID_ARG;
+    if (p->summary > 0 && p->area == 0) return SA_ERR_INVALID_ARG;
     if (p->causal != 0 && p->causal != 1) return SA_ERR_UNSUPPORTED;
     if (p->stride > 0 && (p->causal == 0 || p->area > 0)) return SA_ERR_UNSUPPORTED;
     return SA_OK;
@@ -80,8 +82,21 @@ int pattern_status(const sa_pattern* p)
 // the others the per-row interval count.
 bool general_form(const sa_pattern& p) { return p.causal == 0 || p.area > 0; }
 
-// Allowed keys of row q as a union of closed intervals (no stride), clipped
-// to [lo, hi]; returns how many keys of [lo, hi] it holds.
+// Summary keys (kv mod A >= A - c) in [0, n].
+int64_t summary_upto(int64_t n, int64_t A, int64_t c)
+{
+    if (n < 0) return 0;
+    const int64_t m = n + 1;
+    return (m / A) * c + std::max<int64_t>(0, m % A - (A - c));
+}
+int64_t summary_in(int64_t x, int64_t y, int64_t A, int64_t c)
+{
+    return x > y ? 0 : summary_upto(y, A, c) - summary_upto(x - 1, A, c);
+}
+
+// Allowed keys of row q as a union of closed intervals (no stride) and the
+// periodic summary columns, clipped to [lo, hi]; returns how many keys of
+// [lo, hi] it holds.
 int64_t row_keys_in(const sa_pattern& p, int64_t N, int64_t q, int64_t lo, int64_t hi)
 {
     if (p.causal) hi = std::min(hi, q);
@@ -114,17 +129,26 @@ int64_t row_keys_in(const sa_pattern& p, int64_t N, int64_t q, int64_t lo, int64
                 std::swap(a[i], a[j]);
                 std::swap(b[i], b[j]);
             }
+    // summary columns not already inside the intervals: all of them in [lo, hi]
+    // minus those inside each merged interval
+    const int64_t A = p.area, c = std::min<int64_t>(p.summary, p.area);
     int64_t total = 0, cur_a = 0, cur_b = -1;
+    if (c > 0) total += summary_in(lo, hi, A, c);
+    auto close = [&]() {
+        if (cur_b < cur_a) return;
+        total += cur_b - cur_a + 1;
+        if (c > 0) total -= summary_in(cur_a, cur_b, A, c);
+    };
     for (int i = 0; i < n; i++) {
         if (a[i] > cur_b + 1 || cur_b < cur_a) {
-            if (cur_b >= cur_a) total += cur_b - cur_a + 1;
+            close();
             cur_a = a[i];
             cur_b = b[i];
         } else {
             cur_b = std::max(cur_b, b[i]);
         }
     }
-    if (cur_b >= cur_a) total += cur_b - cur_a + 1;
+    close();
     return total;
 }
 

@@ -80,6 +80,7 @@ int bwd_run(const void* Q, const void* K, const void* V, const void* O, const fl
     p.n_global = pt.n_global;
     p.causal = pt.causal;
     p.area = pt.area > s.N ? s.N : pt.area;
+    p.summary = pt.summary < pt.area ? pt.summary : pt.area;
     p.scale_log2 = scale * 1.44269504088896340736f;
     p.scale = scale;
 
@@ -127,7 +128,9 @@ extern "C" int sparse_attn_bwd(const void* Q, const void* K, const void* V, cons
     const sa_pattern pt = *pattern;
     if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
-    if (pt.window < -1 || pt.sinks < 0 || pt.stride < 0 || pt.n_global < 0 || pt.area < 0) return SA_ERR_INVALID_ARG;
+    if (pt.window < -1 || pt.sinks < 0 || pt.stride < 0 || pt.n_global < 0 || pt.area < 0 || pt.summary < 0)
+        return SA_ERR_INVALID_ARG;
+    if (pt.summary > 0 && pt.area == 0) return SA_ERR_INVALID_ARG;
     if (pt.causal != 0 && pt.causal != 1) return SA_ERR_UNSUPPORTED;
     if (pt.stride > 0 && (pt.causal == 0 || pt.area > 0)) return SA_ERR_UNSUPPORTED;
     if (s.D != 64 && s.D != 128) return SA_ERR_UNSUPPORTED;

@@ -77,7 +77,7 @@ struct BwdParams {
     int32_t* status;
     long long timeout;       // SM cycles per bounded wait
     int32_t T, N, B, Hq, Hkv, group;
-    int32_t window, sinks, stride, n_global, causal, area;  // window and area clipped to N
+    int32_t window, sinks, stride, n_global, causal, area, summary;  // window, area clipped to N; summary <= area
     float scale_log2;        // scale * log2(e)
     float scale;
 };
@@ -128,6 +128,7 @@ __device__ __forceinline__ uint32_t bwd_allow_word(const BwdParams& p, int qb, i
     if (kv >= p.N) return 0u;
     const uint32_t in_range = bwd_bits((p.causal ? kv : 0) - qb, p.N - 1 - qb);  // (kv <=) q < N
     if (kv < max(p.sinks, p.n_global)) return in_range;
+    if (p.summary > 0 && kv % p.area >= p.area - p.summary) return in_range;  // a summary column
     uint32_t m = 0u;
     if (p.window >= 0) m |= bwd_bits(kv - p.window - qb, kv + p.window - qb);
     if (p.n_global > 0) m |= bwd_bits(0, p.n_global - 1 - qb);

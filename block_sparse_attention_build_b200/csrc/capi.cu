@@ -91,7 +91,9 @@ int launch_any(int D, int block, const CUtensorMap& mq, const CUtensorMap& mk, c
 // or with stripes).
 int pattern_status(const sa_pattern& pt)
 {
-    if (pt.window < -1 || pt.sinks < 0 || pt.stride < 0 || pt.n_global < 0 || pt.area < 0) return SA_ERR_INVALID_ARG;
+    if (pt.window < -1 || pt.sinks < 0 || pt.stride < 0 || pt.n_global < 0 || pt.area < 0 || pt.summary < 0)
+        return SA_ERR_INVALID_ARG;
+    if (pt.summary > 0 && pt.area == 0) return SA_ERR_INVALID_ARG;
     if (pt.causal != 0 && pt.causal != 1) return SA_ERR_UNSUPPORTED;
     if (pt.stride > 0 && (pt.causal == 0 || pt.area > 0)) return SA_ERR_UNSUPPORTED;
     return SA_OK;
@@ -213,6 +215,7 @@ int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* m
         hp.pat[i].n_global = patterns[i].n_global;
         hp.pat[i].causal = patterns[i].causal;
         hp.pat[i].area = clip_to(patterns[i].area, s.N);
+        hp.pat[i].summary = patterns[i].summary < patterns[i].area ? patterns[i].summary : patterns[i].area;
     }
     for (int h = 0; h < s.Hq; h++) hp.head[h] = per_head ? static_cast<uint8_t>(head_pattern[h]) : 0;
     return launch_any<true>(s.D, mask->block, mq, mk, mv, mo, p, hp, g, st);
@@ -335,4 +338,4 @@ extern "C" const char* sparse_attn_status_string(int status)
     }
 }
 
-extern "C" int32_t sparse_attn_version(void) { return 200; }
+extern "C" int32_t sparse_attn_version(void) { return 201; }

@@ -86,7 +86,7 @@ extern "C" int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void*
     if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
     // the causal band / sinks / stride / global forms only (no pattern table here)
-    if (pattern->causal != 1 || pattern->area != 0) return SA_ERR_UNSUPPORTED;
+    if (pattern->causal != 1 || pattern->area != 0 || pattern->summary != 0) return SA_ERR_UNSUPPORTED;
     if (pattern->window < -1 || pattern->sinks < 0 || pattern->stride < 0 || pattern->n_global < 0)
         return SA_ERR_INVALID_ARG;
     if (s.D != 64 && s.D != 128) return SA_ERR_UNSUPPORTED;

@@ -107,7 +107,7 @@ struct PatternRef {
     const int32_t* kv_count;  // [T]
     const int32_t* kv_index;  // [T * T]
     const uint8_t* kv_full;   // [T * T]
-    int32_t window, sinks, stride, n_global, causal, area;
+    int32_t window, sinks, stride, n_global, causal, area, summary;  // summary <= area
 };
 struct HeadPatterns {
     PatternRef pat[kMaxPatterns];
@@ -905,6 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int cols = max(p.sinks, p.n_global);
         int pw = p.window, ps = p.stride, pg = p.n_global;  // this slot's pattern (per unit when MULTI)
         int qlim = 0, a_lo = 0, a_hi = -1;                   // MULTI: last allowed key (causal bound), stripe
+        int s_area = 0, s_cnt = 0;                           // MULTI: summary columns kv mod s_area >= s_area - s_cnt
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
         int steps = 0, units = 0;
         int units_b = 0;   // slot A only: completed phases of o_full[1] (slot B's last PV of a unit)
@@ -931,6 +932,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pg = pr.n_global;
                 cols = max(pr.sinks, pr.n_global);
                 qlim = pr.causal ? q : p.N - 1;
+                s_area = pr.area;
+                s_cnt = pr.summary;
                 if (pr.area > 0) {
                     a_lo = (q / pr.area) * pr.area;
                     a_hi = a_lo + pr.area - 1;
@@ -964,7 +967,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int base = 32 * w;
                         uint32_t m = bits_between(0, cols - 1 - kv0 - base);
                         if (pw >= 0) m |= bits_between(dq - pw - base, MULTI ? dq + pw - base : 31);
-                        if constexpr (MULTI) m |= bits_between(a_lo - kv0 - base, a_hi - kv0 - base);
+                        if constexpr (MULTI) {
+                            m |= bits_between(a_lo - kv0 - base, a_hi - kv0 - base);
+                            if (s_cnt > 0) {  // the summary columns of the stripes this word touches
+                                const int kb = kv0 + base;
+                                for (int st = kb / s_area; st * s_area <= kb + 31; st++)
+                                    m |= bits_between(st * s_area + s_area - s_cnt - kb, st * s_area + s_area - 1 - kb);
+                            }
+                        }
                         if (ps > 0) {
                             int r0 = dq % ps;
                             if (r0 < 0) r0 += ps;

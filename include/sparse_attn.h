@@ -52,16 +52,21 @@ extern "C" {
  *           or kv < sinks
  *           or (stride > 0 and (q - kv) mod stride == 0)
  *           or kv < n_global or q < n_global
- *           or (area > 0 and floor(q / area) == floor(kv / area)) ).
+ *           or (area > 0 and floor(q / area) == floor(kv / area))
+           or (area > 0 and summary > 0 and kv mod area >= area - summary) ).
  * Pages: "Sparse Attention", sections "Gängige Sparsity-Muster" and "Ein
  * Muster in Einsparungen verwandeln" (window inclusive, as in local_plus_sinks),
  * and section "Anwendungen" (Area Attention: attention only inside stripes of
  * consecutive tokens); "Sparse-трансформеры", section "Основные шаблоны
  * разреженности" (without causality the window reaches w tokens on both
- * sides).  The stride counts back from the query (every s-th prior token) and
+ * sides), and the "fixed" pattern of the same section: blocks of `area`
+ * tokens with local attention inside, linked through summary positions, read
+ * as the last `summary` positions of every block.  The stride counts back from
+ * the query (every s-th prior token) and
  * needs causal == 1; with causal == 1 the global rows and columns stay causal.
  * Supported forms: causal == 1 with any of the rules; causal == 0 with window,
- * sinks, n_global and area (stride > 0 gives SA_ERR_UNSUPPORTED).
+ * sinks, n_global, area and summary (stride > 0 gives SA_ERR_UNSUPPORTED, as
+ * does a stride with area); summary > 0 needs area > 0 (SA_ERR_INVALID_ARG).
  */
 typedef struct {
     int32_t causal;
@@ -69,7 +74,8 @@ typedef struct {
     int32_t sinks;
     int32_t stride;
     int32_t n_global;
-    int32_t area;  /* stripe length; 0 for none */
+    int32_t area;     /* stripe (block) length; 0 for none */
+    int32_t summary;  /* summary positions at the end of every stripe; 0 for none */
 } sa_pattern;
 
 /*
@@ -108,7 +114,8 @@ int32_t sparse_attn_num_tiles(int64_t N, int32_t block);
  * partial or full and write the lists described at sa_block_mask: for causal
  * patterns without stripes analytically per tile (no per-pair or per-row
  * loop); for the others (causal == 0, or area > 0) from each row's allowed
- * keys, a union of at most four intervals, counted per tile.  Host-only; `out` holds
+ * keys, a union of at most four intervals plus the periodic summary columns,
+ * counted per tile in closed form.  Host-only; `out` holds
  * caller-owned host arrays with capacity out->n_q_tiles rows of
  * out->n_kv_tiles entries, both at least T (else SA_ERR_BUFFER_TOO_SMALL).
  * block is 64 or 128; N >= 0 (N = 0 gives T = 0).

@@ -27,6 +27,7 @@ class Workload:
     seed: int = 0
     causal: int = 1
     area: int = 0
+    summary: int = 0
 
     @property
     def scale(self) -> float:
@@ -34,7 +35,7 @@ class Workload:
 
     def pattern_args(self) -> dict:
         return dict(window=self.window, sinks=self.sinks, stride=self.stride, n_global=self.n_global,
-                    causal=self.causal, area=self.area)
+                    causal=self.causal, area=self.area, summary=self.summary)
 
 
 WORKLOADS = {

@@ -42,7 +42,7 @@ def test_version_and_status_strings():
 
 def opattern(p: sa.Pattern):
     return oracle.Pattern(window=p.window, sinks=p.sinks, stride=p.stride, n_global=p.n_global, causal=p.causal,
-                          area=p.area)
+                          area=p.area, summary=p.summary)
 
 
 SWEEP = [
@@ -230,6 +230,13 @@ GENERAL = [
                             (300, 1, 2, 0, 130), (0, 0, 0, 0, 1), (-1, 0, 0, 0, 0), (5000, 0, 0, 0, 0)]
     for N in (1, 100, 500, 1000, 1600)
     for b in (64, 128)
+] + [
+    # the fixed pattern: blocks of `area` plus the last `summary` positions of every block
+    (sa.Pattern(window=w, sinks=s, causal=c, area=a, summary=m), N, b)
+    for (w, s, c, a, m) in [(-1, 0, 1, 128, 16), (-1, 0, 1, 100, 10), (-1, 0, 0, 64, 8), (3, 2, 1, 50, 7),
+                            (-1, 0, 1, 16, 16), (-1, 0, 1, 40, 100), (10, 0, 0, 33, 1)]
+    for N in (1, 300, 1000)
+    for b in (64, 128)
 ]
 
 
@@ -252,7 +259,9 @@ def test_general_pattern_errors():
     for p, rc in [(sa.Pattern(window=4, stride=8, causal=0), sa.SA_ERR_UNSUPPORTED),
                   (sa.Pattern(window=4, stride=8, area=64), sa.SA_ERR_UNSUPPORTED),
                   (sa.Pattern(window=4, causal=2), sa.SA_ERR_UNSUPPORTED),
-                  (sa.Pattern(window=4, area=-1), sa.SA_ERR_INVALID_ARG)]:
+                  (sa.Pattern(window=4, area=-1), sa.SA_ERR_INVALID_ARG),
+                  (sa.Pattern(window=4, summary=2), sa.SA_ERR_INVALID_ARG),       # summary needs area
+                  (sa.Pattern(window=4, area=8, summary=-1), sa.SA_ERR_INVALID_ARG)]:
         with pytest.raises(sa.SparseAttnError) as e:
             sa.build_block_mask(p, 100, 64)
         assert e.value.status == rc
@@ -274,3 +283,10 @@ def test_general_pattern_errors():
     big = sa._Shape(1, 300, 300, 100, 128)  # general forms use the pattern-table kernel: Hq <= 256
     assert sa.lib.sparse_attn_fwd(fake, fake, fake, ctypes.byref(m), ctypes.byref(area), ctypes.byref(big), 0.1,
                                   fake, fake, None) == sa.SA_ERR_UNSUPPORTED
+
+
+def test_fixed_pattern_pair_count_closed_form():
+    # causal: q mod A + 1 keys of the own block, plus c summary keys in every earlier block
+    for N, A, c in [(1024, 128, 16), (1000, 100, 10), (333, 64, 1)]:
+        assert sa.count_pairs(sa.Pattern(window=-1, area=A, summary=c), N) == sum(
+            q % A + 1 + (q // A) * c for q in range(N))

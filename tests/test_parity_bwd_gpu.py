@@ -32,7 +32,7 @@ def to_dev(bits: np.ndarray) -> torch.Tensor:
 
 def opattern(p: sa.Pattern):
     return oracle.Pattern(window=p.window, sinks=p.sinks, stride=p.stride, n_global=p.n_global, causal=p.causal,
-                          area=p.area)
+                          area=p.area, summary=p.summary)
 
 
 def inputs(B, Hq, Hkv, N, D, seed):
@@ -84,6 +84,8 @@ CASES = [
     (2, 2, 1, 1000, 128, sa.Pattern(window=100, causal=0)),            # two-sided window, GQA
     (1, 2, 2, 900, 128, sa.Pattern(window=-1, sinks=4, n_global=3, causal=0, area=200)),
     (1, 2, 2, 1100, 64, sa.Pattern(window=20, causal=1, area=300)),    # block-causal stripes + band
+    (1, 2, 2, 2048, 128, sa.Pattern(window=-1, area=128, summary=16)),  # fixed pattern
+    (1, 2, 1, 1000, 64, sa.Pattern(window=-1, causal=0, area=24, summary=3)),
 ]
 
 

@@ -51,7 +51,7 @@ def compare(O, LSE, Oref, LSEref):
 
 def opattern(p: sa.Pattern):
     return oracle.Pattern(window=p.window, sinks=p.sinks, stride=p.stride, n_global=p.n_global, causal=p.causal,
-                          area=p.area)
+                          area=p.area, summary=p.summary)
 
 
 SMALL = [
@@ -255,6 +255,9 @@ GENERAL_CASES = [
     (1, 3, 3, 900, 128, sa.Pattern(window=-1, sinks=4, n_global=3, causal=0, area=200), 128),
     (1, 2, 2, 1100, 64, sa.Pattern(window=20, causal=1, area=300), 64),       # block-causal stripes + band
     (1, 1, 1, 333, 128, sa.Pattern(window=10, causal=0, area=50), 128),       # ragged, stripes inside a tile
+    (1, 2, 2, 2048, 128, sa.Pattern(window=-1, area=128, summary=16), 128),   # fixed pattern, blocks = tiles
+    (2, 2, 1, 1000, 64, sa.Pattern(window=-1, area=100, summary=10), 64),     # fixed pattern, ragged blocks
+    (1, 2, 2, 700, 128, sa.Pattern(window=-1, causal=0, area=24, summary=3), 128),  # short blocks, no causality
 ]
 
 
