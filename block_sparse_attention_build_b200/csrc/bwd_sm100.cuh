@@ -21,23 +21,23 @@
 //                    the fp32 accumulator with vector reductions;
 //   bwd_dq_kernel    dQ accumulator -> bf16.
 //
-// bwd_kernel, 320 threads: warps 0-7 the element-wise work (two threads per
-// kv row, each one half of the columns; tensor-memory lane = kv row), warp 8
-// the TMA producer, warp 9 tensor memory allocation and the single
-// MMA-issuing lane.  Per step (one query
-// tile of one head):
-//   Sᵀ = K Qᵀ, dPᵀ = V dOᵀ                 tcgen05 SS, fp32 in tensor memory
+// bwd_kernel, 448 threads: warps 0-7 the element-wise work (two threads per
+// kv row, tensor-memory lane = kv row), warps 8-11 the dQ read-out and
+// reductions, warp 12 the TMA producer, warp 13 tensor memory allocation and
+// the single MMA-issuing lane.  A step (one query tile of one head) runs as
+// two half-steps of 64 query columns, double-buffered in tensor memory (half
+// h in columns 128h .. 128h+127; dV, dK in 256 .. 256+2D), so that the tensor
+// core computes one half while the element-wise warps work on the other:
+//   Sᵀ = K Qᵀ, dPᵀ = V dOᵀ                 tcgen05 SS, N = 64, fp32 in tensor memory
 //   Pᵀ = exp2(Sᵀ·scale·log2e − LSE₂)      masked on partial tiles
 //   dSᵀ = Pᵀ ∘ (dPᵀ − Δ) · scale           both bf16 back into the Sᵀ columns of
 //                                           tensor memory; dSᵀ also to shared memory
-//   dV += Pᵀ dO, dK += dSᵀ Q               TS: A from tensor memory
+//   dV += Pᵀ dO, dK += dSᵀ Q               TS: A from tensor memory, K = 64
 //   dQᵀ = Kᵀ dSᵀ                            SS, both operands MN-major, into the dPᵀ
-//                columns with lanes = features; read out (releasing tensor
-//                memory for the next step's MMAs) and reduced into global
-//                memory, each warp instruction adding one query row's 32
-//                consecutive features (one 128-byte line).
-// Shared memory carries only the SS operands, the TMA fills and the dSᵀ tile:
-// its bandwidth, not the tensor pipe, is what bounds a step of this design.
+//                columns with lanes = features; the dQ warps read it out
+//                (releasing the buffer) and reduce it into global memory,
+//                each warp instruction adding one query row's 32 consecutive
+//                features (one 128-byte line).
 // Every wait is bounded; on expiry a role sets a status bit, raises an abort
 // flag and leaves its loop; the MMA lane drains its MMAs and the producer its
 // copies before tensor memory is freed.
@@ -52,10 +52,12 @@
 
 namespace sa {
 
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 448;
 constexpr int kBwdElemThreads = 256;  // warps 0-7
-constexpr int kBwdProducerWarp = 8;
-constexpr int kBwdMmaWarp = 9;
+constexpr int kBwdDqWarp0 = 8;        // warps 8-11
+constexpr int kBwdDqThreads = 128;
+constexpr int kBwdProducerWarp = 12;
+constexpr int kBwdMmaWarp = 13;
 constexpr int kBwdTile = 128;  // query and kv tile edge (the block mask's block)
 
 enum : int32_t {
@@ -92,11 +94,11 @@ struct BwdCfg {
     static constexpr int kOffdO = kOffQ + 2 * kTileBytes;  // two buffers
     static constexpr int kOffdS = kOffdO + 2 * kTileBytes; // dSᵀ: 128 kv rows x 128 q columns, two panels
     static constexpr int kOffBar = kOffdS + 2 * kPanel;
-    static constexpr int kNumBars = 10;
+    static constexpr int kNumBars = 14;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tensor-memory base, abort flag
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
-    static constexpr uint32_t kColS = 0;         // Sᵀ (fp32), then Pᵀ and dSᵀ (bf16 pairs), 16 columns each per 32
-    static constexpr uint32_t kColdP = 128;      // dPᵀ (fp32), then the step's dQᵀ tile (lanes = features)
+    // half h of a step: Sᵀ (fp32, then Pᵀ and dSᵀ bf16 pairs) in columns 128h ..
+    // 128h+63, dPᵀ (fp32, then the half's dQᵀ with lanes = features) in 128h+64 .. +127
     static constexpr uint32_t kColdV = 256;
     static constexpr uint32_t kColdK = 256 + D;
     static constexpr uint32_t kTmemCols = 512;
@@ -222,14 +224,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint8_t* sdO = smem + C::kOffdO;
     uint8_t* sdS = smem + C::kOffdS;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-    uint64_t* kv_full = bars;         // K and V landed
-    uint64_t* qd_full = bars + 1;     // [2] Q and dO of a step landed
-    uint64_t* qd_empty = bars + 3;    // [2] the step's dV and dK MMAs are done with them
-    uint64_t* s_full = bars + 5;      // Sᵀ and dPᵀ are in tensor memory
-    uint64_t* ds_full = bars + 6;     // Pᵀ (tensor memory) and dSᵀ (shared memory) written (256 threads)
-    uint64_t* dq_full = bars + 7;     // the step's dQ tile is in tensor memory (and every earlier MMA done)
-    uint64_t* dq_empty = bars + 8;    // the dQ tile has been read out of tensor memory (256 threads)
-    uint64_t* drain = bars + 9;
+    uint64_t* kv_full = bars;        // K and V landed
+    uint64_t* qd_full = bars + 1;    // [2] Q and dO of a step landed
+    uint64_t* qd_empty = bars + 3;   // [2] both halves' dV and dK MMAs are done with them
+    uint64_t* s_full = bars + 5;     // [2] per half: Sᵀ and dPᵀ are in tensor memory
+    uint64_t* ds_full = bars + 7;    // [2] per half: Pᵀ, dSᵀ written (256 element-wise threads)
+    uint64_t* dq_full = bars + 9;    // [2] per half: dQᵀ in tensor memory (and every earlier MMA done)
+    uint64_t* dq_empty = bars + 11;  // [2] per half: dQᵀ read out of tensor memory (128 dQ threads)
+    uint64_t* drain = bars + 13;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -242,17 +244,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int hkv = bh % p.Hkv;
     const int n_list = min(max(__ldg(&p.t_count[c]), 0), p.T);
     const int steps = p.group * n_list;
+    const int halves = 2 * steps;  // half-step k: step k / 2, query columns 64 (k % 2) .. +63
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
         for (int x = 0; x < 2; x++) {
             mbar_init(&qd_full[x], 1);
             mbar_init(&qd_empty[x], 1);
+            mbar_init(&s_full[x], 1);
+            mbar_init(&ds_full[x], kBwdElemThreads);
+            mbar_init(&dq_full[x], 1);
+            mbar_init(&dq_empty[x], kBwdDqThreads);
         }
-        mbar_init(s_full, 1);
-        mbar_init(ds_full, kBwdElemThreads);
-        mbar_init(dq_full, 1);
-        mbar_init(dq_empty, kBwdElemThreads);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -321,13 +324,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     } else if (warp == kBwdMmaWarp) {
         // ================================================================ MMA issuer
         // The warp runs converged; one elected lane issues each MMA and commit.
+        // Order: Sᵀ, dPᵀ of half k + 1 (into buffer (k + 1) % 2, free once the
+        // dQ warps have read half k - 1's dQᵀ), then dV, dK and dQᵀ of half k
+        // (once the element-wise warps have written its Pᵀ and dSᵀ): the tensor
+        // core computes one half while the element-wise warps work on the other.
         if (steps > 0) {
-            constexpr uint32_t id_s = idesc_bf16_f32(kBwdTile, kBwdTile, false, false);
-            constexpr uint32_t id_kv = idesc_bf16_f32(kBwdTile, D, false, true);
-            // dQᵀ = Kᵀ dSᵀ: M = 128 feature rows (at D = 64 the upper 64 read the V tile
-            // and are never used), N = 128 query rows, both operands MN-major
-            constexpr uint32_t id_q = idesc_bf16_f32(kBwdTile, kBwdTile, true, true);
+            constexpr uint32_t id_s = idesc_bf16_f32(kBwdTile, 64, false, false);    // Sᵀ, dPᵀ: N = 64 query rows
+            constexpr uint32_t id_kv = idesc_bf16_f32(kBwdTile, D, false, true);     // dV, dK
+            // dQᵀ = Kᵀ dSᵀ: M = 128 feature rows (at D = 64 the upper 64 read the V
+            // tile and are never used), N = 64 query rows, both operands MN-major
+            constexpr uint32_t id_q = idesc_bf16_f32(kBwdTile, 64, true, true);
             constexpr uint32_t kTileU = C::kTileBytes >> 4;  // descriptor units (16 bytes)
+            constexpr uint32_t kHalfRowsU = (64 * 128) >> 4;  // 64 rows of a 128-byte panel
             const uint64_t d0 = smem_desc_sw128(smem_addr(sK), 16, 1024);
             const uint32_t hi = static_cast<uint32_t>(d0 >> 32);
             const uint32_t k_km = static_cast<uint32_t>(d0);
@@ -348,183 +356,214 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (elect_one()) tc_commit(bar);
                 __syncwarp();
             };
-            bool ok = wait(kv_full, 0);
-            for (int j = 0; j < steps && ok; j++) {
-                const int buf = j & 1;
-                const uint32_t bo = buf * kTileU;
-                ok = wait(&qd_full[buf], (j >> 1) & 1) && (j == 0 || wait(dq_empty, (j - 1) & 1));
-                if (!ok || __any_sync(0xffffffffu, *abort_flag != 0)) break;
-                tc_fence_after_sync();
-                // Sᵀ = K Qᵀ and dPᵀ = V dOᵀ (M = kv rows, N = query rows, K = D)
+            // Sᵀ = K Qᵀ and dPᵀ = V dOᵀ of half k (M = kv rows, N = 64 query rows, K = D)
+            auto issue_sdp = [&](int k) {
+                const int hf = k & 1;
+                const uint32_t bo = ((k >> 1) & 1) * kTileU + hf * kHalfRowsU;
+                const uint32_t col = tmem + hf * 128;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; kk++) {
                     if (elect_one())
-                        mma_ss(tmem + C::kColS, desc_from_halves(k_km + km(kk), hi),
-                               desc_from_halves(q_km + bo + km(kk), hi), id_s, kk > 0 ? 1u : 0u);
+                        mma_ss(col, desc_from_halves(k_km + km(kk), hi), desc_from_halves(q_km + bo + km(kk), hi), id_s,
+                               kk > 0 ? 1u : 0u);
                     __syncwarp();
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; kk++) {
                     if (elect_one())
-                        mma_ss(tmem + C::kColdP, desc_from_halves(v_km + km(kk), hi),
-                               desc_from_halves(o_km + bo + km(kk), hi), id_s, kk > 0 ? 1u : 0u);
+                        mma_ss(col + 64, desc_from_halves(v_km + km(kk), hi), desc_from_halves(o_km + bo + km(kk), hi),
+                               id_s, kk > 0 ? 1u : 0u);
                     __syncwarp();
                 }
-                commit(s_full);
-                ok = wait(ds_full, j & 1);
+                commit(&s_full[hf]);
+            };
+            bool ok = wait(kv_full, 0) && wait(&qd_full[0], 0);
+            if (ok) {
+                tc_fence_after_sync();
+                issue_sdp(0);
+            }
+            for (int k = 0; k < halves && ok; k++) {
+                const int hf = k & 1;
+                const int j = k >> 1;
+                const int kn = k + 1;
+                if (kn < halves) {
+                    const int jn = kn >> 1;
+                    // buffer kn % 2 is free once half kn - 2's dQᵀ has been read (all MMAs up to it done)
+                    ok = (kn < 2 || wait(&dq_empty[kn & 1], ((kn - 2) >> 1) & 1)) &&
+                         ((kn & 1) || wait(&qd_full[jn & 1], (jn >> 1) & 1));
+                    if (!ok || __any_sync(0xffffffffu, *abort_flag != 0)) break;
+                    tc_fence_after_sync();
+                    issue_sdp(kn);
+                }
+                ok = wait(&ds_full[hf], j & 1);
                 if (!ok || __any_sync(0xffffffffu, *abort_flag != 0)) break;
                 tc_fence_after_sync();
-                // dV += Pᵀ dO and dK += dSᵀ Q (M = kv rows, N = D, K = query rows), A
-                // from tensor memory: query columns 32c .. 32c+31 (c = kk / 2) hold
-                // Pᵀ in packed columns 32c .. 32c+15 and dSᵀ in 32c+16 .. 32c+31
+                const uint32_t bo = (j & 1) * kTileU + hf * kHalfRowsU;
+                const uint32_t scol = tmem + hf * 128;
+                // dV += Pᵀ dO and dK += dSᵀ Q over this half's 64 query rows (K = 64): A
+                // from tensor memory, query columns 32u .. 32u+31 of the half hold Pᵀ
+                // in packed columns 32u .. 32u+15 and dSᵀ in 32u+16 .. 32u+31
 #pragma unroll
-                for (int kk = 0; kk < kBwdTile / 16; kk++) {
+                for (int kk = 0; kk < 4; kk++) {
                     if (elect_one())
-                        mma_ts(tmem + C::kColdV, tmem + C::kColS + (kk / 2) * 32 + (kk % 2) * 8,
-                               desc_from_halves(o_mn + bo + mn(kk), hi), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts(tmem + C::kColdV, scol + (kk / 2) * 32 + (kk % 2) * 8,
+                               desc_from_halves(o_mn + bo + mn(kk), hi), id_kv, (k > 0 || kk > 0) ? 1u : 0u);
                     __syncwarp();
                 }
 #pragma unroll
-                for (int kk = 0; kk < kBwdTile / 16; kk++) {
+                for (int kk = 0; kk < 4; kk++) {
                     if (elect_one())
-                        mma_ts(tmem + C::kColdK, tmem + C::kColS + (kk / 2) * 32 + 16 + (kk % 2) * 8,
-                               desc_from_halves(q_mn + bo + mn(kk), hi), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts(tmem + C::kColdK, scol + (kk / 2) * 32 + 16 + (kk % 2) * 8,
+                               desc_from_halves(q_mn + bo + mn(kk), hi), id_kv, (k > 0 || kk > 0) ? 1u : 0u);
                     __syncwarp();
                 }
-                commit(&qd_empty[buf]);
-                // dQᵀ = Kᵀ dSᵀ (M = feature rows, N = query rows, K = kv rows), into the dPᵀ columns
+                if (hf) commit(&qd_empty[j & 1]);
+                // dQᵀ = Kᵀ dSᵀ (M = feature rows, N = 64 query rows, K = kv rows), into
+                // the half's dPᵀ columns; dSᵀ of half hf is panel hf of the shared tile
 #pragma unroll
                 for (int kk = 0; kk < kBwdTile / 16; kk++) {
                     if (elect_one())
-                        mma_ss(tmem + C::kColdP, desc_from_halves(k_mn + mn(kk), hi),
-                               desc_from_halves(s_mn + mn(kk), hi), id_q, kk > 0 ? 1u : 0u);
+                        mma_ss(scol + 64, desc_from_halves(k_mn + mn(kk), hi),
+                               desc_from_halves(s_mn + hf * (C::kPanel >> 4) + mn(kk), hi), id_q, kk > 0 ? 1u : 0u);
                     __syncwarp();
                 }
-                commit(dq_full);
+                commit(&dq_full[hf]);
             }
             if (!ok && lane == 0) bwd_report(p, abort_flag, ST_BWD_MMA_WAIT);
             // every MMA issued so far is complete before tensor memory is freed
             commit(drain);
             if (!wait(drain, 0) && lane == 0) bwd_report(p, abort_flag, ST_BWD_DRAIN_WAIT);
         }
-    } else {
-        // ================================================================ element-wise warps 0-7
-        // Warp w serves tensor-memory lanes 32 (w % 4) .. +31 (kv rows of Sᵀ,
-        // dPᵀ, dK, dV; query rows of dQ) and column half h = w / 4: query
-        // columns 64h .. 64h+63 of Sᵀ / dPᵀ, columns h D/2 .. of dQ, dK, dV.
-        // Each warp decides to leave its loop as a whole (every test goes
-        // through a vote); the warps never wait on one another except through
-        // bounded mbarrier waits.
+    } else if (warp >= kBwdDqWarp0) {
+        // ================================================================ dQ warps 8-11
+        // Warp w reads lanes 32 (w % 4) .. +31 of each half's dQᵀ (lane = feature
+        // d, columns = the half's 64 query rows), releases the columns, then adds
+        // them to the fp32 accumulator: each reduction instruction covers one
+        // query row's 32 consecutive features (one 128-byte line).
         const int quarter = warp % 4;
-        const int half = warp / 4;
-        const int t = quarter * 32 + lane;  // kv row (and query row of dQ) of this thread
         const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
-        const int kv = c * kBwdTile + t;
-        const bool kv_ragged = (c + 1) * kBwdTile > p.N;
-        constexpr int kHalfD = D / 2;
+        const int dcol = quarter * 32 + lane;
         bool ok = true;
-        for (int j = 0; j < steps; j++) {
+        for (int k = 0; k < halves; k++) {
+            const int hf = k & 1;
+            const int j = k >> 1;
             int hq, r;
             bool full;
             step_of(j, hq, r, full);
-            const int q0 = r * kBwdTile;
+            const int qh = r * kBwdTile + hf * 64;  // first query row of the half
             const int64_t qrow0 = (int64_t(b) * p.Hq + hq) * p.N;
-            // LSE₂ and Δ of query column 64 half + 32 cc + lane, handed to the other lanes by shuffles
-            float lse_r[2], dl_r[2];
-#pragma unroll
-            for (int cc = 0; cc < 2; cc++) {
-                const int q = q0 + half * 64 + cc * 32 + lane;
-                lse_r[cc] = q < p.N ? __ldg(&p.lse2[qrow0 + q]) : INFINITY;
-                dl_r[cc] = q < p.N ? __ldg(&p.delta[qrow0 + q]) : 0.f;
-            }
-            ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, lim) && !*abort_flag);
+            ok = __all_sync(0xffffffffu, mbar_wait(&dq_full[hf], j & 1, lim) && !*abort_flag);
             if (!ok) break;
             tc_fence_after_sync();
-            const bool masked = !full || kv_ragged || q0 + kBwdTile > p.N;
-#pragma unroll 1
-            for (int cc = 0; cc < 2; cc++) {
-                const int col = half * 64 + cc * 32;  // first query column of the chunk
-                uint32_t s[32], d[32];
-                tmem_ld_32x32b_x32(tmem + lanes + C::kColS + col, s);
-                tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + col, d);
-                const float lse_c = cc == 0 ? lse_r[0] : lse_r[1];
-                const float dl_c = cc == 0 ? dl_r[0] : dl_r[1];
-                const uint32_t allow = masked ? bwd_allow_word(p, q0 + col, kv) : 0xffffffffu;
-                tmem_wait_ld();
-                reg_fence(s);
-                reg_fence(d);
-                uint32_t pk[16], gk[16];
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float l0 = __shfl_sync(0xffffffffu, lse_c, i);
-                    const float l1 = __shfl_sync(0xffffffffu, lse_c, i + 1);
-                    const float e0 = __shfl_sync(0xffffffffu, dl_c, i);
-                    const float e1 = __shfl_sync(0xffffffffu, dl_c, i + 1);
-                    float p0 = ex2_approx(fmaf(__uint_as_float(s[i]), p.scale_log2, -l0));
-                    float p1 = ex2_approx(fmaf(__uint_as_float(s[i + 1]), p.scale_log2, -l1));
-                    p0 = (allow >> i) & 1u ? p0 : 0.f;
-                    p1 = (allow >> (i + 1)) & 1u ? p1 : 0.f;
-                    const float g0 = p0 * (__uint_as_float(d[i]) - e0) * p.scale;
-                    const float g1 = p1 * (__uint_as_float(d[i + 1]) - e1) * p.scale;
-                    pk[i / 2] = pack_bf16x2(p0, p1);
-                    gk[i / 2] = pack_bf16x2(g0, g1);
-                }
-                // Pᵀ and dSᵀ (bf16 pairs) over the 32 Sᵀ columns of this chunk, just
-                // read by this thread: Pᵀ in col .. col+15, dSᵀ in col+16 .. col+31
-                tmem_st_32x32b_x16(tmem + lanes + C::kColS + col, pk);
-                tmem_st_32x32b_x16(tmem + lanes + C::kColS + col + 16, gk);
-                // dSᵀ row t, query columns col .. col+31: four 16-byte units of panel `half`
-                uint8_t* rowp = sdS + half * C::kPanel + t * 128;
-#pragma unroll
-                for (int k = 0; k < 4; k++) {
-                    const int u = cc * 4 + k;
-                    *reinterpret_cast<uint4*>(rowp + ((u ^ (t & 7)) << 4)) =
-                        make_uint4(gk[4 * k], gk[4 * k + 1], gk[4 * k + 2], gk[4 * k + 3]);
-                }
-            }
-            tmem_wait_st();
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            mbar_arrive(ds_full);
-            ok = __all_sync(0xffffffffu, mbar_wait(dq_full, j & 1, lim) && !*abort_flag);
-            if (!ok) break;
-            tc_fence_after_sync();
-            // dQᵀ: lane = feature d = 32 quarter + lane, columns = query rows 64 half
-            // .. +63.  All of it out of tensor memory first, so the next step's
-            // MMAs may start; then each reduction instruction adds one query
-            // row's 32 consecutive features: 128 contiguous bytes per warp.
             uint32_t g[64];
-            tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
-            tmem_ld_32x32b_x32(tmem + lanes + C::kColdP + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
+            tmem_ld_32x32b_x32(tmem + lanes + hf * 128 + 64, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+            tmem_ld_32x32b_x32(tmem + lanes + hf * 128 + 96, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
             tmem_wait_ld();
             reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&g[0]));
             reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&g[32]));
             tc_fence_before_sync();
-            mbar_arrive(dq_empty);
-            const int dcol = quarter * 32 + lane;
-            if (dcol < D) {  // warp-uniform: at D = 64 warps of quarters 2, 3 hold no feature
-                float* dst = p.dq_acc + (qrow0 + q0 + half * 64) * D + dcol;
-                const int nq = min(64, p.N - (q0 + half * 64));
+            mbar_arrive(&dq_empty[hf]);
+            if (dcol < D) {  // warp-uniform: at D = 64 quarters 2, 3 hold no feature
+                float* dst = p.dq_acc + (qrow0 + qh) * D + dcol;
+                const int nq = min(64, p.N - qh);
 #pragma unroll
                 for (int i = 0; i < 64; i++)
                     if (i < nq) red_add_f32(dst + int64_t(i) * D, __uint_as_float(g[i]));
             }
         }
         if (!ok && lane == 0) bwd_report(p, abort_flag, ST_BWD_ELEM_WAIT);
+    } else {
+        // ================================================================ element-wise warps 0-7
+        // Warp w serves tensor-memory lanes 32 (w % 4) .. +31 (kv rows of Sᵀ,
+        // dPᵀ, dK, dV) and, in every half, query columns 32 (w / 4) .. +31 of it.
+        // Each warp decides to leave its loop as a whole (every test goes through
+        // a vote); warps never wait on one another except through bounded
+        // mbarrier waits.
+        const int quarter = warp % 4;
+        const int sub = warp / 4;
+        const int t = quarter * 32 + lane;  // kv row of this thread
+        const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
+        const int kv = c * kBwdTile + t;
+        const bool kv_ragged = (c + 1) * kBwdTile > p.N;
+        bool ok = true;
+        for (int k = 0; k < halves; k++) {
+            const int hf = k & 1;
+            const int j = k >> 1;
+            int hq, r;
+            bool full;
+            step_of(j, hq, r, full);
+            const int q0 = r * kBwdTile;
+            const int qc = q0 + hf * 64 + sub * 32;  // first query column of this thread's chunk
+            const int64_t qrow0 = (int64_t(b) * p.Hq + hq) * p.N;
+            // LSE₂ and Δ of query column qc + lane, handed to the other lanes by shuffles
+            const float lse_c = qc + lane < p.N ? __ldg(&p.lse2[qrow0 + qc + lane]) : INFINITY;
+            const float dl_c = qc + lane < p.N ? __ldg(&p.delta[qrow0 + qc + lane]) : 0.f;
+            const bool masked = !full || kv_ragged || q0 + kBwdTile > p.N;
+            const uint32_t allow = masked ? bwd_allow_word(p, qc, kv) : 0xffffffffu;
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[hf], j & 1, lim) && !*abort_flag);
+            if (!ok) break;
+            tc_fence_after_sync();
+            const uint32_t col = hf * 128 + sub * 32;  // this chunk's Sᵀ columns; dPᵀ at +64
+            uint32_t s[32], d[32];
+            tmem_ld_32x32b_x32(tmem + lanes + col, s);
+            tmem_ld_32x32b_x32(tmem + lanes + col + 64, d);
+            tmem_wait_ld();
+            reg_fence(s);
+            reg_fence(d);
+            uint32_t pk[16], gk[16];
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                const float l0 = __shfl_sync(0xffffffffu, lse_c, i);
+                const float l1 = __shfl_sync(0xffffffffu, lse_c, i + 1);
+                const float e0 = __shfl_sync(0xffffffffu, dl_c, i);
+                const float e1 = __shfl_sync(0xffffffffu, dl_c, i + 1);
+                float p0 = ex2_approx(fmaf(__uint_as_float(s[i]), p.scale_log2, -l0));
+                float p1 = ex2_approx(fmaf(__uint_as_float(s[i + 1]), p.scale_log2, -l1));
+                p0 = (allow >> i) & 1u ? p0 : 0.f;
+                p1 = (allow >> (i + 1)) & 1u ? p1 : 0.f;
+                const float g0 = p0 * (__uint_as_float(d[i]) - e0) * p.scale;
+                const float g1 = p1 * (__uint_as_float(d[i + 1]) - e1) * p.scale;
+                pk[i / 2] = pack_bf16x2(p0, p1);
+                gk[i / 2] = pack_bf16x2(g0, g1);
+            }
+            // Pᵀ and dSᵀ (bf16 pairs) over the 32 Sᵀ columns just read by this
+            // thread: Pᵀ in col .. col+15, dSᵀ in col+16 .. col+31
+            tmem_st_32x32b_x16(tmem + lanes + col, pk);
+            tmem_st_32x32b_x16(tmem + lanes + col + 16, gk);
+            // dSᵀ row t, query columns 32 sub .. +31 of the half: panel hf of the shared tile
+            uint8_t* rowp = sdS + hf * C::kPanel + t * 128;
+#pragma unroll
+            for (int k4 = 0; k4 < 4; k4++) {
+                const int u = sub * 4 + k4;
+                *reinterpret_cast<uint4*>(rowp + ((u ^ (t & 7)) << 4)) =
+                    make_uint4(gk[4 * k4], gk[4 * k4 + 1], gk[4 * k4 + 2], gk[4 * k4 + 3]);
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(&ds_full[hf]);
+        }
+        if (!ok && lane == 0) bwd_report(p, abort_flag, ST_BWD_ELEM_WAIT);
         // dK and dV rows of this kv tile, this warp's column half (zeros when no
-        // query attends to it); the tensor-memory loads are warp-collective,
-        // the stores per row
+        // query attends to it), after the last half's MMAs (its dq_full)
+        if (ok && halves > 0) {
+            const int kl = halves - 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&dq_full[kl & 1], (kl >> 1) & 1, lim) && !*abort_flag);
+            if (!ok && lane == 0) bwd_report(p, abort_flag, ST_BWD_ELEM_WAIT);
+            tc_fence_after_sync();
+        }
         if (ok) {
+            constexpr int kHalfD = D / 2;
             const int64_t orow = (int64_t(b) * p.Hkv + hkv) * p.N + kv;
 #pragma unroll 1
             for (int which = 0; which < 2; which++) {
-                uint4* dst = reinterpret_cast<uint4*>((which == 0 ? p.dV : p.dK) + orow * D + half * kHalfD);
-                const uint32_t col = (which == 0 ? C::kColdV : C::kColdK) + half * kHalfD;
+                uint4* dst = reinterpret_cast<uint4*>((which == 0 ? p.dV : p.dK) + orow * D + sub * kHalfD);
+                const uint32_t col = (which == 0 ? C::kColdV : C::kColdK) + sub * kHalfD;
 #pragma unroll 1
-                for (int k = 0; k < kHalfD / 32; k++) {
+                for (int k2 = 0; k2 < kHalfD / 32; k2++) {
                     uint32_t gg[32];
                     if (steps > 0) {
-                        tmem_ld_32x32b_x32(tmem + lanes + col + k * 32, gg);
+                        tmem_ld_32x32b_x32(tmem + lanes + col + k2 * 32, gg);
                         tmem_wait_ld();
                         reg_fence(gg);
                     } else {
@@ -534,7 +573,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     if (kv < p.N) {
 #pragma unroll
                         for (int i = 0; i < 32; i += 8)
-                            dst[(k * 32 + i) / 8] = make_uint4(
+                            dst[(k2 * 32 + i) / 8] = make_uint4(
                                 pack_bf16x2(__uint_as_float(gg[i]), __uint_as_float(gg[i + 1])),
                                 pack_bf16x2(__uint_as_float(gg[i + 2]), __uint_as_float(gg[i + 3])),
                                 pack_bf16x2(__uint_as_float(gg[i + 4]), __uint_as_float(gg[i + 5])),
