@@ -23,6 +23,12 @@ forward's O and LSE computed once before timing; value counts 10 * D useful
 FLOP per allowed pair (S, dP, dV, dK, dQ) and the roofline takes the whole
 step's device time (the launch list in profiles/ gives each kernel's share).
 
+With --path stride (patterns with a stride) one step is the stride-aware
+forward: three grouping copies, the pattern without its stride in token
+order, the remaining stride pairs on tokens grouped by residue, and the merge;
+the roofline then counts the executed tiles of both passes over the whole
+step's device time.
+
 With --impl reference the oracle is the timed program (rank 0 only).
 Multi-GPU (torchrun): every rank runs its own batch of the workload (the
 problems are independent; no collective on the data path); value is the sum
@@ -297,6 +303,15 @@ def run_gpu(args, w):
 
     p, mask_h, pairs, useful, executed, min_bytes = workload_counts(w)
     mask = mask_h.to_device(dev)
+    stride_path = args.path == "stride"
+    if stride_path:
+        if w.stride <= 0:
+            raise SystemExit("--path stride needs a workload with a stride")
+        plan_h = sa.stride_plan(p, w.N, w.block)
+        plan = tuple(m.to_device(dev) for m in plan_h)
+        executed = 4.0 * w.D * w.block * w.block * sum(m.n_live for m in plan_h) * w.B * w.Hq
+        sws = torch.empty(sa.fwd_stride_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.D), dtype=torch.uint8,
+                          device=dev)
 
     # inputs: every rank its own batch (seed offset by rank); rotate sets past L2
     q, k, v = synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=rank_seed(w, rank))
@@ -314,7 +329,11 @@ def run_gpu(args, w):
 
     def step(i):
         Qi, Ki, Vi, Oi, Li = sets[i % n_sets]
-        sa.fwd(Qi, Ki, Vi, mask, p, scale=w.scale, out=Oi, lse=Li, stream=stream)
+        if stride_path:
+            sa.fwd_stride(Qi, Ki, Vi, plan[0], plan[1], p, scale=w.scale, out=Oi, lse=Li, workspace=sws,
+                          stream=stream)
+        else:
+            sa.fwd(Qi, Ki, Vi, mask, p, scale=w.scale, out=Oi, lse=Li, stream=stream)
 
     for i in range(args.warmup):
         step(i)
@@ -346,7 +365,7 @@ def run_gpu(args, w):
 
     # end to end through the host-buffer entry point (pinned memory)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not stride_path:
         pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
         Qh, Kh, Vh = pin(q), pin(k), pin(v)
         Oh = torch.empty((w.B, w.Hq, w.N, w.D), dtype=torch.bfloat16).pin_memory()
@@ -397,14 +416,18 @@ def run_gpu(args, w):
             "l2": f"{n_sets} rotating input sets of {set_bytes / 1e6:.1f} MB "
                   f"({n_sets * set_bytes / 1e6:.0f} MB > {L2_BYTES / 1e6:.0f} MB L2)",
             "live_tiles": int(mask_h.n_live), "full_tiles": int(mask_h.n_full),
-            "allowed_pairs_per_head": int(pairs)}),
+            "allowed_pairs_per_head": int(pairs),
+            **({"path": "stride-aware", "executed_tiles_per_head": int(sum(m.n_live for m in plan_h))}
+               if stride_path else {})}),
         "useful_frac_of_peak": value / world / peak,
         "executed_tflops": job_tflops(world, executed, args.steps, elapsed_ms),
         "executed_frac_of_peak": executed / (elapsed_ms / args.steps * 1e-3) / 1e12 / peak,
         "peak_kind": f"bf16 dense, {peak_kind} ({peak} TFLOP/s burst)",
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(w.name),
-                     "kernel": "fwd_kernel<D,BN>", "mean_launch_us": mean_launch_ms * 1e3,
+                     "frac": achieved / peak, "traffic": None if stride_path else profiled_traffic(w.name),
+                     "kernel": ("stride-aware step: 3 grouping copies + 2 x fwd_kernel + merge" if stride_path
+                                else "fwd_kernel<D,BN>"),
+                     "mean_launch_us": mean_launch_ms * 1e3,
                      "algorithmic_flop_per_launch": executed,
                      "hbm_gbs_min_bytes": min_bytes / (mean_launch_ms * 1e-3) / 1e9},
         "cpu_baseline": cpu,
@@ -595,6 +618,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling runs)")
     ap.add_argument("--sets", type=int, default=0, help="rotating input sets (0: enough to exceed L2)")
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"])
+    ap.add_argument("--path", default="plain", choices=["plain", "stride"],
+                    help="forward path: one block-sparse kernel, or the stride-aware two-pass path")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

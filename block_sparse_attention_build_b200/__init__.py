@@ -42,6 +42,7 @@ EXPORTED = (
     "sparse_attn_check_device", "sparse_attn_set_debug", "sparse_attn_status_string",
     "sparse_attn_version", "sparse_attn_fwd_noalloc", "sparse_attn_fwd_heads",
     "sparse_attn_transpose_block_mask", "sparse_attn_bwd_workspace", "sparse_attn_bwd",
+    "sparse_attn_stride_plan", "sparse_attn_fwd_stride_workspace", "sparse_attn_fwd_stride",
 )
 
 
@@ -89,6 +90,9 @@ def _load() -> ctypes.CDLL:
     L.sparse_attn_bwd_workspace.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
     L.sparse_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp, vp,
                                   ctypes.c_size_t, vp]
+    L.sparse_attn_stride_plan.argtypes = [P, ctypes.c_int64, ctypes.c_int32, M, M]
+    L.sparse_attn_fwd_stride_workspace.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
+    L.sparse_attn_fwd_stride.argtypes = [vp, vp, vp, M, M, P, S, ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp]
     L.sparse_attn_check_device.argtypes = [vp]
     L.sparse_attn_set_debug.argtypes = [ctypes.c_int32, ctypes.c_int64]
     L.sparse_attn_status_string.argtypes = [ctypes.c_int]
@@ -98,7 +102,8 @@ def _load() -> ctypes.CDLL:
     for name in ("sparse_attn_build_block_mask", "sparse_attn_count_pairs", "sparse_attn_fwd",
                  "sparse_attn_fwd_host", "sparse_attn_fwd_host_workspace", "sparse_attn_check_device",
                  "sparse_attn_set_debug", "sparse_attn_fwd_noalloc", "sparse_attn_fwd_heads",
-                 "sparse_attn_transpose_block_mask", "sparse_attn_bwd_workspace", "sparse_attn_bwd"):
+                 "sparse_attn_transpose_block_mask", "sparse_attn_bwd_workspace", "sparse_attn_bwd",
+                 "sparse_attn_stride_plan", "sparse_attn_fwd_stride_workspace", "sparse_attn_fwd_stride"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -196,6 +201,24 @@ def transpose_block_mask(mask: BlockMask) -> BlockMask:
     _check(lib.sparse_attn_transpose_block_mask(ctypes.byref(src), ctypes.byref(out)),
            "sparse_attn_transpose_block_mask")
     return BlockMask(counts, index, full, out.block, out.n_live, out.n_full, out.max_per_row, mask.N)
+
+
+def stride_plan(pattern: Pattern, N: int, block: int = 128):
+    """(pass1, pass2) host block masks of the stride-aware path (see
+    ``fwd_stride``): the pattern without its stride in token order, and the
+    remaining stride pairs on tokens grouped by residue."""
+    T = max(num_tiles(N, block), 0)
+    arrays = []
+    cms = []
+    for _ in range(2):
+        a = (np.zeros(T, dtype=np.int32), np.zeros((T, T), dtype=np.int32), np.zeros((T, T), dtype=np.uint8))
+        arrays.append(a)
+        cms.append(_BlockMask(T, T, 0, 0, 0, 0, a[0].ctypes.data if T else None, a[1].ctypes.data if T else None,
+                              a[2].ctypes.data if T else None))
+    _check(lib.sparse_attn_stride_plan(ctypes.byref(pattern._c()), N, block, ctypes.byref(cms[0]),
+                                       ctypes.byref(cms[1])), "sparse_attn_stride_plan")
+    return tuple(BlockMask(a[0], a[1], a[2], m.block, m.n_live, m.n_full, m.max_per_row, N)
+                 for a, m in zip(arrays, cms))
 
 
 def count_pairs(pattern: Pattern, N: int) -> int:
@@ -314,6 +337,41 @@ def bwd(q, k, v, o, lse, do, mask_t: BlockMask, pattern: Pattern, scale: float |
                                    ctypes.byref(shape), float(scale), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                                    workspace.data_ptr(), workspace.numel(), st), "sparse_attn_bwd")
     return dq, dk, dv
+
+
+def fwd_stride_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, D: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.sparse_attn_fwd_stride_workspace(ctypes.byref(_Shape(B, Hq, Hkv, N, D)), ctypes.byref(n)),
+           "sparse_attn_fwd_stride_workspace")
+    return n.value
+
+
+def fwd_stride(q, k, v, pass1: BlockMask, pass2: BlockMask, pattern: Pattern, scale: float | None = None,
+               out=None, lse=None, workspace=None, stream=None):
+    """Forward pass of a strided pattern by the stride-aware path (``stride_plan``'s
+    masks on q's device); same results as ``fwd`` with the whole pattern."""
+    import torch
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError("q, k, v must be contiguous bf16 CUDA tensors")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    shape = _Shape(B, Hq, Hkv, N, D)
+    n = ctypes.c_size_t(0)
+    _check(lib.sparse_attn_fwd_stride_workspace(ctypes.byref(shape), ctypes.byref(n)), "sparse_attn_fwd_stride_workspace")
+    if workspace is None:
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        st = _stream_handle(stream, q.device)
+        _check(lib.sparse_attn_fwd_stride(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(pass1._c()),
+                                          ctypes.byref(pass2._c()), ctypes.byref(pattern._c()), ctypes.byref(shape),
+                                          float(scale), out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                                          workspace.numel(), st), "sparse_attn_fwd_stride")
+    return out, lse
 
 
 def fwd_host_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, D: int) -> int:

@@ -10,7 +10,7 @@ CSRC = os.path.join(PKG, "csrc")
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libsparse_attn.so")
 SOURCES = ["capi.cu", "block_mask.cpp", "fwd_noalloc.cu", "bwd.cu"]
-HEADERS = ["sm100.cuh", "fwd_sm100.cuh", "bwd_sm100.cuh", "tma_host.h", "runtime.h"]
+HEADERS = ["sm100.cuh", "fwd_sm100.cuh", "bwd_sm100.cuh", "stride_sm100.cuh", "tma_host.h", "runtime.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]

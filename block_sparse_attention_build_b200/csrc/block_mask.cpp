@@ -16,6 +16,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <vector>
 
 #include "../../include/sparse_attn.h"
 
@@ -320,5 +321,68 @@ extern "C" int sparse_attn_transpose_block_mask(const sa_block_mask* rows, sa_bl
     cols->max_per_row = max_col;
     cols->n_live = live;
     cols->n_full = nfull;
+    return SA_OK;
+}
+
+extern "C" int sparse_attn_stride_plan(const sa_pattern* pattern, int64_t N, int32_t block, sa_block_mask* pass1,
+                                       sa_block_mask* pass2)
+{
+    if (!pattern || !pass1 || !pass2 || N < 0) return SA_ERR_INVALID_ARG;
+    if (int rc = sa::pattern_status(pattern)) return rc;
+    const sa_pattern pt = *pattern;
+    if (pt.causal != 1 || pt.stride <= 0 || pt.area != 0) return SA_ERR_UNSUPPORTED;
+    if (N % pt.stride != 0) return SA_ERR_UNSUPPORTED;
+    // pass 1: the pattern without its stride, token order
+    sa_pattern p1 = pt;
+    p1.stride = 0;
+    if (int rc = sparse_attn_build_block_mask(&p1, N, block, pass1)) return rc;
+    // pass 2: grouped order P = (t mod s) * n + t / s; row P of group g allows
+    // [g n + ceil((C - g) / s), P - shift]: the stride pairs outside the band
+    // (q - kv > window), the sink/global columns (kv >= C) and the global rows
+    const int32_t T = pass1->n_q_tiles;
+    if (pass2->n_q_tiles < T || pass2->n_kv_tiles < T) return SA_ERR_BUFFER_TOO_SMALL;
+    if (T > 0 && (!pass2->kv_count || !pass2->kv_index || !pass2->kv_full)) return SA_ERR_INVALID_ARG;
+    const int64_t s = pt.stride, n = N / s;
+    const int64_t C = std::max(pt.sinks, pt.n_global);
+    const int64_t shift = pt.window >= 0 ? std::min<int64_t>(pt.window, N) / s + 1 : 0;
+    std::vector<int64_t> cnt(static_cast<size_t>(T > 0 ? T : 1));
+    int32_t max_row = 0;
+    int64_t live = 0, nfull = 0;
+    for (int32_t i = 0; i < T; i++) {
+        std::fill(cnt.begin(), cnt.end(), 0);
+        const int64_t q0 = int64_t(i) * block, q1 = std::min<int64_t>(N, q0 + block) - 1;
+        for (int64_t P = q0; P <= q1; P++) {
+            const int64_t g = P / n;
+            const int64_t lo = g * n + (C > g ? (C - g + s - 1) / s : 0);
+            const int64_t hi = P - shift;
+            if (lo > hi) continue;
+            for (int64_t c = lo / block; c <= hi / block; c++)
+                cnt[c] += std::min<int64_t>(hi, c * block + block - 1) - std::max<int64_t>(lo, c * block) + 1;
+        }
+        int32_t* idx = pass2->kv_index + int64_t(i) * T;
+        uint8_t* full = pass2->kv_full + int64_t(i) * T;
+        int32_t k = 0;
+        for (int32_t c = 0; c < T; c++) {
+            if (cnt[c] == 0) continue;
+            const int64_t k0 = int64_t(c) * block, k1 = std::min<int64_t>(N, k0 + block) - 1;
+            idx[k] = c;
+            full[k] = cnt[c] == (q1 - q0 + 1) * (k1 - k0 + 1) ? 1 : 0;
+            nfull += full[k];
+            k++;
+        }
+        for (int32_t e = k; e < T; e++) {
+            idx[e] = -1;
+            full[e] = 0;
+        }
+        pass2->kv_count[i] = k;
+        live += k;
+        max_row = std::max(max_row, k);
+    }
+    pass2->n_q_tiles = T;
+    pass2->n_kv_tiles = T;
+    pass2->block = block;
+    pass2->max_per_row = max_row;
+    pass2->n_live = live;
+    pass2->n_full = nfull;
     return SA_OK;
 }

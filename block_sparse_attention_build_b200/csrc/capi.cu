@@ -9,6 +9,7 @@
 #include "../../include/sparse_attn.h"
 #include "fwd_sm100.cuh"
 #include "runtime.h"
+#include "stride_sm100.cuh"
 #include "tma_host.h"
 
 namespace sa {
@@ -107,16 +108,26 @@ bool general_form(const sa_pattern& pt) { return pt.causal == 0 || pt.area > 0; 
 // kernels' q - kv +- window and stripe bounds stay inside int32.
 int32_t clip_to(int32_t v, int32_t N) { return v > N ? N : v; }
 
+// Pass 2 of the stride-aware path: the residual stride pairs in the grouped
+// order (PatternRef mode 1).
+struct ResidualStride {
+    int32_t n;       // group length N / stride
+    int32_t shift;   // floor(window / stride) + 1 (0 without a band)
+    int32_t col_lo;  // max(sinks, n_global)
+    int32_t stride;
+};
+
 // The forward pass behind sparse_attn_fwd (one pattern: n_patterns = 1,
-// head_pattern = null) and sparse_attn_fwd_heads (a pattern per query head).
+// head_pattern = null), sparse_attn_fwd_heads (a pattern per query head) and
+// pass 2 of sparse_attn_fwd_stride (rs non-null).
 int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* masks, const sa_pattern* patterns,
              int32_t n_patterns, const int32_t* head_pattern, const sa_shape* shape, float scale, void* O, float* LSE,
-             void* stream)
+             void* stream, const ResidualStride* rs = nullptr)
 {
     if (!masks || !patterns || !shape) return SA_ERR_INVALID_ARG;
     const bool per_head = head_pattern != nullptr;
     if (n_patterns < 1 || n_patterns > (per_head ? kMaxPatterns : 1)) return SA_ERR_INVALID_ARG;
-    bool multi = per_head;  // general forms also take the pattern-table kernel
+    bool multi = per_head || rs != nullptr;  // general forms also take the pattern-table kernel
     for (int i = 0; i < n_patterns; i++) multi = multi || general_form(patterns[i]);
     const sa_block_mask* mask = &masks[0];
     const sa_pattern* pattern = &patterns[0];
@@ -216,6 +227,14 @@ int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* m
         hp.pat[i].causal = patterns[i].causal;
         hp.pat[i].area = clip_to(patterns[i].area, s.N);
         hp.pat[i].summary = patterns[i].summary < patterns[i].area ? patterns[i].summary : patterns[i].area;
+        hp.pat[i].mode = 0;
+    }
+    if (rs) {
+        hp.pat[0].mode = 1;
+        hp.pat[0].area = rs->n;
+        hp.pat[0].shift = rs->shift;
+        hp.pat[0].col_lo = rs->col_lo;
+        hp.pat[0].stride = rs->stride;
     }
     for (int h = 0; h < s.Hq; h++) hp.head[h] = per_head ? static_cast<uint8_t>(head_pattern[h]) : 0;
     return launch_any<true>(s.D, mask->block, mq, mk, mv, mo, p, hp, g, st);
@@ -248,6 +267,112 @@ extern "C" int sparse_attn_fwd_heads(const void* Q, const void* K, const void* V
 {
     if (!head_pattern) return SA_ERR_INVALID_ARG;
     return sa::fwd_impl(Q, K, V, masks, patterns, n_patterns, head_pattern, shape, scale, O, LSE, stream);
+}
+
+namespace sa {
+namespace {
+
+struct StrideLayout {
+    size_t q, k, v, o2, l1, l2, total;  // byte offsets, each 256-aligned
+};
+
+StrideLayout stride_layout(const sa_shape& s)
+{
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t qb = size_t(s.B) * s.Hq * s.N * s.D * 2, kvb = size_t(s.B) * s.Hkv * s.N * s.D * 2;
+    const size_t lb = size_t(s.B) * s.Hq * s.N * 4;
+    StrideLayout w;
+    w.q = 0;
+    w.k = w.q + up(qb);
+    w.v = w.k + up(kvb);
+    w.o2 = w.v + up(kvb);
+    w.l1 = w.o2 + up(qb);
+    w.l2 = w.l1 + up(lb);
+    w.total = w.l2 + up(lb);
+    return w;
+}
+
+unsigned grid_for(int64_t items)
+{
+    const int n_sm = sm_count();
+    int64_t g = (items + 255) / 256;
+    const int64_t cap = int64_t(n_sm > 0 ? n_sm : 148) * 16;
+    return static_cast<unsigned>(g < cap ? (g > 0 ? g : 1) : cap);
+}
+
+template <int D>
+int stride_run(const void* Q, const void* K, const void* V, const sa_block_mask* pass1, const sa_block_mask* pass2,
+               const sa_pattern& pt, const sa_shape& s, float scale, void* O, float* LSE, uint8_t* ws,
+               cudaStream_t st)
+{
+    const StrideLayout L = stride_layout(s);
+    const int n = s.N / pt.stride;
+    constexpr int U = D * 2 / 16;
+    const int64_t qp = int64_t(s.B) * s.Hq, kp = int64_t(s.B) * s.Hkv;
+    group_by_residue_kernel<D><<<grid_for(qp * s.N * U), 256, 0, st>>>(
+        static_cast<const uint4*>(Q), reinterpret_cast<uint4*>(ws + L.q), qp, s.N, pt.stride, n);
+    group_by_residue_kernel<D><<<grid_for(kp * s.N * U), 256, 0, st>>>(
+        static_cast<const uint4*>(K), reinterpret_cast<uint4*>(ws + L.k), kp, s.N, pt.stride, n);
+    group_by_residue_kernel<D><<<grid_for(kp * s.N * U), 256, 0, st>>>(
+        static_cast<const uint4*>(V), reinterpret_cast<uint4*>(ws + L.v), kp, s.N, pt.stride, n);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+    // pass 1: the pattern without its stride, token order; O holds O1, L1 in the workspace
+    sa_pattern p1 = pt;
+    p1.stride = 0;
+    float* l1 = reinterpret_cast<float*>(ws + L.l1);
+    if (int rc = fwd_impl(Q, K, V, pass1, &p1, 1, nullptr, &s, scale, O, l1, st)) return rc;
+    // pass 2: the residual stride pairs, grouped order
+    ResidualStride rs;
+    rs.n = n;
+    rs.shift = pt.window >= 0 ? (pt.window > s.N ? s.N : pt.window) / pt.stride + 1 : 0;
+    rs.col_lo = pt.sinks > pt.n_global ? pt.sinks : pt.n_global;
+    rs.stride = pt.stride;
+    float* l2 = reinterpret_cast<float*>(ws + L.l2);
+    if (int rc = fwd_impl(ws + L.q, ws + L.k, ws + L.v, pass2, &pt, 1, nullptr, &s, scale, ws + L.o2, l2, st, &rs))
+        return rc;
+    merge_passes_kernel<D><<<grid_for(qp * s.N * U), 256, 0, st>>>(
+        static_cast<__nv_bfloat16*>(O), LSE, reinterpret_cast<const __nv_bfloat16*>(ws + L.o2), l1, l2, qp, s.N,
+        pt.stride, n);
+    return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace sa
+
+extern "C" int sparse_attn_fwd_stride_workspace(const sa_shape* shape, size_t* bytes)
+{
+    if (!shape || !bytes) return SA_ERR_INVALID_ARG;
+    const sa_shape s = *shape;
+    if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
+    *bytes = sa::stride_layout(s).total;
+    return SA_OK;
+}
+
+extern "C" int sparse_attn_fwd_stride(const void* Q, const void* K, const void* V, const sa_block_mask* pass1,
+                                      const sa_block_mask* pass2, const sa_pattern* pattern, const sa_shape* shape,
+                                      float scale, void* O, float* LSE, void* workspace, size_t workspace_bytes,
+                                      void* stream)
+{
+    if (!pass1 || !pass2 || !pattern || !shape) return SA_ERR_INVALID_ARG;
+    const sa_pattern pt = *pattern;
+    const sa_shape s = *shape;
+    if (int rc = sa::pattern_status(pt)) return rc;
+    if (pt.causal != 1 || pt.stride <= 0 || pt.area != 0) return SA_ERR_UNSUPPORTED;
+    if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
+    if (s.D != 64 && s.D != 128) return SA_ERR_UNSUPPORTED;
+    if (s.B == 0 || s.Hq == 0 || s.N == 0) return SA_OK;
+    if (s.N % pt.stride != 0) return SA_ERR_UNSUPPORTED;  // groups of equal length
+    if (pass1->block != pass2->block) return SA_ERR_MASK_MISMATCH;
+    if (!workspace || !Q || !K || !V || !O || !LSE) return SA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SA_ERR_MISALIGNED;
+    if (!sa::aligned16(Q) || !sa::aligned16(K) || !sa::aligned16(V) || !sa::aligned16(O) || !sa::aligned16(LSE))
+        return SA_ERR_MISALIGNED;
+    if (workspace_bytes < sa::stride_layout(s).total) return SA_ERR_BUFFER_TOO_SMALL;
+    // the passes check shapes and masks themselves before launching
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (s.D == 128) return sa::stride_run<128>(Q, K, V, pass1, pass2, pt, s, scale, O, LSE, ws, st);
+    return sa::stride_run<64>(Q, K, V, pass1, pass2, pt, s, scale, O, LSE, ws, st);
 }
 
 extern "C" int sparse_attn_fwd_host_workspace(const sa_shape* shape, size_t* bytes)

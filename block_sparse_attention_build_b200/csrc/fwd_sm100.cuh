@@ -108,6 +108,12 @@ struct PatternRef {
     const int32_t* kv_index;  // [T * T]
     const uint8_t* kv_full;   // [T * T]
     int32_t window, sinks, stride, n_global, causal, area, summary;  // summary <= area
+    // mode 1: the residual stride pass of the stride-aware path, on tokens
+    // grouped by residue (position P = (t mod stride) * area + t / stride): row P
+    // of group g = P / area allows the one interval [g * area + ceil((col_lo - g) /
+    // stride), P - shift] (stride pairs not already in the band, the sink or
+    // global columns or a global row)
+    int32_t mode, shift, col_lo;
 };
 struct HeadPatterns {
     PatternRef pat[kMaxPatterns];
@@ -927,19 +933,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int64_t orow = (static_cast<int64_t>(w.b) * p.Hq + (x == 0 ? w.hq[0] : w.hq[1])) * p.N + q;
             if constexpr (MULTI) {
                 const PatternRef& pr = hp.pat[hp.head[x == 0 ? w.hq[0] : w.hq[1]]];
-                pw = pr.window;
-                ps = pr.stride;
-                pg = pr.n_global;
-                cols = max(pr.sinks, pr.n_global);
-                qlim = pr.causal ? q : p.N - 1;
-                s_area = pr.area;
-                s_cnt = pr.summary;
-                if (pr.area > 0) {
-                    a_lo = (q / pr.area) * pr.area;
-                    a_hi = a_lo + pr.area - 1;
+                if (pr.mode == 1) {
+                    const int grp = q / pr.area;
+                    const int need = pr.col_lo - grp;
+                    a_lo = grp * pr.area + (need > 0 ? (need + pr.stride - 1) / pr.stride : 0);
+                    a_hi = q - pr.shift;
+                    pw = -1;
+                    ps = 0;
+                    pg = 0;
+                    cols = 0;
+                    s_cnt = 0;
+                    qlim = p.N - 1;
                 } else {
-                    a_lo = 0;
-                    a_hi = -1;
+                    pw = pr.window;
+                    ps = pr.stride;
+                    pg = pr.n_global;
+                    cols = max(pr.sinks, pr.n_global);
+                    qlim = pr.causal ? q : p.N - 1;
+                    s_area = pr.area;
+                    s_cnt = pr.summary;
+                    if (pr.area > 0) {
+                        a_lo = (q / pr.area) * pr.area;
+                        a_hi = a_lo + pr.area - 1;
+                    } else {
+                        a_lo = 0;
+                        a_hi = -1;
+                    }
                 }
             }
             const bool row_all = q < pg;

@@ -285,6 +285,42 @@ int sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O, 
                     const sa_block_mask* mask_t, const sa_pattern* pattern, const sa_shape* shape, float scale,
                     void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Stride-aware path for causal patterns with a stride s (every s-th prior
+ * token): in token order those pairs touch every tile below the diagonal once
+ * per row.  The plan splits the pattern into
+ *   pass 1  the pattern without its stride, in token order, and
+ *   pass 2  the stride pairs that pass 1 does not admit, on tokens grouped by
+ *           residue (position P = (t mod s) * n + floor(t / s), n = N / s),
+ *           where they form dense tiles along the diagonal,
+ * and sparse_attn_fwd_stride merges the two partial softmaxes exactly.  Needs
+ * causal == 1, stride > 0, area == 0, and N a multiple of the stride (else
+ * SA_ERR_UNSUPPORTED).  Host-only; pass1 and pass2 hold caller-owned host
+ * arrays of capacity T x T each (T = ceil(N / block)), as for
+ * sparse_attn_build_block_mask.
+ */
+int sparse_attn_stride_plan(const sa_pattern* pattern, int64_t N, int32_t block, sa_block_mask* pass1,
+                            sa_block_mask* pass2);
+
+/* Device workspace bytes that sparse_attn_fwd_stride needs: grouped copies of
+ * Q, K, V, pass 2's O (bf16), and both passes' LSE (fp32), each rounded up to
+ * 256 bytes. */
+int sparse_attn_fwd_stride_workspace(const sa_shape* shape, size_t* bytes);
+
+/*
+ * The forward pass by the stride-aware path: results as sparse_attn_fwd with
+ * `pattern` (O, LSE of the whole pattern).  pass1 and pass2 are the plan's
+ * masks with their arrays in DEVICE memory; workspace is device memory of at
+ * least sparse_attn_fwd_stride_workspace bytes, 256-byte aligned.  Launches
+ * three grouping copies, the two passes and the merge on `stream`; returns
+ * without waiting.  Errors as sparse_attn_fwd, plus SA_ERR_UNSUPPORTED for a
+ * pattern the plan does not take and SA_ERR_BUFFER_TOO_SMALL for a short
+ * workspace.
+ */
+int sparse_attn_fwd_stride(const void* Q, const void* K, const void* V, const sa_block_mask* pass1,
+                           const sa_block_mask* pass2, const sa_pattern* pattern, const sa_shape* shape, float scale,
+                           void* O, float* LSE, void* workspace, size_t workspace_bytes, void* stream);
+
 const char* sparse_attn_status_string(int status);
 
 /* ABI version: major * 10000 + minor * 100 + patch. */

@@ -290,3 +290,61 @@ def test_fixed_pattern_pair_count_closed_form():
     for N, A, c in [(1024, 128, 16), (1000, 100, 10), (333, 64, 1)]:
         assert sa.count_pairs(sa.Pattern(window=-1, area=A, summary=c), N) == sum(
             q % A + 1 + (q // A) * c for q in range(N))
+
+
+STRIDE_PLANS = [
+    (sa.Pattern(window=8, stride=8, n_global=2), 128, 64),      # the strided-global shape, scaled down
+    (sa.Pattern(window=5, stride=4, sinks=3), 192, 64),
+    (sa.Pattern(window=-1, stride=6), 192, 64),                 # stride only
+    (sa.Pattern(window=13, stride=4, n_global=9), 256, 64),     # global wider than the stride
+    (sa.Pattern(window=2, stride=16, sinks=1), 256, 64),        # groups of 16 inside a tile
+    (sa.Pattern(window=128, stride=128, n_global=16), 1024, 64),  # groups of 8 tokens
+    (sa.Pattern(window=40, stride=2, sinks=4), 256, 128),       # groups of 128: one tile each
+]
+
+
+@pytest.mark.parametrize("p,N,b", STRIDE_PLANS)
+def test_stride_plan_matches_brute_force(p, N, b):
+    pass1, pass2 = sa.stride_plan(p, N, b)
+    p1 = sa.Pattern(window=p.window, sinks=p.sinks, n_global=p.n_global)
+    c, i, f = oracle.block_mask(opattern(p1), N, b)
+    assert np.array_equal(pass1.counts, c) and np.array_equal(pass1.index, i) and np.array_equal(pass1.full, f)
+    # pass 2 must hold exactly the pairs of the whole pattern that pass 1 lacks, in the grouped order
+    s, n = p.stride, N // p.stride
+    pos = lambda t: (t % s) * n + t // s
+    full_p, base_p = opattern(p), opattern(p1)
+    grid = np.zeros((N, N), dtype=bool)
+    for q in range(N):
+        for kv in range(q + 1):
+            if oracle.allowed(full_p, q, kv) and not oracle.allowed(base_p, q, kv):
+                grid[pos(q), pos(kv)] = True
+    T = -(-N // b)
+    for ti in range(T):
+        rows = grid[ti * b:(ti + 1) * b]
+        js = [tj for tj in range(T) if rows[:, tj * b:(tj + 1) * b].any()]
+        assert pass2.counts[ti] == len(js)
+        assert list(pass2.index[ti, :len(js)]) == js and all(pass2.index[ti, len(js):] == -1)
+        fl = [int(rows[:, tj * b:(tj + 1) * b].all()) for tj in js]
+        assert list(pass2.full[ti, :len(js)]) == fl
+    assert grid.sum() + oracle.count_pairs(base_p, N) == oracle.count_pairs(full_p, N)
+
+
+def test_stride_plan_errors():
+    for p, N, rc in [(sa.Pattern(window=4), 64, sa.SA_ERR_UNSUPPORTED),                 # no stride
+                     (sa.Pattern(window=4, stride=6), 64, sa.SA_ERR_UNSUPPORTED),       # N not a multiple
+                     (sa.Pattern(window=4, stride=4, causal=0), 64, sa.SA_ERR_UNSUPPORTED)]:
+        with pytest.raises(sa.SparseAttnError) as e:
+            sa.stride_plan(p, N, 64)
+        assert e.value.status == rc
+    m = sa._BlockMask(1, 1, 128, 1, 1, 0, 16, 16, 16)
+    fake = 1 << 20
+    shape = sa._Shape(1, 2, 2, 96, 128)
+    good = sa.Pattern(window=8, stride=8)._c()
+    call = lambda pat, ws=fake, nbytes=1 << 30, ptr=fake: sa.lib.sparse_attn_fwd_stride(
+        ptr, ptr, ptr, ctypes.byref(m), ctypes.byref(m), ctypes.byref(pat), ctypes.byref(shape), 0.1, ptr, ptr, ws,
+        nbytes, None)
+    assert call(sa.Pattern(window=8)._c()) == sa.SA_ERR_UNSUPPORTED
+    assert call(sa.Pattern(window=8, stride=7)._c()) == sa.SA_ERR_UNSUPPORTED  # 96 % 7
+    assert call(good, ws=fake + 16) == sa.SA_ERR_MISALIGNED
+    assert call(good, nbytes=100) == sa.SA_ERR_BUFFER_TOO_SMALL
+    assert call(good, ptr=fake + 8) == sa.SA_ERR_MISALIGNED
