@@ -43,6 +43,7 @@ EXPORTED = (
     "sparse_attn_version", "sparse_attn_fwd_noalloc", "sparse_attn_fwd_heads",
     "sparse_attn_transpose_block_mask", "sparse_attn_bwd_workspace", "sparse_attn_bwd",
     "sparse_attn_stride_plan", "sparse_attn_fwd_stride_workspace", "sparse_attn_fwd_stride",
+    "sparse_attn_bwd_heads",
 )
 
 
@@ -93,6 +94,8 @@ def _load() -> ctypes.CDLL:
     L.sparse_attn_stride_plan.argtypes = [P, ctypes.c_int64, ctypes.c_int32, M, M]
     L.sparse_attn_fwd_stride_workspace.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
     L.sparse_attn_fwd_stride.argtypes = [vp, vp, vp, M, M, P, S, ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp]
+    L.sparse_attn_bwd_heads.argtypes = [vp, vp, vp, vp, vp, vp, M, P, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32),
+                                        S, ctypes.c_float, vp, vp, vp, vp, ctypes.c_size_t, vp]
     L.sparse_attn_check_device.argtypes = [vp]
     L.sparse_attn_set_debug.argtypes = [ctypes.c_int32, ctypes.c_int64]
     L.sparse_attn_status_string.argtypes = [ctypes.c_int]
@@ -103,7 +106,8 @@ def _load() -> ctypes.CDLL:
                  "sparse_attn_fwd_host", "sparse_attn_fwd_host_workspace", "sparse_attn_check_device",
                  "sparse_attn_set_debug", "sparse_attn_fwd_noalloc", "sparse_attn_fwd_heads",
                  "sparse_attn_transpose_block_mask", "sparse_attn_bwd_workspace", "sparse_attn_bwd",
-                 "sparse_attn_stride_plan", "sparse_attn_fwd_stride_workspace", "sparse_attn_fwd_stride"):
+                 "sparse_attn_stride_plan", "sparse_attn_fwd_stride_workspace", "sparse_attn_fwd_stride",
+                 "sparse_attn_bwd_heads"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -372,6 +376,40 @@ def fwd_stride(q, k, v, pass1: BlockMask, pass2: BlockMask, pattern: Pattern, sc
                                           float(scale), out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
                                           workspace.numel(), st), "sparse_attn_fwd_stride")
     return out, lse
+
+
+def bwd_heads(q, k, v, o, lse, do, masks_t, patterns, head_pattern, scale: float | None = None,
+              dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients with a pattern per query head: head h under ``patterns[head_pattern[h]]``
+    with the transposed device mask ``masks_t[head_pattern[h]]``.  Otherwise as ``bwd``."""
+    import torch
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    for t in (q, k, v, o, do):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError("q, k, v, o, do must be contiguous bf16 CUDA tensors")
+    if len(masks_t) != len(patterns):
+        raise ValueError("one transposed block mask per pattern")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_bytes(B, Hq, Hkv, N, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    n = len(patterns)
+    cmasks = (_BlockMask * max(n, 1))(*[m._c() for m in masks_t])
+    cpats = (_Pattern * max(n, 1))(*[p_._c() for p_ in patterns])
+    heads = (ctypes.c_int32 * max(len(head_pattern), 1))(*[int(h) for h in head_pattern])
+    shape = _Shape(B, Hq, Hkv, N, D)
+    with torch.cuda.device(q.device):
+        st = _stream_handle(stream, q.device)
+        _check(lib.sparse_attn_bwd_heads(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                         do.data_ptr(), cmasks, cpats, n, heads, ctypes.byref(shape), float(scale),
+                                         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                                         workspace.numel(), st), "sparse_attn_bwd_heads")
+    return dq, dk, dv
 
 
 def fwd_host_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, D: int) -> int:

@@ -1,5 +1,6 @@
-// C ABI of the backward pass: argument checks, the workspace layout, TMA
-// descriptors and the three launches (prep, main, dQ conversion).
+// C ABI of the backward pass (one pattern, or a pattern per query head):
+// argument checks, the workspace layout, the pattern table, TMA descriptors
+// and the three launches (prep, main, dQ conversion).
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -35,8 +36,8 @@ bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <int D>
 int bwd_run(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
-            const sa_block_mask& mt, const sa_pattern& pt, const sa_shape& s, float scale, void* dQ, void* dK,
-            void* dV, uint8_t* ws, cudaStream_t st)
+            const BwdHeads& hb, int32_t T, const sa_shape& s, float scale, void* dQ, void* dK, void* dV, uint8_t* ws,
+            cudaStream_t st)
 {
     int32_t* status = nullptr;
     if (int rc = device_status_word(&status)) return rc;
@@ -58,9 +59,6 @@ int bwd_run(const void* Q, const void* K, const void* V, const void* O, const fl
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
 
     BwdParams p;
-    p.t_count = mt.kv_count;
-    p.t_index = mt.kv_index;
-    p.t_full = mt.kv_full;
     p.lse2 = lse2;
     p.delta = delta;
     p.dq_acc = dq_acc;
@@ -68,19 +66,12 @@ int bwd_run(const void* Q, const void* K, const void* V, const void* O, const fl
     p.dV = static_cast<__nv_bfloat16*>(dV);
     p.status = status;
     p.timeout = wait_limit_cycles();
-    p.T = mt.n_q_tiles;
+    p.T = T;
     p.N = s.N;
     p.B = s.B;
     p.Hq = s.Hq;
     p.Hkv = s.Hkv;
     p.group = s.Hq / s.Hkv;
-    p.window = pt.window > s.N ? s.N : pt.window;  // same allowed set, no int32 overflow in the kernel
-    p.sinks = pt.sinks;
-    p.stride = pt.stride;
-    p.n_global = pt.n_global;
-    p.causal = pt.causal;
-    p.area = pt.area > s.N ? s.N : pt.area;
-    p.summary = pt.summary < pt.area ? pt.summary : pt.area;
     p.scale_log2 = scale * 1.44269504088896340736f;
     p.scale = scale;
 
@@ -95,7 +86,7 @@ int bwd_run(const void* Q, const void* K, const void* V, const void* O, const fl
         attr_set[dev] = true;
     }
     const unsigned grid = static_cast<unsigned>(int64_t(s.B) * s.Hkv * p.T);
-    bwd_kernel<D><<<grid, kBwdThreads, C::kSmemBytes, st>>>(mq, mdo, mk, mv, p);
+    bwd_kernel<D><<<grid, kBwdThreads, C::kSmemBytes, st>>>(mq, mdo, mk, mv, p, hb);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
 
     const int64_t n8 = rows * D / 8;
@@ -104,6 +95,75 @@ int bwd_run(const void* Q, const void* K, const void* V, const void* O, const fl
     if (n_sm > 0 && g > int64_t(n_sm) * 8) g = int64_t(n_sm) * 8;
     bwd_dq_kernel<<<static_cast<unsigned>(g), 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), n8);
     return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+int pattern_check(const sa_pattern& pt)
+{
+    if (pt.window < -1 || pt.sinks < 0 || pt.stride < 0 || pt.n_global < 0 || pt.area < 0 || pt.summary < 0)
+        return SA_ERR_INVALID_ARG;
+    if (pt.summary > 0 && pt.area == 0) return SA_ERR_INVALID_ARG;
+    if (pt.causal != 0 && pt.causal != 1) return SA_ERR_UNSUPPORTED;
+    if (pt.stride > 0 && (pt.causal == 0 || pt.area > 0)) return SA_ERR_UNSUPPORTED;
+    return SA_OK;
+}
+
+// The backward pass behind sparse_attn_bwd (one pattern, head_pattern null)
+// and sparse_attn_bwd_heads (a pattern per query head).
+int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
+             const sa_block_mask* masks_t, const sa_pattern* patterns, int32_t n_patterns, const int32_t* head_pattern,
+             const sa_shape* shape, float scale, void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes,
+             void* stream)
+{
+    if (!masks_t || !patterns || !shape) return SA_ERR_INVALID_ARG;
+    const bool per_head = head_pattern != nullptr;
+    if (n_patterns < 1 || n_patterns > (per_head ? kBwdMaxPatterns : 1)) return SA_ERR_INVALID_ARG;
+    const sa_shape s = *shape;
+    if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
+    for (int i = 0; i < n_patterns; i++)
+        if (int rc = pattern_check(patterns[i])) return rc;
+    if (s.D != 64 && s.D != 128) return SA_ERR_UNSUPPORTED;
+    for (int i = 0; i < n_patterns; i++)
+        if (masks_t[i].block != kBwdTile) return SA_ERR_UNSUPPORTED;
+    if (s.Hq > kBwdMaxHeads) return SA_ERR_UNSUPPORTED;
+    if (per_head)
+        for (int h = 0; h < s.Hq; h++)
+            if (head_pattern[h] < 0 || head_pattern[h] >= n_patterns) return SA_ERR_INVALID_ARG;
+    if (s.B == 0 || s.Hq == 0 || s.N == 0) return SA_OK;  // nothing to compute
+    if (s.Hkv <= 0 || s.Hq % s.Hkv != 0) return SA_ERR_UNSUPPORTED;
+    const int64_t T = (int64_t(s.N) + kBwdTile - 1) / kBwdTile;
+    for (int i = 0; i < n_patterns; i++) {
+        if (masks_t[i].n_q_tiles != T || masks_t[i].n_kv_tiles != T) return SA_ERR_MASK_MISMATCH;
+        if (!masks_t[i].kv_count || !masks_t[i].kv_index || !masks_t[i].kv_full) return SA_ERR_INVALID_ARG;
+    }
+    if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV || !workspace) return SA_ERR_INVALID_ARG;
+    if (!al16(Q) || !al16(K) || !al16(V) || !al16(O) || !al16(LSE) || !al16(dO) || !al16(dQ) || !al16(dK) ||
+        !al16(dV) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return SA_ERR_MISALIGNED;
+    if (workspace_bytes < bwd_layout(s).total) return SA_ERR_BUFFER_TOO_SMALL;
+    const int64_t rows = int64_t(s.B) * s.Hq * s.N;
+    if (int64_t(s.B) * s.Hkv * T > INT32_MAX || (rows + 7) / 8 > INT32_MAX) return SA_ERR_UNSUPPORTED;
+    BwdHeads hb{};
+    for (int i = 0; i < n_patterns; i++) {
+        const sa_pattern& pt = patterns[i];
+        BwdPattern& bp = hb.pat[i];
+        bp.t_count = masks_t[i].kv_count;
+        bp.t_index = masks_t[i].kv_index;
+        bp.t_full = masks_t[i].kv_full;
+        bp.window = pt.window > s.N ? s.N : pt.window;  // same allowed set, no int32 overflow in the kernel
+        bp.sinks = pt.sinks;
+        bp.stride = pt.stride;
+        bp.n_global = pt.n_global;
+        bp.causal = pt.causal;
+        bp.area = pt.area > s.N ? s.N : pt.area;
+        bp.summary = pt.summary < pt.area ? pt.summary : pt.area;
+    }
+    for (int h = 0; h < s.Hq; h++) hb.head[h] = per_head ? static_cast<uint8_t>(head_pattern[h]) : 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int32_t T32 = static_cast<int32_t>(T);
+    if (s.D == 128) return bwd_run<128>(Q, K, V, O, LSE, dO, hb, T32, s, scale, dQ, dK, dV, ws, st);
+    return bwd_run<64>(Q, K, V, O, LSE, dO, hb, T32, s, scale, dQ, dK, dV, ws, st);
 }
 
 }  // namespace
@@ -123,33 +183,17 @@ extern "C" int sparse_attn_bwd(const void* Q, const void* K, const void* V, cons
                                const sa_shape* shape, float scale, void* dQ, void* dK, void* dV, void* workspace,
                                size_t workspace_bytes, void* stream)
 {
-    if (!mask_t || !pattern || !shape) return SA_ERR_INVALID_ARG;
-    const sa_shape s = *shape;
-    const sa_pattern pt = *pattern;
-    if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
-    if (!(scale > 0.f) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
-    if (pt.window < -1 || pt.sinks < 0 || pt.stride < 0 || pt.n_global < 0 || pt.area < 0 || pt.summary < 0)
-        return SA_ERR_INVALID_ARG;
-    if (pt.summary > 0 && pt.area == 0) return SA_ERR_INVALID_ARG;
-    if (pt.causal != 0 && pt.causal != 1) return SA_ERR_UNSUPPORTED;
-    if (pt.stride > 0 && (pt.causal == 0 || pt.area > 0)) return SA_ERR_UNSUPPORTED;
-    if (s.D != 64 && s.D != 128) return SA_ERR_UNSUPPORTED;
-    if (mask_t->block != sa::kBwdTile) return SA_ERR_UNSUPPORTED;
-    if (s.B == 0 || s.Hq == 0 || s.N == 0) return SA_OK;  // nothing to compute
-    if (s.Hkv <= 0 || s.Hq % s.Hkv != 0) return SA_ERR_UNSUPPORTED;
-    const int64_t T = (int64_t(s.N) + sa::kBwdTile - 1) / sa::kBwdTile;
-    if (mask_t->n_q_tiles != T || mask_t->n_kv_tiles != T) return SA_ERR_MASK_MISMATCH;
-    if (!mask_t->kv_count || !mask_t->kv_index || !mask_t->kv_full) return SA_ERR_INVALID_ARG;
-    if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV || !workspace) return SA_ERR_INVALID_ARG;
-    using sa::al16;
-    if (!al16(Q) || !al16(K) || !al16(V) || !al16(O) || !al16(LSE) || !al16(dO) || !al16(dQ) || !al16(dK) ||
-        !al16(dV) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-        return SA_ERR_MISALIGNED;
-    if (workspace_bytes < sa::bwd_layout(s).total) return SA_ERR_BUFFER_TOO_SMALL;
-    const int64_t rows = int64_t(s.B) * s.Hq * s.N;
-    if (int64_t(s.B) * s.Hkv * T > INT32_MAX || (rows + 7) / 8 > INT32_MAX) return SA_ERR_UNSUPPORTED;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    if (s.D == 128) return sa::bwd_run<128>(Q, K, V, O, LSE, dO, *mask_t, pt, s, scale, dQ, dK, dV, ws, st);
-    return sa::bwd_run<64>(Q, K, V, O, LSE, dO, *mask_t, pt, s, scale, dQ, dK, dV, ws, st);
+    return sa::bwd_impl(Q, K, V, O, LSE, dO, mask_t, pattern, 1, nullptr, shape, scale, dQ, dK, dV, workspace,
+                        workspace_bytes, stream);
+}
+
+extern "C" int sparse_attn_bwd_heads(const void* Q, const void* K, const void* V, const void* O, const float* LSE,
+                                     const void* dO, const sa_block_mask* masks_t, const sa_pattern* patterns,
+                                     int32_t n_patterns, const int32_t* head_pattern, const sa_shape* shape,
+                                     float scale, void* dQ, void* dK, void* dV, void* workspace,
+                                     size_t workspace_bytes, void* stream)
+{
+    if (!head_pattern) return SA_ERR_INVALID_ARG;
+    return sa::bwd_impl(Q, K, V, O, LSE, dO, masks_t, patterns, n_patterns, head_pattern, shape, scale, dQ, dK, dV,
+                        workspace, workspace_bytes, stream);
 }

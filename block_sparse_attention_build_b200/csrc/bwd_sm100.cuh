@@ -67,10 +67,26 @@ enum : int32_t {
     ST_BWD_DRAIN_WAIT = 1 << 11,
 };
 
-struct BwdParams {
-    const int32_t* t_count;  // [T] query tiles listed for kv tile c (transposed block mask)
+// One pattern of the backward: its transposed block mask (per kv tile the
+// query tiles that attend to it) and the rule its partial tiles are masked
+// with.  Window and area clipped to N; summary <= area.
+struct BwdPattern {
+    const int32_t* t_count;  // [T] query tiles listed for kv tile c
     const int32_t* t_index;  // [T * T] their indices, ascending
     const uint8_t* t_full;   // [T * T] 1 when every in-range pair of the tile is allowed
+    int32_t window, sinks, stride, n_global, causal, area, summary;
+};
+constexpr int kBwdMaxPatterns = 8;
+constexpr int kBwdMaxHeads = 256;
+// The patterns of a backward launch and the pattern of each query head
+// (different heads of a layer may carry different patterns: "Sparse-
+// трансформеры" page, section "Комбинация — норма, а не исключение").
+struct BwdHeads {
+    BwdPattern pat[kBwdMaxPatterns];
+    uint8_t head[kBwdMaxHeads];
+};
+
+struct BwdParams {
     const float* lse2;       // [B * Hq * N] LSE in base 2; +inf for a row without keys
     const float* delta;      // [B * Hq * N] Δ = rowsum(dO ∘ O)
     float* dq_acc;           // [B * Hq * N * D] fp32, zeroed by the prep kernel
@@ -79,7 +95,6 @@ struct BwdParams {
     int32_t* status;
     long long timeout;       // SM cycles per bounded wait
     int32_t T, N, B, Hq, Hkv, group;
-    int32_t window, sinks, stride, n_global, causal, area, summary;  // window, area clipped to N; summary <= area
     float scale_log2;        // scale * log2(e)
     float scale;
 };
@@ -125,10 +140,10 @@ __device__ __forceinline__ uint32_t bwd_bits(int lo, int hi)
 // Allowed pairs (q, kv) for q = qb + i, i in [0, 32), as bits: the pattern's
 // rule (two-sided band, sink and global columns, global rows, stripe, stride)
 // under causality (if set) and the sequence bound.
-__device__ __forceinline__ uint32_t bwd_allow_word(const BwdParams& p, int qb, int kv)
+__device__ __forceinline__ uint32_t bwd_allow_word(const BwdPattern& p, int N, int qb, int kv)
 {
-    if (kv >= p.N) return 0u;
-    const uint32_t in_range = bwd_bits((p.causal ? kv : 0) - qb, p.N - 1 - qb);  // (kv <=) q < N
+    if (kv >= N) return 0u;
+    const uint32_t in_range = bwd_bits((p.causal ? kv : 0) - qb, N - 1 - qb);  // (kv <=) q < N
     if (kv < max(p.sinks, p.n_global)) return in_range;
     if (p.summary > 0 && kv % p.area >= p.area - p.summary) return in_range;  // a summary column
     uint32_t m = 0u;
@@ -213,7 +228,8 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ a
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
-               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const BwdParams p)
+               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const BwdParams p,
+               const __grid_constant__ BwdHeads hb)
 {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -242,8 +258,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int c = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.B * p.Hkv));
     const int b = bh / p.Hkv;
     const int hkv = bh % p.Hkv;
-    const int n_list = min(max(__ldg(&p.t_count[c]), 0), p.T);
-    const int steps = p.group * n_list;
+    // steps: for each query head of the group, the query tiles of its pattern's list for kv tile c
+    auto list_len = [&](int h) {
+        const BwdPattern& bp = hb.pat[hb.head[hkv * p.group + h]];
+        return min(max(__ldg(&bp.t_count[c]), 0), p.T);
+    };
+    int steps = 0;
+    for (int h = 0; h < p.group; h++) steps += list_len(h);
     const int halves = 2 * steps;  // half-step k: step k / 2, query columns 64 (k % 2) .. +63
 
     if (threadIdx.x == 0) {
@@ -276,13 +297,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const long long lim = p.timeout;
 
-    // query head and query tile of step j (heads outer, list entries inner)
-    auto step_of = [&](int j, int& hq, int& r, bool& full) {
-        const int h = j / n_list;
-        const int e = j - h * n_list;
-        r = min(max(__ldg(&p.t_index[int64_t(c) * p.T + e]), 0), p.T - 1);
-        full = __ldg(&p.t_full[int64_t(c) * p.T + e]) != 0;
+    // query head, query tile and pattern of step j (heads outer, list entries inner)
+    auto step_of = [&](int j, int& hq, int& r, bool& full) -> const BwdPattern& {
+        int h = 0, e = j;
+        for (; h < p.group - 1; h++) {
+            const int n_h = list_len(h);
+            if (e < n_h) break;
+            e -= n_h;
+        }
         hq = hkv * p.group + h;
+        const BwdPattern& bp = hb.pat[hb.head[hq]];
+        r = min(max(__ldg(&bp.t_index[int64_t(c) * p.T + e]), 0), p.T - 1);
+        full = __ldg(&bp.t_full[int64_t(c) * p.T + e]) != 0;
+        return bp;
     };
 
     if (warp == kBwdProducerWarp) {
@@ -491,7 +518,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int j = k >> 1;
             int hq, r;
             bool full;
-            step_of(j, hq, r, full);
+            const BwdPattern& bp = step_of(j, hq, r, full);
             const int q0 = r * kBwdTile;
             const int qc = q0 + hf * 64 + sub * 32;  // first query column of this thread's chunk
             const int64_t qrow0 = (int64_t(b) * p.Hq + hq) * p.N;
@@ -499,7 +526,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float lse_c = qc + lane < p.N ? __ldg(&p.lse2[qrow0 + qc + lane]) : INFINITY;
             const float dl_c = qc + lane < p.N ? __ldg(&p.delta[qrow0 + qc + lane]) : 0.f;
             const bool masked = !full || kv_ragged || q0 + kBwdTile > p.N;
-            const uint32_t allow = masked ? bwd_allow_word(p, qc, kv) : 0xffffffffu;
+            const uint32_t allow = masked ? bwd_allow_word(bp, p.N, qc, kv) : 0xffffffffu;
             ok = __all_sync(0xffffffffu, mbar_wait(&s_full[hf], j & 1, lim) && !*abort_flag);
             if (!ok) break;
             tc_fence_after_sync();

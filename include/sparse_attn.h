@@ -286,6 +286,20 @@ int sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O, 
                     void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward pass with a pattern per query head, the gradients of
+ * sparse_attn_fwd_heads: query head h under patterns[head_pattern[h]], whose
+ * TRANSPOSED block mask (device arrays, block 128) is masks_t[head_pattern[h]];
+ * for grouped heads dK, dV sum the heads of the group, each under its own
+ * pattern.  n_patterns 1 .. 8, head_pattern [Hq] (host), Hq <= 256; other
+ * arguments, layouts and errors as sparse_attn_bwd (SA_ERR_INVALID_ARG for a
+ * null head table, a count out of range or an index outside [0, n_patterns)).
+ */
+int sparse_attn_bwd_heads(const void* Q, const void* K, const void* V, const void* O, const float* LSE,
+                          const void* dO, const sa_block_mask* masks_t, const sa_pattern* patterns, int32_t n_patterns,
+                          const int32_t* head_pattern, const sa_shape* shape, float scale, void* dQ, void* dK,
+                          void* dV, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Stride-aware path for causal patterns with a stride s (every s-th prior
  * token): in token order those pairs touch every tile below the diagonal once
  * per row.  The plan splits the pattern into

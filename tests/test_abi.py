@@ -348,3 +348,33 @@ def test_stride_plan_errors():
     assert call(good, ws=fake + 16) == sa.SA_ERR_MISALIGNED
     assert call(good, nbytes=100) == sa.SA_ERR_BUFFER_TOO_SMALL
     assert call(good, ptr=fake + 8) == sa.SA_ERR_MISALIGNED
+
+
+def test_bwd_heads_argument_errors_without_gpu():
+    p = sa.Pattern(window=8)._c()
+    p2 = sa.Pattern(window=4, stride=16)._c()
+    m = sa._BlockMask(1, 1, 128, 1, 1, 0, 16, 16, 16)
+    m64 = sa._BlockMask(2, 2, 64, 1, 1, 0, 16, 16, 16)
+    fake = 1 << 20
+    ws = sa.bwd_workspace_bytes(1, 2, 2, 100, 128)
+
+    def call(shape, heads, masks=(m, m), pats=(p, p2), n=None):
+        n = len(pats) if n is None else n
+        cm = (sa._BlockMask * len(masks))(*masks)
+        cp = (sa._Pattern * len(pats))(*pats)
+        ch = (ctypes.c_int32 * max(len(heads), 1))(*heads)
+        return sa.lib.sparse_attn_bwd_heads(fake, fake, fake, fake, fake, fake, cm, cp, n, ch,
+                                            ctypes.byref(sa._Shape(*shape)), 0.125, fake, fake, fake, fake, ws, None)
+
+    assert call((1, 2, 2, 100, 128), [0, 1], n=0) == sa.SA_ERR_INVALID_ARG
+    assert call((1, 2, 2, 100, 128), [0, 1], n=9) == sa.SA_ERR_INVALID_ARG
+    assert call((1, 2, 2, 100, 128), [0, 2]) == sa.SA_ERR_INVALID_ARG
+    assert call((1, 2, 2, 100, 128), [0, 1], masks=(m, m64)) == sa.SA_ERR_UNSUPPORTED   # block 64
+    assert call((1, 300, 300, 100, 128), [0] * 300) == sa.SA_ERR_UNSUPPORTED
+    bad = sa.Pattern(window=8, stride=4, causal=0)._c()
+    assert call((1, 2, 2, 100, 128), [0, 1], pats=(p, bad)) == sa.SA_ERR_UNSUPPORTED
+    assert call((0, 2, 2, 100, 128), [0, 1]) == sa.SA_OK
+    rc = sa.lib.sparse_attn_bwd_heads(fake, fake, fake, fake, fake, fake, (sa._BlockMask * 1)(m),
+                                      (sa._Pattern * 1)(p), 1, None, ctypes.byref(sa._Shape(1, 2, 2, 100, 128)),
+                                      0.125, fake, fake, fake, fake, ws, None)
+    assert rc == sa.SA_ERR_INVALID_ARG
