@@ -17,18 +17,35 @@ namespace {
 constexpr int kMaxDev = 64;
 
 struct BwdLayout {
-    size_t lse2, delta, dq, total;  // byte offsets in the workspace, each 256-aligned
+    size_t lse2, delta, dq, dk, dv, items, n_items, split, steps, total;  // byte offsets, each 256-aligned
 };
+
+// Work items: at most one per (kv tile, kv head) plus one per kBwdChunk steps
+// of its list (a list holds at most group * T steps).
+size_t bwd_item_capacity(const sa_shape& s)
+{
+    const size_t T = (size_t(s.N) + kBwdTile - 1) / kBwdTile;
+    const size_t group = s.Hkv > 0 ? size_t(s.Hq) / size_t(s.Hkv) : 0;
+    return T * size_t(s.Hkv) * (1 + (group * T + kBwdChunk - 1) / kBwdChunk);
+}
 
 BwdLayout bwd_layout(const sa_shape& s)
 {
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
     const size_t rows = size_t(s.B) * size_t(s.Hq) * size_t(s.N);
+    const size_t kvrows = size_t(s.B) * size_t(s.Hkv) * size_t(s.N);
+    const size_t T = (size_t(s.N) + kBwdTile - 1) / kBwdTile;
     BwdLayout w;
     w.lse2 = 0;
     w.delta = up(rows * 4);
     w.dq = w.delta + up(rows * 4);
-    w.total = w.dq + up(rows * size_t(s.D) * 4);
+    w.dk = w.dq + up(rows * size_t(s.D) * 4);
+    w.dv = w.dk + up(kvrows * size_t(s.D) * 4);
+    w.items = w.dv + up(kvrows * size_t(s.D) * 4);
+    w.n_items = w.items + up(bwd_item_capacity(s) * 16);
+    w.split = w.n_items + 256;
+    w.steps = w.split + up(T * size_t(s.Hkv));
+    w.total = w.steps + up(T * size_t(s.Hkv) * 4);
     return w;
 }
 
@@ -45,6 +62,10 @@ int bwd_run(const void* Q, const void* K, const void* V, const void* O, const fl
     float* lse2 = reinterpret_cast<float*>(ws + L.lse2);
     float* delta = reinterpret_cast<float*>(ws + L.delta);
     float* dq_acc = reinterpret_cast<float*>(ws + L.dq);
+    int4* items = reinterpret_cast<int4*>(ws + L.items);
+    int32_t* n_items = reinterpret_cast<int32_t*>(ws + L.n_items);
+    uint8_t* split = ws + L.split;
+    int32_t* steps_scratch = reinterpret_cast<int32_t*>(ws + L.steps);
     const int64_t rows = int64_t(s.B) * s.Hq * s.N;
 
     CUtensorMap mq, mdo, mk, mv;
@@ -54,11 +75,12 @@ int bwd_run(const void* Q, const void* K, const void* V, const void* O, const fl
         !make_map_bf16_3d(&mv, V, D, s.N, uint64_t(s.B) * s.Hkv, kBwdTile))
         return SA_ERR_CUDA;
 
-    bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, lse2, delta, dq_acc, rows);
-    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-
     BwdParams p;
+    p.items = items;
+    p.n_items = n_items;
+    p.split = split;
+    p.dk_acc = reinterpret_cast<float*>(ws + L.dk);
+    p.dv_acc = reinterpret_cast<float*>(ws + L.dv);
     p.lse2 = lse2;
     p.delta = delta;
     p.dq_acc = dq_acc;
@@ -85,15 +107,24 @@ int bwd_run(const void* Q, const void* K, const void* V, const void* O, const fl
             return SA_ERR_CUDA;
         attr_set[dev] = true;
     }
-    const unsigned grid = static_cast<unsigned>(int64_t(s.B) * s.Hkv * p.T);
-    bwd_kernel<D><<<grid, kBwdThreads, C::kSmemBytes, st>>>(mq, mdo, mk, mv, p, hb);
-    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-
-    const int64_t n8 = rows * D / 8;
     const int n_sm = device_sm_count();
-    int64_t g = (n8 + 255) / 256;
-    if (n_sm > 0 && g > int64_t(n_sm) * 8) g = int64_t(n_sm) * 8;
-    bwd_dq_kernel<<<static_cast<unsigned>(g), 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), n8);
+    if (n_sm <= 0) return SA_ERR_CUDA;
+    p.n_sm = n_sm;
+    auto grid_for = [&](int64_t n) {
+        int64_t g = (n + 255) / 256;
+        if (g > int64_t(n_sm) * 8) g = int64_t(n_sm) * 8;
+        return static_cast<unsigned>(g > 0 ? g : 1);
+    };
+    // work items; the prep kernel (row terms, zeroed dQ sums and the fp32 sums
+    // of split kv tiles); the main kernel (persistent, one CTA per SM); the
+    // conversions to bf16 (dQ, and dK, dV of split tiles)
+    bwd_items_kernel<<<1, 1024, 0, st>>>(p, hb, items, n_items, split, steps_scratch);
+    bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, lse2, delta, dq_acc, rows, p);
+    bwd_kernel<D><<<static_cast<unsigned>(n_sm), kBwdThreads, C::kSmemBytes, st>>>(mq, mdo, mk, mv, p, hb);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+    const int64_t n8 = rows * D / 8;
+    bwd_dq_kernel<D><<<grid_for(n8), 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), n8, p);
     return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
