@@ -115,7 +115,12 @@ struct ResidualStride {
     int32_t shift;   // floor(window / stride) + 1 (0 without a band)
     int32_t col_lo;  // max(sinks, n_global)
     int32_t stride;
+    bool view;       // Q, K, V, O are token-order tensors read and written through grouped-view maps
 };
+
+// Grouped-view maps need the group length to be a multiple of the tile
+// heights (128 query rows, `block` kv rows): a tile never spans two groups.
+bool grouped_view_ok(int32_t n, int32_t block) { return n % kBM == 0 && n % block == 0; }
 
 // The forward pass behind sparse_attn_fwd (one pattern: n_patterns = 1,
 // head_pattern = null), sparse_attn_fwd_heads (a pattern per query head) and
@@ -181,11 +186,20 @@ int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* m
 
     CUtensorMap mq, mk, mv, mo;
     const uint32_t bn = static_cast<uint32_t>(mask->block);
-    if (!make_map_bf16_3d(&mq, Q, s.D, s.N, uint64_t(s.B) * s.Hq, kBM) ||
-        !make_map_bf16_3d(&mk, K, s.D, s.N, uint64_t(s.B) * s.Hkv, bn) ||
-        !make_map_bf16_3d(&mv, V, s.D, s.N, uint64_t(s.B) * s.Hkv, bn) ||
-        !make_map_bf16_3d(&mo, O, s.D, s.N, uint64_t(s.B) * s.Hq, bn))
+    const bool view = rs && rs->view;
+    if (view) {
+        const uint64_t sg = static_cast<uint64_t>(rs->stride);
+        if (!make_map_bf16_grouped(&mq, Q, s.D, s.N, uint64_t(s.B) * s.Hq, sg, kBM) ||
+            !make_map_bf16_grouped(&mk, K, s.D, s.N, uint64_t(s.B) * s.Hkv, sg, bn) ||
+            !make_map_bf16_grouped(&mv, V, s.D, s.N, uint64_t(s.B) * s.Hkv, sg, bn) ||
+            !make_map_bf16_grouped(&mo, O, s.D, s.N, uint64_t(s.B) * s.Hq, sg, bn))
+            return SA_ERR_CUDA;
+    } else if (!make_map_bf16_3d(&mq, Q, s.D, s.N, uint64_t(s.B) * s.Hq, kBM) ||
+               !make_map_bf16_3d(&mk, K, s.D, s.N, uint64_t(s.B) * s.Hkv, bn) ||
+               !make_map_bf16_3d(&mv, V, s.D, s.N, uint64_t(s.B) * s.Hkv, bn) ||
+               !make_map_bf16_3d(&mo, O, s.D, s.N, uint64_t(s.B) * s.Hq, bn)) {
         return SA_ERR_CUDA;
+    }
 
     FwdParams p;
     p.kv_count = mask->kv_count;
@@ -215,6 +229,8 @@ int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* m
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int g = static_cast<int>(grid);
     HeadPatterns hp{};
+    hp.grp_n = view ? rs->n : 0;
+    hp.grp_s = view ? rs->stride : 0;
     if (!multi) return launch_any<false>(s.D, mask->block, mq, mk, mv, mo, p, hp, g, st);
     for (int i = 0; i < n_patterns; i++) {
         hp.pat[i].kv_count = masks[i].kv_count;
@@ -309,13 +325,18 @@ int stride_run(const void* Q, const void* K, const void* V, const sa_block_mask*
     const int n = s.N / pt.stride;
     constexpr int U = D * 2 / 16;
     const int64_t qp = int64_t(s.B) * s.Hq, kp = int64_t(s.B) * s.Hkv;
-    group_by_residue_kernel<D><<<grid_for(qp * s.N * U), 256, 0, st>>>(
-        static_cast<const uint4*>(Q), reinterpret_cast<uint4*>(ws + L.q), qp, s.N, pt.stride, n);
-    group_by_residue_kernel<D><<<grid_for(kp * s.N * U), 256, 0, st>>>(
-        static_cast<const uint4*>(K), reinterpret_cast<uint4*>(ws + L.k), kp, s.N, pt.stride, n);
-    group_by_residue_kernel<D><<<grid_for(kp * s.N * U), 256, 0, st>>>(
-        static_cast<const uint4*>(V), reinterpret_cast<uint4*>(ws + L.v), kp, s.N, pt.stride, n);
-    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+    // pass 2 reads and writes the token-order tensors through grouped-view maps
+    // when the group length fits the tiles; else through grouped copies
+    const bool view = grouped_view_ok(n, pass2->block);
+    if (!view) {
+        group_by_residue_kernel<D><<<grid_for(qp * s.N * U), 256, 0, st>>>(
+            static_cast<const uint4*>(Q), reinterpret_cast<uint4*>(ws + L.q), qp, s.N, pt.stride, n);
+        group_by_residue_kernel<D><<<grid_for(kp * s.N * U), 256, 0, st>>>(
+            static_cast<const uint4*>(K), reinterpret_cast<uint4*>(ws + L.k), kp, s.N, pt.stride, n);
+        group_by_residue_kernel<D><<<grid_for(kp * s.N * U), 256, 0, st>>>(
+            static_cast<const uint4*>(V), reinterpret_cast<uint4*>(ws + L.v), kp, s.N, pt.stride, n);
+        if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+    }
     // pass 1: the pattern without its stride, token order; O holds O1, L1 in the workspace
     sa_pattern p1 = pt;
     p1.stride = 0;
@@ -327,12 +348,16 @@ int stride_run(const void* Q, const void* K, const void* V, const sa_block_mask*
     rs.shift = pt.window >= 0 ? (pt.window > s.N ? s.N : pt.window) / pt.stride + 1 : 0;
     rs.col_lo = pt.sinks > pt.n_global ? pt.sinks : pt.n_global;
     rs.stride = pt.stride;
+    rs.view = view;
     float* l2 = reinterpret_cast<float*>(ws + L.l2);
-    if (int rc = fwd_impl(ws + L.q, ws + L.k, ws + L.v, pass2, &pt, 1, nullptr, &s, scale, ws + L.o2, l2, st, &rs))
-        return rc;
+    const void* q2 = view ? Q : static_cast<const void*>(ws + L.q);
+    const void* k2 = view ? K : static_cast<const void*>(ws + L.k);
+    const void* v2 = view ? V : static_cast<const void*>(ws + L.v);
+    if (int rc = fwd_impl(q2, k2, v2, pass2, &pt, 1, nullptr, &s, scale, ws + L.o2, l2, st, &rs)) return rc;
+    // with the grouped view pass 2's O and LSE are already in token order
     merge_passes_kernel<D><<<grid_for(qp * s.N * U), 256, 0, st>>>(
         static_cast<__nv_bfloat16*>(O), LSE, reinterpret_cast<const __nv_bfloat16*>(ws + L.o2), l1, l2, qp, s.N,
-        pt.stride, n);
+        view ? 1 : pt.stride, view ? s.N : n);
     return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 

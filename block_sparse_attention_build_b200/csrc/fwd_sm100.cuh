@@ -118,6 +118,10 @@ struct PatternRef {
 struct HeadPatterns {
     PatternRef pat[kMaxPatterns];
     uint8_t head[kMaxHeadsMulti];  // pattern of each query head
+    // > 0: the tensor maps view the residue-grouped order P = (t mod grp_s) *
+    // grp_n + t / grp_s of token-order tensors as 4-D (feature, P / grp_n,
+    // P mod grp_n, plane); LSE and zeroed O rows go to token t
+    int32_t grp_n, grp_s;
 };
 
 enum : int32_t {
@@ -517,6 +521,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const long long lim = p.timeout;
+    // rows r0 .. of a plane into / out of shared memory: the token-order 3-D maps,
+    // or (pattern-table kernel, grouped view) the 4-D maps at (P / n, P mod n)
+    const int grp_n = MULTI ? hp.grp_n : 0;
+    const int grp_s = MULTI ? hp.grp_s : 0;
+    auto load_rows = [grp_n](void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int r0, int plane,
+                             uint64_t pol) {
+        if (MULTI && grp_n > 0)
+            tma_load_4d(dst, map, bar, c0, r0 / grp_n, r0 % grp_n, plane, pol);
+        else
+            tma_load_3d(dst, map, bar, c0, r0, plane, pol);
+    };
+    auto store_rows = [grp_n](const CUtensorMap* map, const void* src, int c0, int r0, int plane) {
+        if (MULTI && grp_n > 0)
+            tma_store_4d(map, src, c0, r0 / grp_n, r0 % grp_n, plane);
+        else
+            tma_store_3d(map, src, c0, r0, plane);
+    };
     // warp-uniform warpgroup index, so that the register split applies per branch
     const int wg = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x) / 128, 0);
 
@@ -586,8 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (elect_one()) {
                             mbar_arrive_expect_tx(&q_full[x], C::kQBytes);
                             for (int c = 0; c < D / 64; c++)
-                                tma_load_3d(sQ + x * C::kQBytes + c * C::kQPanel, &tmQ, &q_full[x], c * 64,
-                                            w.qtile[x] * kBM, w.b * p.Hq + w.hq[x], pol_q);
+                                load_rows(sQ + x * C::kQBytes + c * C::kQPanel, &tmQ, &q_full[x], c * 64,
+                                          w.qtile[x] * kBM, w.b * p.Hq + w.hq[x], pol_q);
                         }
                         __syncwarp();
                         q_issued[x]++;
@@ -605,8 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (elect_one()) {
                                 mbar_arrive_expect_tx(&ring_full[st], C::kKVBytes);
                                 for (int c = 0; c < D / 64; c++)
-                                    tma_load_3d(ring + st * C::kKVBytes + c * C::kKVPanel, v == 0 ? &tmK : &tmV,
-                                                &ring_full[st], c * 64, kv * BN, plane, pol_kv);
+                                    load_rows(ring + st * C::kKVBytes + c * C::kKVPanel, v == 0 ? &tmK : &tmV,
+                                              &ring_full[st], c * 64, kv * BN, plane, pol_kv);
                             }
                             __syncwarp();
                             pos++;
@@ -627,8 +648,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (elect_one()) {
                                 mbar_arrive_expect_tx(&ring_full[st], C::kKVBytes);
                                 for (int c = 0; c < D / 64; c++)
-                                    tma_load_3d(ring + st * C::kKVBytes + c * C::kKVPanel, is_v ? &tmV : &tmK,
-                                                &ring_full[st], c * 64, kv * BN, plane, pol_kv);
+                                    load_rows(ring + st * C::kKVBytes + c * C::kKVPanel, is_v ? &tmV : &tmK,
+                                              &ring_full[st], c * 64, kv * BN, plane, pol_kv);
                             }
                             __syncwarp();
                             pos++;
@@ -887,8 +908,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int plane = w.b * p.Hq + w.hq[x];
                     for (int b = 0; b < C::kOBlocks; b++)
                         for (int c = 0; c < D / 64; c++)
-                            tma_store_3d(&tmO, ring + ((first + b) % S) * C::kKVBytes + c * C::kKVPanel, c * 64,
-                                         w.qtile[x] * kBM + b * BN, plane);
+                            store_rows(&tmO, ring + ((first + b) % S) * C::kKVBytes + c * C::kKVPanel, c * 64,
+                                       w.qtile[x] * kBM + b * BN, plane);
                     bulk_commit_group();
                     bulk_wait_read_all();
                     for (int b = 0; b < C::kOBlocks; b++) mbar_arrive(&ring_empty[(first + b) % S]);
@@ -930,7 +951,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 continue;
             }
             const int q = (x == 0 ? w.qtile[0] : w.qtile[1]) * kBM + row;
-            const int64_t orow = (static_cast<int64_t>(w.b) * p.Hq + (x == 0 ? w.hq[0] : w.hq[1])) * p.N + q;
+            // token row of query q (grouped view: t = (q mod n) s + q / n)
+            const int qt = (MULTI && grp_n > 0) ? (q % grp_n) * grp_s + q / grp_n : q;
+            const int64_t orow = (static_cast<int64_t>(w.b) * p.Hq + (x == 0 ? w.hq[0] : w.hq[1])) * p.N + qt;
             if constexpr (MULTI) {
                 const PatternRef& pr = hp.pat[hp.head[x == 0 ? w.hq[0] : w.hq[1]]];
                 if (pr.mode == 1) {
