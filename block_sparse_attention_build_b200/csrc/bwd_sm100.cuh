@@ -597,20 +597,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         auto issue_sdp = [&](int q, int hf) {
             const uint32_t bo = (q & 1) * kTileU + hf * kHalfRowsU;
             const uint32_t col = tmem + hf * 128;
+            if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; kk++) {
-                if (elect_one())
+                for (int kk = 0; kk < D / 16; kk++)
                     mma_ss(col, desc_from_halves(k_km + km(kk), hi), desc_from_halves(q_km + bo + km(kk), hi), id_s,
                            kk > 0 ? 1u : 0u);
-                __syncwarp();
             }
+            __syncwarp();
+            if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; kk++) {
-                if (elect_one())
+                for (int kk = 0; kk < D / 16; kk++)
                     mma_ss(col + 64, desc_from_halves(v_km + km(kk), hi), desc_from_halves(o_km + bo + km(kk), hi),
                            id_s, kk > 0 ? 1u : 0u);
-                __syncwarp();
             }
+            __syncwarp();
             commit(&s_full[hf]);
         };
         bool ok = true;
@@ -651,30 +651,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 // dV += Pᵀ dO and dK += dSᵀ Q over this half's 64 query rows (K = 64): A
                 // from tensor memory, query columns 32u .. 32u+31 of the half hold Pᵀ
                 // in packed columns 32u .. 32u+15 and dSᵀ in 32u+16 .. 32u+31
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < 4; kk++) {
-                    if (elect_one())
+                    for (int kk = 0; kk < 4; kk++)
                         mma_ts(tmem + C::kColdV, scol + (kk / 2) * 32 + (kk % 2) * 8,
                                desc_from_halves(o_mn + bo + mn(kk), hi), id_kv, (k > 0 || kk > 0) ? 1u : 0u);
-                    __syncwarp();
                 }
+                __syncwarp();
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < 4; kk++) {
-                    if (elect_one())
+                    for (int kk = 0; kk < 4; kk++)
                         mma_ts(tmem + C::kColdK, scol + (kk / 2) * 32 + 16 + (kk % 2) * 8,
                                desc_from_halves(q_mn + bo + mn(kk), hi), id_kv, (k > 0 || kk > 0) ? 1u : 0u);
-                    __syncwarp();
                 }
+                __syncwarp();
                 if (hf) commit(&qd_empty[q & 1]);
                 // dQᵀ = Kᵀ dSᵀ (M = feature rows, N = 64 query rows, K = kv rows), into
                 // the half's dPᵀ columns; dSᵀ of half hf is panel hf of the shared tile
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < kBwdTile / 16; kk++) {
-                    if (elect_one())
+                    for (int kk = 0; kk < kBwdTile / 16; kk++)
                         mma_ss(scol + 64, desc_from_halves(k_mn + mn(kk), hi),
                                desc_from_halves(s_mn + hf * (C::kPanel >> 4) + mn(kk), hi), id_q, kk > 0 ? 1u : 0u);
-                    __syncwarp();
                 }
+                __syncwarp();
                 commit(&dq_full[hf]);
             }
             commit(kv_empty);  // every MMA of this item issued: K, V free once they complete

@@ -704,26 +704,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto issue_s = [&](int x, int stage) {
                 const uint32_t a0 = q_lo + static_cast<uint32_t>((x * C::kQBytes) >> 4);
                 const uint32_t b0 = k_lo + static_cast<uint32_t>((stage * C::kKVBytes) >> 4);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; kk++) {
-                    const uint32_t qo = static_cast<uint32_t>(((kk / 4) * C::kQPanel + (kk % 4) * 32) >> 4);
-                    const uint32_t ko = static_cast<uint32_t>(((kk / 4) * C::kKVPanel + (kk % 4) * 32) >> 4);
-                    if (elect_one())
+                    for (int kk = 0; kk < D / 16; kk++) {
+                        const uint32_t qo = static_cast<uint32_t>(((kk / 4) * C::kQPanel + (kk % 4) * 32) >> 4);
+                        const uint32_t ko = static_cast<uint32_t>(((kk / 4) * C::kKVPanel + (kk % 4) * 32) >> 4);
                         mma_ss(tm + x * BN, desc_from_halves(a0 + qo, d_hi), desc_from_halves(b0 + ko, d_hi), idesc_s,
                                kk > 0 ? 1u : 0u);
-                    __syncwarp();
+                    }
                 }
+                __syncwarp();
             };
             auto issue_pv = [&](int x, int stage, bool accumulate) {
                 const uint32_t b0 = v_lo + static_cast<uint32_t>((stage * C::kKVBytes) >> 4);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; kk++) {
-                    if (elect_one())
+                    for (int kk = 0; kk < BN / 16; kk++)
                         mma_ts(tm + 2 * BN + x * D, tm + x * BN + kk * 8,
                                desc_from_halves(b0 + static_cast<uint32_t>(kk * 128), d_hi), idesc_o,
                                (accumulate || kk > 0) ? 1u : 0u);
-                    __syncwarp();
                 }
+                __syncwarp();
             };
             // every lane polls; the outcome is made warp-uniform
             auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
