@@ -197,6 +197,10 @@ HEAD_CASES = [
     (2, 4, 2, 777, 64, 64, [sa.Pattern(window=100, sinks=3), sa.Pattern(window=0, stride=37, n_global=5)], [0, 1, 1, 0]),
     (1, 6, 2, 1300, 128, 128,
      [sa.Pattern(window=300), sa.Pattern(window=1300), sa.Pattern(window=20, sinks=130)], [0, 1, 2, 2, 1, 0]),
+    # one query head of each kv group sees no key at all: in every unit one slot has
+    # no live step (its rows are O = 0, LSE = -inf) while the other runs
+    (1, 4, 2, 900, 128, 128, [sa.Pattern(window=200, sinks=4), sa.Pattern(window=-1)], [0, 1, 1, 0]),
+    (1, 4, 2, 700, 64, 64, [sa.Pattern(window=-1), sa.Pattern(window=90, sinks=2)], [0, 1, 1, 0]),
 ]
 
 
