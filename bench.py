@@ -176,10 +176,10 @@ def _sample_rows(w, n):
 
 
 def _sample_flops(w, rows):
-    """Useful FLOP of the sampled rows: 4 * D * (allowed keys of each row) * B * Hq."""
-    import block_sparse_attention_build_b200 as sa
-    p = sa.Pattern(**w.pattern_args())
-    keys = sum(sa.count_pairs(p, int(r) + 1) - sa.count_pairs(p, int(r)) for r in rows)
+    """Useful FLOP of the sampled rows: 4 * D * (allowed keys of each row) * B * Hq,
+    the keys counted by the oracle (the CPU arms never load the CUDA library)."""
+    import oracle
+    keys = int(oracle.row_counts(oracle.Pattern(**w.pattern_args()), w.N, rows).sum())
     return 4.0 * w.D * keys * w.B * w.Hq
 
 
@@ -374,19 +374,20 @@ def run_gpu(args, w):
                          device=dev)
         e2e_steps = max(3, min(args.steps, 20))
         for _ in range(2):
-            sa.fwd_host(Qh, Kh, Vh, mask, p, Oh, Lh, ws, scale=w.scale, stream=stream)
+            sa.fwd_host(Qh, Kh, Vh, mask_h, p, Oh, Lh, ws, scale=w.scale, stream=stream)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
         e0.record(stream)
         for _ in range(e2e_steps):
-            sa.fwd_host(Qh, Kh, Vh, mask, p, Oh, Lh, ws, scale=w.scale, stream=stream)
+            sa.fwd_host(Qh, Kh, Vh, mask_h, p, Oh, Lh, ws, scale=w.scale, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = e0.elapsed_time(e1)
         e2e_ms = max_over_ranks(e2e_ms, dist if world > 1 else None, dev)
         h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh))
+        h2d += sum(a.nbytes for a in (mask_h.counts, mask_h.index, mask_h.full))  # the host block mask
         d2h = Oh.numel() * Oh.element_size() + Lh.numel() * Lh.element_size()
         e2e = {"value": job_tflops(world, useful, e2e_steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,

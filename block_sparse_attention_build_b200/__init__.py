@@ -422,8 +422,11 @@ def fwd_host_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, D: int) -> int:
 def fwd_host(q_host, k_host, v_host, mask: BlockMask, pattern: Pattern, o_host, lse_host, workspace,
              scale: float | None = None, stream=None) -> None:
     """Forward from host (ideally pinned) tensors: copies in, computes, copies
-    out and waits.  ``workspace`` is a device tensor of at least
-    ``fwd_host_workspace_bytes`` bytes; ``mask`` is device-resident."""
+    out and waits, in chunks of kv heads whose copies overlap the kernels.
+    ``workspace`` is a device tensor of at least ``fwd_host_workspace_bytes``
+    bytes; ``mask`` is the HOST block mask from ``build_block_mask``."""
+    if not isinstance(mask.counts, np.ndarray):
+        raise TypeError("fwd_host takes the host block mask (numpy arrays), not a device copy")
     B, Hq, N, D = q_host.shape
     Hkv = k_host.shape[1]
     if scale is None:

@@ -30,9 +30,14 @@ int status_word(int32_t** out)
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SA_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_status[dev]) {
+        // first use on this device: allocate and clear the word, and wait for
+        // the clear, so that no stream's kernel can see it before it is zero
         int32_t* p = nullptr;
         if (cudaMalloc(&p, sizeof(int32_t)) != cudaSuccess) return SA_ERR_CUDA;
-        if (cudaMemset(p, 0, sizeof(int32_t)) != cudaSuccess) return SA_ERR_CUDA;
+        if (cudaMemset(p, 0, sizeof(int32_t)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+            cudaFree(p);
+            return SA_ERR_CUDA;
+        }
         g_status[dev] = p;
     }
     *out = g_status[dev];
@@ -159,7 +164,8 @@ int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* m
 
     if (T > kMaxTiles) return SA_ERR_UNSUPPORTED;
     if (!Q || !K || !V || !O || !LSE) return SA_ERR_INVALID_ARG;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    // LSE is written one fp32 at a time: 4-byte alignment is enough
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || (reinterpret_cast<uintptr_t>(LSE) & 3u))
         return SA_ERR_MISALIGNED;
     const int64_t n_qtiles = (int64_t(s.N) + kBM - 1) / kBM;
     const int64_t group = s.Hq / s.Hkv;
@@ -264,6 +270,29 @@ long long wait_limit_cycles()
 {
     std::lock_guard<std::mutex> lk(g_mu);
     return g_timeout;
+}
+
+int32_t debug_flags()
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    return g_debug_flags;
+}
+
+int check_host_mask(const sa_block_mask* m, int64_t T)
+{
+    if (!m || !m->kv_count || !m->kv_index || !m->kv_full) return SA_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < T; i++) {
+        const int32_t c = m->kv_count[i];
+        if (c < 0 || c > T) return SA_ERR_INVALID_ARG;
+        const int32_t* idx = m->kv_index + i * T;
+        const uint8_t* full = m->kv_full + i * T;
+        int32_t prev = -1;
+        for (int32_t e = 0; e < c; e++) {
+            if (idx[e] <= prev || idx[e] >= T || full[e] > 1) return SA_ERR_INVALID_ARG;
+            prev = idx[e];
+        }
+    }
+    return SA_OK;
 }
 
 int device_sm_count() { return sm_count(); }
@@ -400,50 +429,173 @@ extern "C" int sparse_attn_fwd_stride(const void* Q, const void* K, const void* 
     return sa::stride_run<64>(Q, K, V, pass1, pass2, pt, s, scale, O, LSE, ws, st);
 }
 
+namespace sa {
+namespace {
+
+// The host-buffer path works in chunks of whole kv heads (flattened over batch
+// and head, index b * Hkv + h): a chunk's Q, K, V, O and LSE are one
+// contiguous byte range of each tensor, so each moves with one copy, and chunk
+// c + 1's inputs cross the bus while chunk c computes and chunk c - 1's
+// outputs come back.
+constexpr int kHostChunks = 16;
+
+struct HostLayout {
+    size_t count, index, full, q, k, v, o, lse, total;  // byte offsets, each 256-aligned
+};
+
+HostLayout host_layout(const sa_shape& s)
+{
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    // the mask copy is sized for the smaller tile (64), which has more tiles
+    const size_t T = (size_t(s.N) + 63) / 64;
+    const size_t qb = size_t(s.B) * s.Hq * s.N * s.D * 2, kvb = size_t(s.B) * s.Hkv * s.N * s.D * 2;
+    HostLayout L;
+    L.count = 0;
+    L.index = L.count + up(T * 4);
+    L.full = L.index + up(T * T * 4);
+    L.q = L.full + up(T * T);
+    L.k = L.q + up(qb);
+    L.v = L.k + up(kvb);
+    L.o = L.v + up(kvb);
+    L.lse = L.o + up(qb);
+    L.total = L.lse + up(size_t(s.B) * s.Hq * s.N * 4);
+    return L;
+}
+
+// Per device: the streams the chunks' copies and kernels run on, and the
+// events that order them (created on first use, kept until exit).
+struct HostStreams {
+    cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, done = nullptr;
+    cudaEvent_t landed[kHostChunks] = {}, computed[kHostChunks] = {};
+};
+HostStreams g_host[kMaxDevices];
+std::mutex g_host_mu[kMaxDevices];
+
+int host_streams(int dev, HostStreams** out)
+{
+    HostStreams& h = g_host[dev];
+    if (!h.in) {
+        const unsigned ef = cudaEventDisableTiming;
+        if (cudaStreamCreateWithFlags(&h.comp, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&h.start, ef) != cudaSuccess || cudaEventCreateWithFlags(&h.done, ef) != cudaSuccess)
+            return SA_ERR_CUDA;
+        for (int c = 0; c < kHostChunks; c++)
+            if (cudaEventCreateWithFlags(&h.landed[c], ef) != cudaSuccess ||
+                cudaEventCreateWithFlags(&h.computed[c], ef) != cudaSuccess)
+                return SA_ERR_CUDA;
+        if (cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking) != cudaSuccess) return SA_ERR_CUDA;
+    }
+    *out = &h;
+    return SA_OK;
+}
+
+}  // namespace
+}  // namespace sa
+
 extern "C" int sparse_attn_fwd_host_workspace(const sa_shape* shape, size_t* bytes)
 {
     if (!shape || !bytes) return SA_ERR_INVALID_ARG;
     const sa_shape s = *shape;
     if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
-    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-    const size_t q = size_t(s.B) * s.Hq * s.N * s.D * 2;
-    const size_t kv = size_t(s.B) * s.Hkv * s.N * s.D * 2;
-    const size_t lse = size_t(s.B) * s.Hq * s.N * 4;
-    *bytes = up(q) + 2 * up(kv) + up(q) + up(lse);
+    *bytes = sa::host_layout(s).total;
     return SA_OK;
 }
 
 extern "C" int sparse_attn_fwd_host(const void* Q_host, const void* K_host, const void* V_host,
-                                    const sa_block_mask* mask, const sa_pattern* pattern, const sa_shape* shape,
+                                    const sa_block_mask* mask_host, const sa_pattern* pattern, const sa_shape* shape,
                                     float scale, void* O_host, float* LSE_host, void* workspace,
                                     size_t workspace_bytes, void* stream)
 {
-    if (!shape || !mask || !pattern) return SA_ERR_INVALID_ARG;
-    size_t need = 0;
-    if (int rc = sparse_attn_fwd_host_workspace(shape, &need)) return rc;
+    if (!shape || !mask_host || !pattern) return SA_ERR_INVALID_ARG;
     const sa_shape s = *shape;
+    if (s.B < 0 || s.Hq < 0 || s.Hkv < 0 || s.N < 0 || s.D <= 0) return SA_ERR_INVALID_ARG;
     if (s.B == 0 || s.Hq == 0 || s.N == 0) return SA_OK;
+    if (s.Hkv <= 0 || s.Hq % s.Hkv != 0) return SA_ERR_UNSUPPORTED;
+    if (mask_host->block != 64 && mask_host->block != 128) return SA_ERR_UNSUPPORTED;
+    const int64_t T = (int64_t(s.N) + mask_host->block - 1) / mask_host->block;
+    if (mask_host->n_q_tiles != T || mask_host->n_kv_tiles != T) return SA_ERR_MASK_MISMATCH;
+    if (int rc = sa::check_host_mask(mask_host, T)) return rc;
     if (!Q_host || !K_host || !V_host || !O_host || !LSE_host || !workspace) return SA_ERR_INVALID_ARG;
-    if (workspace_bytes < need) return SA_ERR_BUFFER_TOO_SMALL;
+    const sa::HostLayout L = sa::host_layout(s);
+    if (workspace_bytes < L.total) return SA_ERR_BUFFER_TOO_SMALL;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SA_ERR_MISALIGNED;
-    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-    const size_t qb = size_t(s.B) * s.Hq * s.N * s.D * 2;
-    const size_t kvb = size_t(s.B) * s.Hkv * s.N * s.D * 2;
-    const size_t lseb = size_t(s.B) * s.Hq * s.N * 4;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= sa::kMaxDevices) return SA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(sa::g_host_mu[dev]);
+    sa::HostStreams* hs = nullptr;
+    if (int rc = sa::host_streams(dev, &hs)) return rc;
+    // the status word exists before any chunk is queued (its first use waits for the device)
+    int32_t* status = nullptr;
+    if (int rc = sa::status_word(&status)) return rc;
+
     uint8_t* w = static_cast<uint8_t*>(workspace);
-    void* dQ = w;
-    void* dK = w + up(qb);
-    void* dV = w + up(qb) + up(kvb);
-    void* dO = w + up(qb) + 2 * up(kvb);
-    float* dL = reinterpret_cast<float*>(w + 2 * up(qb) + 2 * up(kvb));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (cudaMemcpyAsync(dQ, Q_host, qb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dK, K_host, kvb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dV, V_host, kvb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    // everything queued before this call on the caller's stream comes first
+    if (cudaEventRecord(hs->start, st) != cudaSuccess || cudaStreamWaitEvent(hs->in, hs->start, 0) != cudaSuccess)
         return SA_ERR_CUDA;
-    if (int rc = sparse_attn_fwd(dQ, dK, dV, mask, pattern, shape, scale, dO, dL, stream)) return rc;
-    if (cudaMemcpyAsync(O_host, dO, qb, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-        cudaMemcpyAsync(LSE_host, dL, lseb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    sa_block_mask dmask = *mask_host;
+    dmask.kv_count = reinterpret_cast<int32_t*>(w + L.count);
+    dmask.kv_index = reinterpret_cast<int32_t*>(w + L.index);
+    dmask.kv_full = w + L.full;
+    if (cudaMemcpyAsync(dmask.kv_count, mask_host->kv_count, size_t(T) * 4, cudaMemcpyHostToDevice, hs->in) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(dmask.kv_index, mask_host->kv_index, size_t(T) * T * 4, cudaMemcpyHostToDevice, hs->in) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(dmask.kv_full, mask_host->kv_full, size_t(T) * T, cudaMemcpyHostToDevice, hs->in) !=
+            cudaSuccess)
+        return SA_ERR_CUDA;
+
+    const int64_t heads = int64_t(s.B) * s.Hkv;  // flattened kv heads
+    const int64_t group = s.Hq / s.Hkv;
+    const int n_chunks = static_cast<int>(heads < sa::kHostChunks ? heads : sa::kHostChunks);
+    const size_t qh = size_t(s.N) * s.D * 2, lh = size_t(s.N) * 4;  // bytes of one head of Q (K, V, O) and LSE
+    auto chunk_heads = [&](int c, int64_t& h0, int64_t& h1) {
+        h0 = heads * c / n_chunks;
+        h1 = heads * (c + 1) / n_chunks;
+    };
+    auto at = [](const void* p, size_t off) { return static_cast<const uint8_t*>(p) + off; };
+    // every chunk's inputs first: the copy engine streams them back to back
+    // while the host queues the kernels and the copies back
+    for (int c = 0; c < n_chunks; c++) {
+        int64_t h0, h1;
+        chunk_heads(c, h0, h1);
+        const size_t kv_off = size_t(h0) * qh, kv_len = size_t(h1 - h0) * qh;
+        const size_t q_off = kv_off * group, q_len = kv_len * group;
+        if (cudaMemcpyAsync(w + L.q + q_off, at(Q_host, q_off), q_len, cudaMemcpyHostToDevice, hs->in) !=
+                cudaSuccess ||
+            cudaMemcpyAsync(w + L.k + kv_off, at(K_host, kv_off), kv_len, cudaMemcpyHostToDevice, hs->in) !=
+                cudaSuccess ||
+            cudaMemcpyAsync(w + L.v + kv_off, at(V_host, kv_off), kv_len, cudaMemcpyHostToDevice, hs->in) !=
+                cudaSuccess ||
+            cudaEventRecord(hs->landed[c], hs->in) != cudaSuccess)
+            return SA_ERR_CUDA;
+    }
+    for (int c = 0; c < n_chunks; c++) {
+        int64_t h0, h1;
+        chunk_heads(c, h0, h1);
+        const size_t kv_off = size_t(h0) * qh, q_off = kv_off * group, q_len = size_t(h1 - h0) * qh * group;
+        const size_t l_off = size_t(h0) * group * lh, l_len = size_t(h1 - h0) * group * lh;
+        if (cudaStreamWaitEvent(hs->comp, hs->landed[c], 0) != cudaSuccess) return SA_ERR_CUDA;
+        // the chunk as a batch of one: its kv heads and their query heads
+        sa_shape cs = s;
+        cs.B = 1;
+        cs.Hkv = static_cast<int32_t>(h1 - h0);
+        cs.Hq = static_cast<int32_t>((h1 - h0) * group);
+        if (int rc = sparse_attn_fwd(w + L.q + q_off, w + L.k + kv_off, w + L.v + kv_off, &dmask, pattern, &cs, scale,
+                                     w + L.o + q_off, reinterpret_cast<float*>(w + L.lse + l_off), hs->comp))
+            return rc;
+        if (cudaEventRecord(hs->computed[c], hs->comp) != cudaSuccess ||
+            cudaStreamWaitEvent(hs->out, hs->computed[c], 0) != cudaSuccess ||
+            cudaMemcpyAsync(static_cast<uint8_t*>(O_host) + q_off, w + L.o + q_off, q_len, cudaMemcpyDeviceToHost,
+                            hs->out) != cudaSuccess ||
+            cudaMemcpyAsync(reinterpret_cast<uint8_t*>(LSE_host) + l_off, w + L.lse + l_off, l_len,
+                            cudaMemcpyDeviceToHost, hs->out) != cudaSuccess)
+            return SA_ERR_CUDA;
+    }
+    // the caller's stream continues after the last copy back
+    if (cudaEventRecord(hs->done, hs->out) != cudaSuccess || cudaStreamWaitEvent(st, hs->done, 0) != cudaSuccess)
         return SA_ERR_CUDA;
     return sparse_attn_check_device(stream);
 }
@@ -488,4 +640,4 @@ extern "C" const char* sparse_attn_status_string(int status)
     }
 }
 
-extern "C" int32_t sparse_attn_version(void) { return 201; }
+extern "C" int32_t sparse_attn_version(void) { return 300; }

@@ -28,6 +28,7 @@
 
 #include "../../include/sparse_attn.h"
 #include "fwd_sm100.cuh"
+#include "runtime.h"
 #include "tma_host.h"
 
 namespace sa {
@@ -96,9 +97,10 @@ extern "C" int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void*
     const int64_t T = (int64_t(s.N) + mask->block - 1) / mask->block;
     if (mask->n_q_tiles != T || mask->n_kv_tiles != T) return SA_ERR_MASK_MISMATCH;
     if (scratch_bytes(T) > SA_NOALLOC_SCRATCH_BYTES) return SA_ERR_SCRATCH_TOO_SMALL;
-    if (!Q || !K || !V || !O || !LSE || !mask->kv_count || !mask->kv_index || !mask->kv_full)
-        return SA_ERR_INVALID_ARG;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    if (!Q || !K || !V || !O || !LSE) return SA_ERR_INVALID_ARG;
+    // the mask is read on the host: a malformed one is refused before any device work
+    if (int rc = check_host_mask(mask, T)) return rc;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || (reinterpret_cast<uintptr_t>(LSE) & 3u))
         return SA_ERR_MISALIGNED;
     const int64_t n_qtiles = (int64_t(s.N) + kBM - 1) / kBM;
     const int64_t group = s.Hq / s.Hkv;
@@ -166,8 +168,8 @@ extern "C" int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void*
     p.O = static_cast<__nv_bfloat16*>(O);
     p.LSE = LSE;
     p.status = status;
-    p.timeout = 2000000000LL;
-    p.debug_flags = 0;
+    p.timeout = wait_limit_cycles();
+    p.debug_flags = debug_flags() & 1;  // the skip-Q-load test hook; work units are never split here
     const int grid = static_cast<int>(n_items < n_sm ? n_items : n_sm);
     int rc;
     if (s.D == 128 && bn == 128)

@@ -527,16 +527,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int grp_s = MULTI ? hp.grp_s : 0;
     auto load_rows = [grp_n](void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int r0, int plane,
                              uint64_t pol) {
-        if (MULTI && grp_n > 0)
-            tma_load_4d(dst, map, bar, c0, r0 / grp_n, r0 % grp_n, plane, pol);
-        else
-            tma_load_3d(dst, map, bar, c0, r0, plane, pol);
+        if constexpr (MULTI) {
+            if (grp_n > 0) {
+                tma_load_4d(dst, map, bar, c0, r0 / grp_n, r0 % grp_n, plane, pol);
+                return;
+            }
+        }
+        tma_load_3d(dst, map, bar, c0, r0, plane, pol);
     };
     auto store_rows = [grp_n](const CUtensorMap* map, const void* src, int c0, int r0, int plane) {
-        if (MULTI && grp_n > 0)
-            tma_store_4d(map, src, c0, r0 / grp_n, r0 % grp_n, plane);
-        else
-            tma_store_3d(map, src, c0, r0, plane);
+        if constexpr (MULTI) {
+            if (grp_n > 0) {
+                tma_store_4d(map, src, c0, r0 / grp_n, r0 % grp_n, plane);
+                return;
+            }
+        }
+        tma_store_3d(map, src, c0, r0, plane);
     };
     // warp-uniform warpgroup index, so that the register split applies per branch
     const int wg = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x) / 128, 0);

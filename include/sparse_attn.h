@@ -130,14 +130,21 @@ int sparse_attn_build_block_mask(const sa_pattern* pattern, int64_t N, int32_t b
 int sparse_attn_count_pairs(const sa_pattern* pattern, int64_t N, int64_t* pairs);
 
 /*
- * Forward pass on the GPU.  Q, K, V, O, LSE are device pointers (16-byte
- * aligned) in the layouts above; `mask` holds DEVICE copies of the arrays
+ * Forward pass on the GPU.  Q, K, V, O, LSE are device pointers (Q, K, V, O
+ * 16-byte aligned, LSE 4-byte aligned) in the layouts above; `mask` holds DEVICE copies of the arrays
  * built by sparse_attn_build_block_mask for this pattern, N and block (its
  * scalar fields as the builder returned them).  scale > 0 multiplies q.k
  * (1/sqrt(D) in the pages' prototype).  `stream` is a cudaStream_t (NULL: the
  * legacy default stream).  Asynchronous: returns once the kernel is queued;
  * launch errors come back as SA_ERR_CUDA, a device-side timeout through
  * sparse_attn_check_device.  Rows with no allowed key get O = 0, LSE = -inf.
+ * The first call on a device (of this or any other entry point that reports
+ * through the status word) allocates the 4-byte device status word with
+ * cudaMalloc and clears it, waiting for the device: that one call blocks the
+ * host; later calls do not.  The kernels clamp a row's count to T and never
+ * address a tile outside [0, T), whatever the device mask holds: a malformed
+ * mask gives wrong results, not out-of-range accesses.  Results of the same
+ * call on the same inputs are bit-identical.
  * Supported: D in {64, 128}, mask block in {64, 128}, Hq % Hkv == 0, the
  * pattern forms listed at sa_pattern, at most 4096 tiles per side (N <= 4096 *
  * block); else SA_ERR_UNSUPPORTED.  Patterns with causal == 0 or area > 0 run
@@ -149,14 +156,25 @@ int sparse_attn_fwd(const void* Q, const void* K, const void* V, const sa_block_
                     void* stream);
 
 /*
- * The same forward pass from HOST buffers: copies Q, K, V from host memory
- * into `workspace` (device memory, at least sparse_attn_fwd_host_workspace
- * bytes, 256-byte aligned), runs sparse_attn_fwd on `stream`, copies O and LSE
- * back to host memory and waits for the stream.  Pinned host memory makes the
- * copies asynchronous DMA.  `mask` is the device-resident block mask.
- * Returns the first error, including a device timeout.
+ * The same forward pass from HOST buffers: Q, K, V, O, LSE and the block mask
+ * (`mask_host`, the arrays as sparse_attn_build_block_mask returned them) are
+ * all in host memory.  The mask is checked on the host first (counts in
+ * [0, T], listed tiles strictly ascending in [0, T), flags 0 or 1; else
+ * SA_ERR_INVALID_ARG, before any device work) and copied into `workspace`
+ * (device memory, at least sparse_attn_fwd_host_workspace bytes, 256-byte
+ * aligned).  The work is cut into up to 16 chunks of whole key/value heads
+ * (with their query heads); chunk c + 1's inputs are copied in while chunk c
+ * computes and chunk c - 1's O and LSE are copied back, on streams the library
+ * creates once per device, ordered after the work already queued on `stream`.
+ * Returns when everything is back in host memory (`stream` then waits on it
+ * too), with the first error, including a device timeout.  Pinned host memory
+ * makes the copies asynchronous DMA; pageable memory works but serialises
+ * them.  Each chunk is a sparse_attn_fwd call on its heads: results are those
+ * of sparse_attn_fwd, bit-identical when neither call splits work units (the
+ * kernel splits units only when they fill its last round of CTAs unevenly).
+ * Calls on one device are serialised.
  */
-int sparse_attn_fwd_host(const void* Q_host, const void* K_host, const void* V_host, const sa_block_mask* mask,
+int sparse_attn_fwd_host(const void* Q_host, const void* K_host, const void* V_host, const sa_block_mask* mask_host,
                          const sa_pattern* pattern, const sa_shape* shape, float scale, void* O_host,
                          float* LSE_host, void* workspace, size_t workspace_bytes, void* stream);
 
@@ -184,7 +202,9 @@ int sparse_attn_fwd_heads(const void* Q, const void* K, const void* V, const sa_
                           const sa_pattern* patterns, int32_t n_patterns, const int32_t* head_pattern,
                           const sa_shape* shape, float scale, void* O, float* LSE, void* stream);
 
-/* Device bytes sparse_attn_fwd_host needs for `shape`. */
+/* Device bytes sparse_attn_fwd_host needs for `shape`: Q, K, V, O, LSE and a
+ * copy of a block mask of ceil(N / 64) tiles per side, each rounded up to 256
+ * bytes. */
 int sparse_attn_fwd_host_workspace(const sa_shape* shape, size_t* bytes);
 
 /*
@@ -195,9 +215,9 @@ int sparse_attn_fwd_host_workspace(const sa_shape* shape, size_t* bytes);
 int sparse_attn_check_device(void* stream);
 
 /*
- * Test hook.  flags: bit 0 makes the next forward launches skip the Q tile
- * load, so the kernel's bounded waits expire and it reports
- * SA_ERR_DEVICE_TIMEOUT instead of computing.  Bit 1 makes sparse_attn_fwd
+ * Test hook.  flags: bit 0 makes the next forward launches (of every forward
+ * entry point) skip the Q tile load, so the kernel's bounded waits expire and
+ * it reports SA_ERR_DEVICE_TIMEOUT instead of computing.  Bit 1 makes sparse_attn_fwd
  * split every work unit (each query tile's kv list walked in two halves that
  * are merged at the end), the path the kernel otherwise takes only for the
  * last, partial round of units; results agree within rounding.
@@ -216,21 +236,28 @@ int sparse_attn_set_debug(int32_t flags, int64_t timeout_cycles);
  * mask from device memory the caller allocated; this call does neither.
  *
  * Arguments as sparse_attn_fwd, except that `mask` holds the HOST arrays
- * returned by sparse_attn_build_block_mask.  Its scratch, the kernel's status
- * word and a device copy of the mask, lives in one static device array of
+ * returned by sparse_attn_build_block_mask, and that only the causal forms are
+ * taken (causal == 1 with window, sinks, stride and n_global; causal == 0,
+ * area > 0 or summary > 0 give SA_ERR_UNSUPPORTED).  The mask is checked on
+ * the host before any device work, as for sparse_attn_fwd_host
+ * (SA_ERR_INVALID_ARG).  Its scratch, the kernel's status word and a device
+ * copy of the mask, lives in one static device array of
  * SA_NOALLOC_SCRATCH_BYTES that the library holds on every GPU that loads it
  * until the process exits.  A mask that does not fit (with 256 bytes for the
  * status word, 4 T + 5 T^2 bytes for T tiles per side: T <= 457) is rejected
- * with SA_ERR_SCRATCH_TOO_SMALL before any device work.
+ * with SA_ERR_SCRATCH_TOO_SMALL before any device work.  The wait limit and
+ * the skip-Q-load hook of sparse_attn_set_debug apply here too.
  *
  * The first call on a device looks up the array's device address with that
- * device current; make it before any stream capture.  Every call clears the
- * status word, copies the mask, launches on `stream`, then waits for the
- * stream and returns the device status (SA_ERR_DEVICE_TIMEOUT if a bounded
- * wait expired).  All calls share the array and it keeps the last call's
- * contents; calls whose kernels overlap on the GPU race on it (calls from
- * several host threads are serialised per device).  Calls no cudaMalloc,
- * cudaFree or other allocating routine.
+ * device current.  Every call clears the status word, copies the mask from
+ * host memory, launches on `stream`, copies the status word back into host
+ * memory and waits for the stream, then returns the device status
+ * (SA_ERR_DEVICE_TIMEOUT if a bounded wait expired): a call therefore cannot
+ * be made while `stream` is being captured into a CUDA graph.  All calls
+ * share the array and it keeps the last call's contents; calls whose kernels
+ * overlap on the GPU race on it (calls from several host threads are
+ * serialised per device).  Calls no cudaMalloc, cudaFree or other allocating
+ * routine.
  */
 #define SA_NOALLOC_SCRATCH_BYTES (1u << 20)
 int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void* V, const sa_block_mask* mask_host,

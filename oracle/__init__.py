@@ -77,6 +77,8 @@ class Oracle:
         L.oracle_allowed.restype = ctypes.c_int
         L.oracle_count_pairs.argtypes = [P, ctypes.c_int64]
         L.oracle_count_pairs.restype = ctypes.c_int64
+        L.oracle_row_counts.argtypes = [P, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
+        L.oracle_row_counts.restype = ctypes.c_int
         L.oracle_block_mask.argtypes = [P, ctypes.c_int64, ctypes.c_int32,
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         L.oracle_block_mask.restype = ctypes.c_int64
@@ -103,6 +105,15 @@ class Oracle:
 
     def count_pairs(self, p: Pattern, N: int) -> int:
         return int(self.L.oracle_count_pairs(ctypes.byref(p.c()), N))
+
+    def row_counts(self, p: Pattern, N: int, rows) -> np.ndarray:
+        """Allowed keys of each of the given query rows (brute force per row)."""
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        out = np.zeros(len(rows), dtype=np.int64)
+        if len(rows) and self.L.oracle_row_counts(ctypes.byref(p.c()), N, rows.ctypes.data, len(rows),
+                                                  out.ctypes.data) != 0:
+            raise ValueError("row outside [0, N)")
+        return out
 
     def block_mask(self, p: Pattern, N: int, block: int):
         """Brute-force tile classification -> (counts[T], index[T, T], full[T, T])."""
@@ -199,6 +210,10 @@ def allowed(p: Pattern, q: int, kv: int) -> bool:
 
 def count_pairs(p: Pattern, N: int) -> int:
     return default().count_pairs(p, N)
+
+
+def row_counts(p: Pattern, N: int, rows) -> np.ndarray:
+    return default().row_counts(p, N, rows)
 
 
 def block_mask(p: Pattern, N: int, block: int):

@@ -98,6 +98,22 @@ int oracle_allowed(const oracle_pattern *p, int64_t q, int64_t kv)
     return 0;
 }
 
+/* Allowed keys of each listed query row, 0 <= kv < N, counted one by one. */
+int oracle_row_counts(const oracle_pattern *p, int64_t N, const int64_t *rows, int64_t n_rows, int64_t *out)
+{
+    for (int64_t r = 0; r < n_rows; r++)
+        if (rows[r] < 0 || rows[r] >= N)
+            return -1;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t r = 0; r < n_rows; r++) {
+        int64_t c = 0;
+        for (int64_t kv = 0; kv < N; kv++)
+            c += oracle_allowed(p, rows[r], kv) == 1;
+        out[r] = c;
+    }
+    return 0;
+}
+
 /* Number of allowed (q, kv) pairs with 0 <= q, kv < N, counted one by one. */
 int64_t oracle_count_pairs(const oracle_pattern *p, int64_t N)
 {

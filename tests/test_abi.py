@@ -378,3 +378,65 @@ def test_bwd_heads_argument_errors_without_gpu():
                                       (sa._Pattern * 1)(p), 1, None, ctypes.byref(sa._Shape(1, 2, 2, 100, 128)),
                                       0.125, fake, fake, fake, fake, ws, None)
     assert rc == sa.SA_ERR_INVALID_ARG
+
+
+def _malformed_masks(N=1000, block=128):
+    """A well-formed host mask and variants that break one rule each."""
+    good = sa.build_block_mask(sa.Pattern(window=300, sinks=4), N, block)
+
+    def variant(edit):
+        c, i, f = good.counts.copy(), good.index.copy(), good.full.copy()
+        edit(c, i, f)
+        return sa.BlockMask(c, i, f, good.block, good.n_live, good.n_full, good.max_per_row, N)
+
+    T = good.T
+    bad = {
+        "count above T": variant(lambda c, i, f: c.__setitem__(2, T + 1)),
+        "negative count": variant(lambda c, i, f: c.__setitem__(3, -1)),
+        "index past T": variant(lambda c, i, f: i.__setitem__((5, c[5] - 1), T)),
+        "negative index": variant(lambda c, i, f: i.__setitem__((4, 0), -1)),
+        "not ascending": variant(lambda c, i, f: i.__setitem__((6, 1), i[6, 0])),
+        "flag not 0 or 1": variant(lambda c, i, f: f.__setitem__((7, 0), 2)),
+    }
+    return good, bad
+
+
+def test_host_mask_checked_before_device_work():
+    """sparse_attn_fwd_host and sparse_attn_fwd_noalloc read the block mask on
+    the host: a malformed one comes back as SA_ERR_INVALID_ARG before any CUDA
+    call (the tensor pointers below are never dereferenced)."""
+    N, D = 1000, 128
+    good, bad = _malformed_masks(N)
+    p = sa.Pattern(window=300, sinks=4)._c()
+    shape = sa._Shape(1, 2, 2, N, D)
+    fake = 1 << 20
+    ws = ctypes.c_size_t(0)
+    assert sa.lib.sparse_attn_fwd_host_workspace(ctypes.byref(shape), ctypes.byref(ws)) == 0
+    for name, m in bad.items():
+        cm = m._c()
+        rc = sa.lib.sparse_attn_fwd_host(fake, fake, fake, ctypes.byref(cm), ctypes.byref(p), ctypes.byref(shape),
+                                         0.088, fake, fake, fake, ws.value, None)
+        assert rc == sa.SA_ERR_INVALID_ARG, (name, rc)
+        rc = sa.lib.sparse_attn_fwd_noalloc(fake, fake, fake, ctypes.byref(cm), ctypes.byref(p), ctypes.byref(shape),
+                                            0.088, fake, fake, None)
+        assert rc == sa.SA_ERR_INVALID_ARG, (name, rc)
+    # a short workspace and a misplaced mask are refused the same way
+    cm = good._c()
+    rc = sa.lib.sparse_attn_fwd_host(fake, fake, fake, ctypes.byref(cm), ctypes.byref(p), ctypes.byref(shape), 0.088,
+                                     fake, fake, fake, ws.value - 1, None)
+    assert rc == sa.SA_ERR_BUFFER_TOO_SMALL
+    other = sa.build_block_mask(sa.Pattern(window=300, sinks=4), 2 * N, 128)._c()
+    rc = sa.lib.sparse_attn_fwd_host(fake, fake, fake, ctypes.byref(other), ctypes.byref(p), ctypes.byref(shape),
+                                     0.088, fake, fake, fake, ws.value, None)
+    assert rc == sa.SA_ERR_MASK_MISMATCH
+
+
+def test_host_workspace_covers_the_mask_copy():
+    """The host-buffer workspace holds Q, K, V, O, LSE and a copy of a mask of
+    ceil(N / 64) tiles per side."""
+    B, Hq, Hkv, N, D = 2, 4, 2, 1000, 64
+    ws = ctypes.c_size_t(0)
+    assert sa.lib.sparse_attn_fwd_host_workspace(ctypes.byref(sa._Shape(B, Hq, Hkv, N, D)), ctypes.byref(ws)) == 0
+    T = -(-N // 64)
+    need = 2 * B * Hq * N * D * 2 + 2 * B * Hkv * N * D * 2 + B * Hq * N * 4 + T * 4 + 5 * T * T
+    assert need <= ws.value <= need + 8 * 256

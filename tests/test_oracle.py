@@ -288,3 +288,56 @@ def test_generator_statistics_and_determinism():
     assert abs((np.abs(x) < 1).mean() - 0.6827) < 3e-3
     c = synth.normal_bf16((1 << 20,), 0, 1)
     assert not np.array_equal(a, c)
+
+
+# ----------------------------------------------------------------------------
+# The other reading of global rows ("global tokens attend to every position",
+# without the causal conjunction): `global_rows_see_all`.  Pinned by closed
+# forms, not by a restatement of the rule.
+
+def closed_row_count_see_all(q, N, l, s, G):
+    """|A(q)| when rows q < G see all N keys; other rows as closed_row_count_strided."""
+    return N if q < G else closed_row_count_strided(q, l, s, G)
+
+
+@pytest.mark.parametrize("N,l,s,G", [(16384, 128, 128, 16), (300, 10, 7, 5), (64, 3, 5, 9), (50, -1, 4, 50)])
+def test_global_rows_see_all_pair_count_closed_form(N, l, s, G):
+    p = Pattern(window=l, stride=s, n_global=G, global_rows_see_all=1)
+    want = sum(closed_row_count_see_all(q, N, l, s, G) for q in range(N))
+    assert oracle.count_pairs(p, N) == want
+    # the two readings differ by the keys after each global row: sum_{q < G} (N - 1 - q)
+    causal = oracle.count_pairs(Pattern(window=l, stride=s, n_global=G), N)
+    g = min(G, N)
+    assert want - causal == g * (N - 1) - g * (g - 1) // 2
+
+
+def test_global_rows_see_all_strided_global_workload_count():
+    # the strided + global workload (N = 16384, local 128, stride 128, 16 global
+    # tokens) under this reading: 3 387 352 causal pairs plus 16 * 16383 - 120
+    assert oracle.count_pairs(Pattern(window=128, stride=128, n_global=16, global_rows_see_all=1),
+                              16384) == 3_387_352 + 16 * 16383 - 120
+
+
+def test_global_rows_see_all_zero_query_gives_log_count_and_mean():
+    # Q = 0: LSE = ln |A(q)| (ln N on a global row) and O = the mean of V over A(q)
+    N, D, l, s, G = 240, 8, 12, 9, 5
+    q = np.zeros((1, 2, N, D), dtype=np.uint16)
+    _, k, v = synth.qkv(1, 2, 1, N, D, seed=31)
+    O, LSE = oracle.attention(q, k, v, Pattern(window=l, stride=s, n_global=G, global_rows_see_all=1), 0.7)
+    cnt = np.array([closed_row_count_see_all(r, N, l, s, G) for r in range(N)])
+    assert np.abs(LSE - np.log(cnt)[None, None]).max() < 1e-12
+    vf = synth.bf16_bits_to_float(v).astype(np.float64)
+    for r in range(G):  # a global row averages every key of the sequence
+        assert np.abs(O[:, :, r] - vf[:, :, :].mean(axis=2)).max() < 1e-12
+
+
+def test_row_counts_match_closed_forms():
+    # per-row brute force (the bench's CPU arms count their work with it) against the closed forms
+    N, w, s = 700, 40, 4
+    rows = np.array([0, 1, 39, 40, 41, 44, 45, 300, 699])
+    got = oracle.row_counts(Pattern(window=w, sinks=s), N, rows)
+    assert list(got) == [min(r, w) + 1 + min(s, max(0, r - w)) for r in rows]
+    got = oracle.row_counts(Pattern(window=10, stride=7, n_global=3), 300, np.arange(300))
+    assert list(got) == [closed_row_count_strided(r, 10, 7, 3) for r in range(300)]
+    assert oracle.row_counts(Pattern(window=10, stride=7, n_global=3), 300, np.arange(300)).sum() == \
+        oracle.count_pairs(Pattern(window=10, stride=7, n_global=3), 300)

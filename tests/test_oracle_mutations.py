@@ -28,6 +28,8 @@ MUTANTS = {
                       "bf16_to_double(kp[c]);\n                        s[t] = dot;"),
     "full_ignores_ragged": ("full[i * T + c] = allowed == (q1 - q0) * (k1 - k0);",
                             "full[i * T + c] = allowed == (int64_t)block * block;"),
+    "global_rows_causal_anyway": ("if (p->global_rows_see_all && q < p->n_global)\n        return 1;",
+                                  "if (p->global_rows_see_all && q < p->n_global)\n        return delta >= 0;"),
 }
 
 
@@ -65,6 +67,10 @@ def pins_hold(o: oracle.Oracle) -> bool:
     _, LSE = o.attention(q, k, v, Pattern(window=w, sinks=s), 0.5)
     cnt = np.array([min(r, w) + 1 + min(s, max(0, r - w)) for r in range(N)])
     if np.abs(LSE[0, 0] - np.log(cnt)).max() > 1e-12:
+        return False
+    # global rows under the reading that they see every key: closed-form count
+    if o.count_pairs(Pattern(window=10, stride=7, n_global=3, global_rows_see_all=1), 300) != 300 * 3 + sum(
+            closed_row_count_strided(q, 10, 7, 3) for q in range(3, 300)):
         return False
     # dense causal with GQA equals the library routine
     B, Hq, Hkv, N, D = 1, 4, 2, 64, 16

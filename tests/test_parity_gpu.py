@@ -154,18 +154,32 @@ def test_repeat_calls_are_deterministic():
     assert np.array_equal(O1, O2) and np.array_equal(L1, L2)
 
 
-def test_host_buffer_entry_point_matches_device_entry_point():
-    B, Hq, Hkv, N, D = 1, 4, 2, 1000, 128
+@pytest.mark.parametrize("B,Hq,Hkv,N,D,block,pinned", [
+    (1, 4, 2, 1000, 128, 128, True),   # 2 chunks of one kv head
+    (2, 6, 3, 777, 64, 64, True),      # 6 chunks across the batch, ragged, block 64
+    (3, 4, 4, 384, 128, 128, True),    # 12 kv heads in 8 chunks of one or two
+    (1, 2, 1, 640, 128, 128, False),   # pageable host memory, one chunk
+])
+def test_host_buffer_entry_point_matches_device_entry_point(B, Hq, Hkv, N, D, block, pinned):
+    """The host-buffer call (chunks of kv heads, copies overlapping the kernels)
+    gives the device call's output bit for bit (neither splits work units at
+    these sizes), and both agree with the oracle."""
     p = sa.Pattern(window=200, sinks=4)
     q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=21)
-    O, LSE = run_gpu(q, k, v, p, 128, 1 / math.sqrt(D))
-    mask = sa.build_block_mask(p, N, 128).to_device("cuda")
-    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
-    Oh = torch.empty((B, Hq, N, D), dtype=torch.bfloat16).pin_memory()
-    Lh = torch.empty((B, Hq, N), dtype=torch.float32).pin_memory()
+    O, LSE = run_gpu(q, k, v, p, block, 1 / math.sqrt(D))
+    mask = sa.build_block_mask(p, N, block)
+    host = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    pin = (lambda a: host(a).pin_memory()) if pinned else host
+    Oh = torch.full((B, Hq, N, D), float("nan"), dtype=torch.bfloat16)
+    Lh = torch.full((B, Hq, N), float("nan"), dtype=torch.float32)
+    if pinned:
+        Oh, Lh = Oh.pin_memory(), Lh.pin_memory()
     ws = torch.empty(sa.fwd_host_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device="cuda")
-    sa.fwd_host(pin(q), pin(k), pin(v), mask, p, Oh, Lh, ws)
-    assert np.array_equal(Oh.float().numpy(), O) and np.array_equal(Lh.numpy(), LSE)
+    for _ in range(2):  # a second call on the same streams and workspace
+        sa.fwd_host(pin(q), pin(k), pin(v), mask, p, Oh, Lh, ws)
+        assert np.array_equal(Oh.float().numpy(), O) and np.array_equal(Lh.numpy(), LSE)
+    Oref, Lref = oracle.attention(q, k, v, oracle.Pattern(window=200, sinks=4), 1 / math.sqrt(D))
+    compare(Oh.float().numpy(), Lh.numpy(), Oref, Lref)
 
 
 def test_device_timeout_is_reported_and_context_survives():

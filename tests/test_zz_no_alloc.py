@@ -5,9 +5,11 @@ must not call cudaMalloc on the request path).
 It runs the same kernel as sparse_attn_fwd, with the kernel's scratch (status
 word, device copy of the block mask) in a static device array of the library.
 Checked here through the C ABI: two calls in a row, with different shapes and
-patterns so the shared scratch is rewritten, each against sparse_attn_fwd on
-the same inputs, within the tolerance the parity tests use.  This file is
-collected last so that a stop at the first failure has run everything else.
+patterns so the shared scratch is rewritten, each bit for bit against
+sparse_attn_fwd on the same inputs and within the parity bars against the
+oracle; and a device timeout reported through the static status word.  This
+file is collected last so that a stop at the first failure has run everything
+else.
 """
 import ctypes
 import math
@@ -35,9 +37,23 @@ def test_mask_larger_than_scratch_is_rejected_before_device_work():
     assert "static scratch" in sa.status_string(rc)
 
 
+def _noalloc(q, k, v, host_mask, p, scale, O, L):
+    import torch
+    B, Hq, N, D = q.shape
+    shape = sa._Shape(B, Hq, k.shape[1], N, D)
+    return sa.lib.sparse_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(host_mask._c()),
+                                          ctypes.byref(p._c()), ctypes.byref(shape), scale, O.data_ptr(), L.data_ptr(),
+                                          torch.cuda.current_stream().cuda_stream)
+
+
 @pytest.mark.gpu
 def test_noalloc_matches_fwd_on_two_calls_in_a_row():
+    """Both entry points run the same kernel on the same inputs with the same
+    work plan, so their outputs agree bit for bit; the no-allocation output is
+    also checked against the fp64 oracle at the parity bars."""
     import torch
+
+    import oracle
 
     cases = [
         # (B, Hq, Hkv, N, D, pattern, block): ragged tail and GQA, then a strided pattern on 64-wide tiles
@@ -46,7 +62,8 @@ def test_noalloc_matches_fwd_on_two_calls_in_a_row():
     ]
     dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
     for i, (B, Hq, Hkv, N, D, p, block) in enumerate(cases):
-        q, k, v = (dev(a) for a in synth.qkv(B, Hq, Hkv, N, D, seed=100 + i))
+        qh, kh, vh = synth.qkv(B, Hq, Hkv, N, D, seed=100 + i)
+        q, k, v = dev(qh), dev(kh), dev(vh)
         scale = 1 / math.sqrt(D)
         host_mask = sa.build_block_mask(p, N, block)
 
@@ -55,12 +72,37 @@ def test_noalloc_matches_fwd_on_two_calls_in_a_row():
 
         O = torch.full_like(q, float("nan"))
         L = torch.full((B, Hq, N), float("nan"), dtype=torch.float32, device="cuda")
-        shape = sa._Shape(B, Hq, Hkv, N, D)
-        rc = sa.lib.sparse_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                            ctypes.byref(host_mask._c()), ctypes.byref(p._c()),
-                                            ctypes.byref(shape), scale, O.data_ptr(), L.data_ptr(),
-                                            torch.cuda.current_stream().cuda_stream)
+        rc = _noalloc(q, k, v, host_mask, p, scale, O, L)
         assert rc == sa.SA_OK, sa.status_string(rc)
-        o_err = (O.float() - O_ref.float()).abs().max().item()
-        l_err = (L - L_ref).abs().max().item()
+        assert torch.equal(O, O_ref) and torch.equal(L, L_ref), i
+
+        op = oracle.Pattern(window=p.window, sinks=p.sinks, stride=p.stride, n_global=p.n_global)
+        Oo, Lo = oracle.attention(qh, kh, vh, op, scale)
+        o_err = float(np.abs(O.float().cpu().numpy() - Oo).max())
+        l_err = float(np.abs(L.cpu().numpy() - Lo).max())
         assert o_err <= O_TOL and l_err <= LSE_TOL, (i, o_err, l_err)
+
+
+@pytest.mark.gpu
+def test_noalloc_reports_a_device_timeout_and_recovers():
+    """The wait limit and the skip-Q-load hook of sparse_attn_set_debug apply:
+    the kernel's bounded waits expire (about 10 ms each), the call returns
+    SA_ERR_DEVICE_TIMEOUT, and the next call on the same context is exact."""
+    import torch
+
+    B, Hq, Hkv, N, D = 1, 2, 2, 512, 128
+    p = sa.Pattern(window=128, sinks=4)
+    dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    q, k, v = (dev(a) for a in synth.qkv(B, Hq, Hkv, N, D, seed=7))
+    host_mask = sa.build_block_mask(p, N, 128)
+    O = torch.empty_like(q)
+    L = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    try:
+        sa.set_debug(sa.DEBUG_SKIP_Q_LOAD, 20_000_000)
+        assert _noalloc(q, k, v, host_mask, p, 1 / math.sqrt(D), O, L) == sa.SA_ERR_DEVICE_TIMEOUT
+    finally:
+        sa.set_debug(0, 0)
+    assert _noalloc(q, k, v, host_mask, p, 1 / math.sqrt(D), O, L) == sa.SA_OK
+    O_ref, L_ref = sa.fwd(q, k, v, host_mask.to_device("cuda"), p, scale=1 / math.sqrt(D))
+    assert sa.check_device() == sa.SA_OK
+    assert torch.equal(O, O_ref) and torch.equal(L, L_ref)
