@@ -452,8 +452,6 @@ def run_gpu_bwd(args, w):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
-    if w.block != 128:
-        raise SystemExit("the backward pass takes block-128 masks")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -462,9 +460,13 @@ def run_gpu_bwd(args, w):
 
     p, mask_h, pairs, _, _, _ = workload_counts(w)
     useful = 10.0 * w.D * pairs * w.B * w.Hq
-    executed = 10.0 * w.D * w.block * w.block * mask_h.n_live * w.B * w.Hq
     mask = mask_h.to_device(dev)
-    mask_t = sa.transpose_block_mask(mask_h).to_device(dev)
+    # The backward works on 128 x 128 tiles whatever tile the forward used: it
+    # takes the transposed block-128 mask of the same pattern (partial tiles are
+    # masked element by element from the rule, so the gradients are the same).
+    mask128 = mask_h if w.block == 128 else sa.build_block_mask(p, w.N, 128)
+    executed = 10.0 * w.D * 128 * 128 * mask128.n_live * w.B * w.Hq
+    mask_t = sa.transpose_block_mask(mask128).to_device(dev)
 
     seed = rank_seed(w, rank)
     q, k, v = synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=seed)
@@ -570,7 +572,7 @@ def run_gpu_bwd(args, w):
             "pass": "bwd",
             "l2": f"{n_sets} rotating input sets of {set_bytes / 1e6:.1f} MB "
                   f"({n_sets * set_bytes / 1e6:.0f} MB > {L2_BYTES / 1e6:.0f} MB L2)",
-            "live_tiles": int(mask_h.n_live), "allowed_pairs_per_head": int(pairs)}),
+            "live_tiles": int(mask128.n_live), "backward_tile": 128, "allowed_pairs_per_head": int(pairs)}),
         "useful_frac_of_peak": value / world / peak,
         "executed_tflops": job_tflops(world, executed, args.steps, elapsed_ms),
         "peak_kind": f"bf16 dense, {peak_kind} ({peak} TFLOP/s burst)",

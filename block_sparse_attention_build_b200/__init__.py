@@ -35,6 +35,7 @@ NOALLOC_SCRATCH_BYTES = 1 << 20
 
 DEBUG_SKIP_Q_LOAD = 1
 DEBUG_SPLIT_ALL = 2
+DEBUG_BWD_SPLIT = 4
 
 EXPORTED = (
     "sparse_attn_num_tiles", "sparse_attn_build_block_mask", "sparse_attn_count_pairs",

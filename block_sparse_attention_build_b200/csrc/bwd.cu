@@ -15,6 +15,7 @@ namespace sa {
 namespace {
 
 constexpr int kMaxDev = 64;
+constexpr int32_t kDebugBwdSplitShort = 4;  // sparse_attn_set_debug bit 2
 
 struct BwdLayout {
     size_t lse2, delta, dq, dk, dv, items, n_items, split, steps, total;  // byte offsets, each 256-aligned
@@ -110,6 +111,7 @@ int bwd_run(const void* Q, const void* K, const void* V, const void* O, const fl
     const int n_sm = device_sm_count();
     if (n_sm <= 0) return SA_ERR_CUDA;
     p.n_sm = n_sm;
+    p.split_short = (debug_flags() & kDebugBwdSplitShort) != 0;
     auto grid_for = [&](int64_t n) {
         int64_t g = (n + 255) / 256;
         if (g > int64_t(n_sm) * 8) g = int64_t(n_sm) * 8;

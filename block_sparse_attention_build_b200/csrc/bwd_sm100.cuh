@@ -105,6 +105,7 @@ struct BwdParams {
     long long timeout;       // SM cycles per bounded wait
     int32_t T, N, B, Hq, Hkv, group;
     int32_t n_sm;            // SMs of the device (the split length follows the per-SM share)
+    int32_t split_short;     // test hook: split every list longer than kBwdChunk steps
     float scale_log2;        // scale * log2(e)
     float scale;
 };
@@ -333,7 +334,8 @@ __global__ void __launch_bounds__(1024) bwd_items_kernel(const BwdParams p, cons
     block_exclusive_scan(my_steps, s_warp, &s_total);
     // split length: an SM's share of all steps (every batch entry), at least kBwdChunk
     const long long share = (s_total * p.B + p.n_sm - 1) / p.n_sm;
-    const int len_max = static_cast<int>(max(static_cast<long long>(kBwdChunk), min(share, 1LL << 30)));
+    const int len_max =
+        p.split_short ? kBwdChunk : static_cast<int>(max(static_cast<long long>(kBwdChunk), min(share, 1LL << 30)));
     int ns = 0, nu = 0;
     for (int idx = lo; idx < hi; idx++) {
         const int st = steps_of[idx];

@@ -220,7 +220,10 @@ int sparse_attn_check_device(void* stream);
  * it reports SA_ERR_DEVICE_TIMEOUT instead of computing.  Bit 1 makes sparse_attn_fwd
  * split every work unit (each query tile's kv list walked in two halves that
  * are merged at the end), the path the kernel otherwise takes only for the
- * last, partial round of units; results agree within rounding.
+ * last, partial round of units; results agree within rounding.  Bit 2 makes
+ * sparse_attn_bwd split every kv tile's list of more than 32 steps into work
+ * items of at most 32 steps whose dK, dV add up in fp32 sums, the path it
+ * otherwise takes only for lists longer than an SM's share of all steps.
  * timeout_cycles bounds every wait in SM clock cycles (<= 0 restores the
  * default, about one second).
  */

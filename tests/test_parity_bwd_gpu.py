@@ -69,6 +69,7 @@ def compare_grads(got, ref):
 
 CASES = [
     # (B, Hq, Hkv, N, D, pattern)
+    (1, 2, 2, 512, 64, sa.Pattern(window=128, sinks=4)),               # the tiny workload (its forward tiles are 64)
     (1, 2, 2, 512, 128, sa.Pattern(window=128, sinks=4)),
     (1, 2, 2, 1000, 128, sa.Pattern(window=300, sinks=4)),             # ragged tail
     (2, 4, 2, 777, 64, sa.Pattern(window=100, sinks=3)),               # GQA, D = 64, ragged
@@ -128,6 +129,50 @@ def test_bwd_headline_size_two_heads():
         sl = slice(h, h + 1)
         _, _, rq, rk, rv = oracle.attention_bwd(q[:, sl], k[:, sl], v[:, sl], do[:, sl], opattern(p), scale)
         compare_grads((dq[:, sl], dk[:, sl], dv[:, sl]), (rq, rk, rv))
+
+
+SPLIT_CASES = [
+    # lists longer than 32 steps, walked as several work items whose dK, dV
+    # add up in fp32 sums (forced by the test hook)
+    (1, 4, 2, 4096, 128, sa.Pattern(window=512, sinks=4)),    # the sink tile: 32 query tiles x 2 heads
+    (1, 2, 1, 4608, 64, sa.Pattern(window=4608)),             # dense causal: up to 36 x 2 steps per tile
+    (2, 8, 1, 1280, 128, sa.Pattern(window=256, sinks=8)),    # a group of 8 heads: 8 steps per query tile
+    (1, 2, 2, 4100, 128, sa.Pattern(window=-1, sinks=130, n_global=3)),  # two sink tiles, ragged tail
+]
+
+
+@pytest.mark.parametrize("case", SPLIT_CASES, ids=lambda c: f"B{c[0]}H{c[1]}/{c[2]}N{c[3]}D{c[4]}-{c[5]}")
+def test_bwd_split_items_parity(case):
+    B, Hq, Hkv, N, D, p = case
+    q, k, v, do = inputs(B, Hq, Hkv, N, D, seed=N + D + 17)
+    scale = 1 / math.sqrt(D)
+    mask_t = sa.transpose_block_mask(sa.build_block_mask(p, N, 128))
+    assert mask_t.counts.max() * (Hq // Hkv) > 32  # some list is long enough to split
+    try:
+        sa.set_debug(sa.DEBUG_BWD_SPLIT, 0)
+        got = run_gpu_bwd(q, k, v, do, p, scale)
+    finally:
+        sa.set_debug(0, 0)
+    _, _, dQ, dK, dV = oracle.attention_bwd(q, k, v, do, opattern(p), scale)
+    compare_grads(got, (dQ, dK, dV))
+
+
+def test_bwd_narrow_window_many_heads_full_size_two_kv_heads():
+    """The 16 384-token narrow-window workload with 64 query heads on 8 kv heads,
+    at full size: every query tile attends to the sink tile, so kv tile 0's list
+    (128 query tiles x 8 heads) is split across work items without any test
+    hook.  Two kv heads (their 16 query heads) are checked against the oracle."""
+    B, Hq, Hkv, N, D = 2, 64, 8, 16384, 64
+    p = sa.Pattern(window=128, sinks=4)
+    q, k, v, do = inputs(B, Hq, Hkv, N, D, seed=0)
+    scale = 1 / math.sqrt(D)
+    dq, dk, dv = run_gpu_bwd(q, k, v, do, p, scale)
+    group = Hq // Hkv
+    for b, hk in ((0, 0), (1, 5)):
+        sq, sk = slice(hk * group, (hk + 1) * group), slice(hk, hk + 1)
+        _, _, rq, rk, rv = oracle.attention_bwd(q[b:b + 1, sq], k[b:b + 1, sk], v[b:b + 1, sk], do[b:b + 1, sq],
+                                                opattern(p), scale)
+        compare_grads((dq[b:b + 1, sq], dk[b:b + 1, sk], dv[b:b + 1, sk]), (rq, rk, rv))
 
 
 HEAD_CASES = [
