@@ -436,8 +436,25 @@ namespace {
 // and head, index b * Hkv + h): a chunk's Q, K, V, O and LSE are one
 // contiguous byte range of each tensor, so each moves with one copy, and chunk
 // c + 1's inputs cross the bus while chunk c computes and chunk c - 1's
-// outputs come back.
+// outputs come back.  Chunks halve in size (half the heads, then half of the
+// rest, ...): few copies, and only the last, one-head chunk's outputs are
+// left to copy back once all inputs are in.
 constexpr int kHostChunks = 16;
+
+// Head boundaries of the chunks: first[0] = 0 < first[1] < ... < first[n] = heads.
+int host_chunks(int64_t heads, int64_t* first)
+{
+    int n = 0;
+    first[0] = 0;
+    int64_t done = 0;
+    while (done < heads) {
+        const int64_t rest = heads - done;
+        const int64_t take = (n == kHostChunks - 1) ? rest : (rest / 2 > 0 ? rest / 2 : 1);
+        done += take;
+        first[++n] = done;
+    }
+    return n;
+}
 
 struct HostLayout {
     size_t count, index, full, q, k, v, o, lse, total;  // byte offsets, each 256-aligned
@@ -549,11 +566,12 @@ extern "C" int sparse_attn_fwd_host(const void* Q_host, const void* K_host, cons
 
     const int64_t heads = int64_t(s.B) * s.Hkv;  // flattened kv heads
     const int64_t group = s.Hq / s.Hkv;
-    const int n_chunks = static_cast<int>(heads < sa::kHostChunks ? heads : sa::kHostChunks);
+    int64_t first[sa::kHostChunks + 1];
+    const int n_chunks = sa::host_chunks(heads, first);
     const size_t qh = size_t(s.N) * s.D * 2, lh = size_t(s.N) * 4;  // bytes of one head of Q (K, V, O) and LSE
     auto chunk_heads = [&](int c, int64_t& h0, int64_t& h1) {
-        h0 = heads * c / n_chunks;
-        h1 = heads * (c + 1) / n_chunks;
+        h0 = first[c];
+        h1 = first[c + 1];
     };
     auto at = [](const void* p, size_t off) { return static_cast<const uint8_t*>(p) + off; };
     // every chunk's inputs first: the copy engine streams them back to back

@@ -162,10 +162,11 @@ int sparse_attn_fwd(const void* Q, const void* K, const void* V, const sa_block_
  * [0, T], listed tiles strictly ascending in [0, T), flags 0 or 1; else
  * SA_ERR_INVALID_ARG, before any device work) and copied into `workspace`
  * (device memory, at least sparse_attn_fwd_host_workspace bytes, 256-byte
- * aligned).  The work is cut into up to 16 chunks of whole key/value heads
- * (with their query heads); chunk c + 1's inputs are copied in while chunk c
- * computes and chunk c - 1's O and LSE are copied back, on streams the library
- * creates once per device, ordered after the work already queued on `stream`.
+ * aligned).  The work is cut into chunks of whole key/value heads (with their
+ * query heads), each half of the heads still left (the last takes one, at
+ * most 16 chunks); chunk c + 1's inputs are copied in while chunk c computes
+ * and chunk c - 1's O and LSE are copied back, on streams the library creates
+ * once per device, ordered after the work already queued on `stream`.
  * Returns when everything is back in host memory (`stream` then waits on it
  * too), with the first error, including a device timeout.  Pinned host memory
  * makes the copies asynchronous DMA; pageable memory works but serialises
