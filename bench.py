@@ -32,7 +32,11 @@ step's device time.
 With --impl reference the oracle is the timed program (rank 0 only).
 Multi-GPU (torchrun): every rank runs its own batch of the workload (the
 problems are independent; no collective on the data path); value is the sum
-over ranks of the work divided by the slowest rank's time.
+over ranks of the work divided by the slowest rank's time ("scaling": "weak").
+With --shard heads the ranks split one workload instead: each takes a
+contiguous range of its batch x kv-head groups with their query heads, again
+with no collective on the data path; value is the workload's work over the
+slowest rank's time ("scaling": "strong").
 """
 from __future__ import annotations
 
@@ -264,6 +268,23 @@ def config_of(w, n_gpus, extra=None):
     return c
 
 
+def shard_heads(n_heads: int, world: int, rank: int):
+    """Rank's contiguous range [h0, h1) of the n_heads kv heads (flattened over
+    batch and head) when one workload is split across ranks."""
+    return n_heads * rank // world, n_heads * (rank + 1) // world
+
+
+def shard_inputs(q, k, v, B, Hq, Hkv, h0, h1):
+    """The rank's part of one workload's inputs: kv heads h0 .. h1 - 1 of the
+    flattened batch x head axis and their query heads, as a batch of one."""
+    g = Hq // Hkv
+    N, D = q.shape[2], q.shape[3]
+    qs = q.reshape(B * Hkv, g, N, D)[h0:h1].reshape(1, (h1 - h0) * g, N, D)
+    ks = k.reshape(B * Hkv, N, D)[h0:h1].reshape(1, h1 - h0, N, D)
+    vs = v.reshape(B * Hkv, N, D)[h0:h1].reshape(1, h1 - h0, N, D)
+    return np.ascontiguousarray(qs), np.ascontiguousarray(ks), np.ascontiguousarray(vs)
+
+
 def rank_seed(w, rank: int) -> int:
     """Every rank runs its own, independent batch of the workload (weak scaling)."""
     return w.seed + rank
@@ -310,11 +331,25 @@ def run_gpu(args, w):
         plan_h = sa.stride_plan(p, w.N, w.block)
         plan = tuple(m.to_device(dev) for m in plan_h)
         executed = 4.0 * w.D * w.block * w.block * sum(m.n_live for m in plan_h) * w.B * w.Hq
+        if args.shard == "heads" and world > 1:
+            raise SystemExit("--shard heads runs the plain path")
         sws = torch.empty(sa.fwd_stride_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.D), dtype=torch.uint8,
                           device=dev)
 
-    # inputs: every rank its own batch (seed offset by rank); rotate sets past L2
-    q, k, v = synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=rank_seed(w, rank))
+    # inputs: every rank its own batch (seed offset by rank), or with --shard
+    # heads its range of the one workload's kv heads; rotate sets past L2
+    shard = args.shard == "heads" and world > 1
+    if shard:
+        if world > w.B * w.Hkv:
+            raise SystemExit(f"--shard heads needs at most {w.B * w.Hkv} ranks for {w.name}")
+        h0, h1 = shard_heads(w.B * w.Hkv, world, rank)
+        q, k, v = shard_inputs(*synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=w.seed), w.B, w.Hq, w.Hkv, h0, h1)
+        rB, rHkv, rHq = 1, h1 - h0, (h1 - h0) * (w.Hq // w.Hkv)
+    else:
+        q, k, v = synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=rank_seed(w, rank))
+        rB, rHkv, rHq = w.B, w.Hkv, w.Hq
+    rank_part = rB * rHkv / (w.B * w.Hkv)  # this rank's share of one workload's work
+    job_useful = useful if shard else world * useful  # work of the whole job per step
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
     set_bytes = min_bytes
     n_sets = args.sets if args.sets > 0 else max(1, min(8, math.ceil(3 * L2_BYTES / set_bytes)))
@@ -323,7 +358,7 @@ def run_gpu(args, w):
     for i in range(n_sets):
         Qi, Ki, Vi = (Q0, K0, V0) if i == 0 else (Q0.clone(), K0.clone(), V0.clone())
         Oi = torch.empty_like(Qi)
-        Li = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+        Li = torch.empty((rB, rHq, w.N), dtype=torch.float32, device=dev)
         sets.append((Qi, Ki, Vi, Oi, Li))
     stream = torch.cuda.current_stream(dev)
 
@@ -368,9 +403,9 @@ def run_gpu(args, w):
     if not args.no_e2e and not stride_path:
         pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
         Qh, Kh, Vh = pin(q), pin(k), pin(v)
-        Oh = torch.empty((w.B, w.Hq, w.N, w.D), dtype=torch.bfloat16).pin_memory()
-        Lh = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32).pin_memory()
-        ws = torch.empty(sa.fwd_host_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.D), dtype=torch.uint8,
+        Oh = torch.empty((rB, rHq, w.N, w.D), dtype=torch.bfloat16).pin_memory()
+        Lh = torch.empty((rB, rHq, w.N), dtype=torch.float32).pin_memory()
+        ws = torch.empty(sa.fwd_host_workspace_bytes(rB, rHq, rHkv, w.N, w.D), dtype=torch.uint8,
                          device=dev)
         e2e_steps = max(3, min(args.steps, 20))
         for _ in range(2):
@@ -389,7 +424,7 @@ def run_gpu(args, w):
         h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh))
         h2d += sum(a.nbytes for a in (mask_h.counts, mask_h.index, mask_h.full))  # the host block mask
         d2h = Oh.numel() * Oh.element_size() + Lh.numel() * Lh.element_size()
-        e2e = {"value": job_tflops(world, useful, e2e_steps, e2e_ms), "unit": UNIT,
+        e2e = {"value": job_tflops(1, job_useful, e2e_steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                "ms_per_step": e2e_ms / e2e_steps}
 
@@ -401,8 +436,8 @@ def run_gpu(args, w):
 
     peaks, peak_kind = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    value = job_tflops(world, useful, args.steps, elapsed_ms)
-    achieved = executed / (mean_launch_ms * 1e-3) / 1e12
+    value = job_tflops(1, job_useful, args.steps, elapsed_ms)
+    achieved = executed * rank_part / (mean_launch_ms * 1e-3) / 1e12  # rank 0's kernel
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         sample = OracleSample(w, args.cpu_seconds)
@@ -412,17 +447,20 @@ def run_gpu(args, w):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "strong" if shard else "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_of(w, world, {
-            "l2": f"{n_sets} rotating input sets of {set_bytes / 1e6:.1f} MB "
-                  f"({n_sets * set_bytes / 1e6:.0f} MB > {L2_BYTES / 1e6:.0f} MB L2)",
+            "l2": f"{n_sets} rotating input sets of {set_bytes * rank_part / 1e6:.1f} MB "
+                  f"({n_sets * set_bytes * rank_part / 1e6:.0f} MB, L2 {L2_BYTES / 1e6:.0f} MB)",
             "live_tiles": int(mask_h.n_live), "full_tiles": int(mask_h.n_full),
+            **({"parallelism": f"kv heads sharded over {world} GPUs (contiguous ranges of the "
+                               f"{w.B * w.Hkv} batch x kv-head groups; no data-path collective)"}
+               if shard else {}),
             "allowed_pairs_per_head": int(pairs),
             **({"path": "stride-aware", "executed_tiles_per_head": int(sum(m.n_live for m in plan_h))}
                if stride_path else {})}),
         "useful_frac_of_peak": value / world / peak,
-        "executed_tflops": job_tflops(world, executed, args.steps, elapsed_ms),
-        "executed_frac_of_peak": executed / (elapsed_ms / args.steps * 1e-3) / 1e12 / peak,
+        "executed_tflops": job_tflops(1, executed if shard else world * executed, args.steps, elapsed_ms),
+        "executed_frac_of_peak": executed * rank_part / (elapsed_ms / args.steps * 1e-3) / 1e12 / peak,
         "peak_kind": f"bf16 dense, {peak_kind} ({peak} TFLOP/s burst)",
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None if stride_path else profiled_traffic(w.name),
@@ -621,6 +659,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling runs)")
     ap.add_argument("--sets", type=int, default=0, help="rotating input sets (0: enough to exceed L2)")
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"])
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="with several GPUs: every rank its own batch (weak scaling), or one workload's "
+                         "kv heads split across the ranks (strong scaling)")
     ap.add_argument("--path", default="plain", choices=["plain", "stride"],
                     help="forward path: one block-sparse kernel, or the stride-aware two-pass path")
     args = ap.parse_args()

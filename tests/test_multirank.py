@@ -1,4 +1,4 @@
-"""The multi-rank path of bench.py on CPU: two gloo ranks, no GPU.
+"""The multi-rank paths of bench.py on CPU: two gloo ranks, no GPU.
 
 Every rank runs its own batch of the workload (the problems are independent,
 so there is no collective on the data path); the job's time is the slowest
@@ -6,6 +6,9 @@ rank's, taken with all_reduce(MAX); the job's throughput is the work of all
 ranks over that time.  Here the oracle stands in for the kernel as each rank's
 work, so the test also checks that a rank's result depends on its own inputs
 only (a shard computed alone equals the same shard computed in the job).
+With --shard heads one workload is split instead: each rank takes a contiguous
+range of its batch x kv-head groups (with their query heads), and the ranks'
+parts put together must equal the whole computed at once.
 """
 import json
 import math
@@ -92,3 +95,56 @@ def test_single_rank_helpers_without_process_group():
     import bench
     assert bench.max_over_ranks(3.5, None, "cpu") == 3.5
     assert math.isclose(bench.job_tflops(1, 2e12, 10, 1000.0), 20.0)
+
+
+@pytest.mark.parametrize("n_heads,world", [(16, 2), (16, 3), (8, 8), (5, 2), (1, 1), (64, 7)])
+def test_head_shards_partition_the_heads(n_heads, world):
+    import bench
+    ranges = [bench.shard_heads(n_heads, world, r) for r in range(world)]
+    assert ranges[0][0] == 0 and ranges[-1][1] == n_heads
+    for (a0, a1), (b0, b1) in zip(ranges, ranges[1:]):
+        assert a1 == b0 and a0 < a1
+    sizes = [h1 - h0 for h0, h1 in ranges]
+    assert max(sizes) - min(sizes) <= 1
+
+
+def shard_rank_main(rank: int, world: int, port: int, out_dir: str):
+    """One workload split across the ranks by kv heads (bench --shard heads):
+    each rank runs its range of the batch x kv-head groups, as a batch of one,
+    with the oracle standing in for the kernel."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+    import synth
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    B, Hq, Hkv, N, D = 2, 6, 3, 300, 32
+    h0, h1 = bench.shard_heads(B * Hkv, world, rank)
+    q, k, v = bench.shard_inputs(*synth.qkv(B, Hq, Hkv, N, D, seed=0), B, Hq, Hkv, h0, h1)
+    O, LSE = oracle.attention(q, k, v, oracle.Pattern(window=60, sinks=4), 1 / math.sqrt(D))
+    np.save(os.path.join(out_dir, f"shard_O_{rank}.npy"), O)
+    np.save(os.path.join(out_dir, f"shard_L_{rank}.npy"), LSE)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_split_one_workload(tmp_path):
+    """The ranks' shards put together equal the whole workload computed at once."""
+    world = 2
+    mp.spawn(shard_rank_main, args=(world, free_port(), str(tmp_path)), nprocs=world, join=True)
+    import oracle
+    import synth
+    B, Hq, Hkv, N, D = 2, 6, 3, 300, 32
+    q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=0)
+    O, LSE = oracle.attention(q, k, v, oracle.Pattern(window=60, sinks=4), 1 / math.sqrt(D))
+    parts_O = [np.load(tmp_path / f"shard_O_{r}.npy") for r in range(world)]
+    parts_L = [np.load(tmp_path / f"shard_L_{r}.npy") for r in range(world)]
+    # flattened batch x query-head order: kv head h's query heads are h * g .. h * g + g - 1
+    got_O = np.concatenate([x[0] for x in parts_O], axis=0).reshape(O.shape)
+    got_L = np.concatenate([x[0] for x in parts_L], axis=0).reshape(LSE.shape)
+    assert np.array_equal(got_O, O) and np.array_equal(got_L, LSE)
+    assert sum(x.shape[1] for x in parts_O) == B * Hq
