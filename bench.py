@@ -249,7 +249,8 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_of(w, args.gpus),
+        "data": "synthetic", "config": config_of(w, args.gpus, None if args.path == "plain" else {"path": "stride-aware"},
+                                                  shard=args.shard == "heads" and args.gpus > 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": sample.threads, "kind": "oracle",
                          "sample": sample.describe(total / args.steps)},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -258,11 +259,17 @@ def run_reference(args, w):
     return 0
 
 
-def config_of(w, n_gpus, extra=None):
+def config_of(w, n_gpus, extra=None, shard=False):
+    """The workload as both arms report it (the same dict for the same run)."""
     c = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "D": w.D,
          "pattern": {"causal": 1, **w.pattern_args()}, "block": w.block, "seed": w.seed,
          "inputs": "iid N(0,1) -> bf16, scale 1/sqrt(D)",
-         "parallelism": "single GPU" if n_gpus == 1 else f"{n_gpus} independent batches, one per GPU"}
+         "l2": f"GPU timing rotates the inputs over up to 8 sets whose footprint exceeds the "
+               f"{L2_BYTES / 1e6:.0f} MB L2 (no flush); workload_info.input_sets gives the sets",
+         "parallelism": ("single GPU" if n_gpus == 1 else
+                         f"kv heads sharded over {n_gpus} GPUs (contiguous ranges of the batch x kv-head "
+                         f"groups; no data-path collective)" if shard else
+                         f"{n_gpus} independent batches, one per GPU")}
     if extra:
         c.update(extra)
     return c
@@ -351,7 +358,7 @@ def run_gpu(args, w):
     rank_part = rB * rHkv / (w.B * w.Hkv)  # this rank's share of one workload's work
     job_useful = useful if shard else world * useful  # work of the whole job per step
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
-    set_bytes = min_bytes
+    set_bytes = min_bytes * rank_part  # this rank's inputs and outputs
     n_sets = args.sets if args.sets > 0 else max(1, min(8, math.ceil(3 * L2_BYTES / set_bytes)))
     Q0, K0, V0 = to_dev(q), to_dev(k), to_dev(v)
     sets = []
@@ -448,16 +455,12 @@ def run_gpu(args, w):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "strong" if shard else "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_of(w, world, {
-            "l2": f"{n_sets} rotating input sets of {set_bytes * rank_part / 1e6:.1f} MB "
-                  f"({n_sets * set_bytes * rank_part / 1e6:.0f} MB, L2 {L2_BYTES / 1e6:.0f} MB)",
+        "config": config_of(w, world, {"path": "stride-aware"} if stride_path else None, shard=shard),
+        "workload_info": {
+            "input_sets": f"{n_sets} of {set_bytes / 1e6:.1f} MB per rank",
             "live_tiles": int(mask_h.n_live), "full_tiles": int(mask_h.n_full),
-            **({"parallelism": f"kv heads sharded over {world} GPUs (contiguous ranges of the "
-                               f"{w.B * w.Hkv} batch x kv-head groups; no data-path collective)"}
-               if shard else {}),
             "allowed_pairs_per_head": int(pairs),
-            **({"path": "stride-aware", "executed_tiles_per_head": int(sum(m.n_live for m in plan_h))}
-               if stride_path else {})}),
+            **({"executed_tiles_per_head": int(sum(m.n_live for m in plan_h))} if stride_path else {})},
         "useful_frac_of_peak": value / world / peak,
         "executed_tflops": job_tflops(1, executed if shard else world * executed, args.steps, elapsed_ms),
         "executed_frac_of_peak": executed * rank_part / (elapsed_ms / args.steps * 1e-3) / 1e12 / peak,
@@ -606,11 +609,10 @@ def run_gpu_bwd(args, w):
         "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_of(w, world, {
-            "pass": "bwd",
-            "l2": f"{n_sets} rotating input sets of {set_bytes / 1e6:.1f} MB "
-                  f"({n_sets * set_bytes / 1e6:.0f} MB > {L2_BYTES / 1e6:.0f} MB L2)",
-            "live_tiles": int(mask128.n_live), "backward_tile": 128, "allowed_pairs_per_head": int(pairs)}),
+        "config": config_of(w, world, {"pass": "bwd"}),
+        "workload_info": {"input_sets": f"{n_sets} of {set_bytes / 1e6:.1f} MB",
+                          "live_tiles": int(mask128.n_live), "backward_tile": 128,
+                          "allowed_pairs_per_head": int(pairs)},
         "useful_frac_of_peak": value / world / peak,
         "executed_tflops": job_tflops(world, executed, args.steps, elapsed_ms),
         "peak_kind": f"bf16 dense, {peak_kind} ({peak} TFLOP/s burst)",
