@@ -14,7 +14,10 @@ roofline   the forward kernel against the measured dense bf16 tensor peak:
            the mean per-launch duration: this rank's K back-to-back launches
            timed with one pair of CUDA events on the launching stream.
 e2e        the same metric through the host-buffer C ABI call (pinned host
-           Q/K/V in, O/LSE out, copies inside the timed region).
+           Q/K/V and the host mask in, O/LSE out, copies inside the timed
+           region), the steps queued back to back (each step's inputs cross
+           PCIe while the previous step's outputs come back); the latency of
+           one blocking call is reported beside it.
 cpu_baseline  the fp64 CPU oracle on a bounded row sample, host cores.
 
 With --pass bwd one step is one backward pass (three launches: prep, the
@@ -418,14 +421,26 @@ def run_gpu(args, w):
         for _ in range(2):
             sa.fwd_host(Qh, Kh, Vh, mask_h, p, Oh, Lh, ws, scale=w.scale, stream=stream)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # one blocking call per step: its latency
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(3):
+            sa.fwd_host(Qh, Kh, Vh, mask_h, p, Oh, Lh, ws, scale=w.scale, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        sync_ms = e0.elapsed_time(e1) / 3
+        # the steps queued back to back: each step's inputs cross PCIe while the
+        # previous step's outputs come back; one wait at the end
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
         e0.record(stream)
         for _ in range(e2e_steps):
-            sa.fwd_host(Qh, Kh, Vh, mask_h, p, Oh, Lh, ws, scale=w.scale, stream=stream)
+            sa.fwd_host(Qh, Kh, Vh, mask_h, p, Oh, Lh, ws, scale=w.scale, stream=stream, wait=False)
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        if sa.check_device(stream) != sa.SA_OK:
+            raise SystemExit("device status not ok after the end-to-end leg")
         e2e_ms = e0.elapsed_time(e1)
         e2e_ms = max_over_ranks(e2e_ms, dist if world > 1 else None, dev)
         h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh))
@@ -433,7 +448,8 @@ def run_gpu(args, w):
         d2h = Oh.numel() * Oh.element_size() + Lh.numel() * Lh.element_size()
         e2e = {"value": job_tflops(1, job_useful, e2e_steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-               "ms_per_step": e2e_ms / e2e_steps}
+               "ms_per_step": e2e_ms / e2e_steps, "api": "sparse_attn_fwd_host_async, steps queued back to back",
+               "blocking_call_ms": sync_ms}
 
     if world > 1:
         dist.barrier()

@@ -39,7 +39,7 @@ DEBUG_BWD_SPLIT = 4
 
 EXPORTED = (
     "sparse_attn_num_tiles", "sparse_attn_build_block_mask", "sparse_attn_count_pairs",
-    "sparse_attn_fwd", "sparse_attn_fwd_host", "sparse_attn_fwd_host_workspace",
+    "sparse_attn_fwd", "sparse_attn_fwd_host", "sparse_attn_fwd_host_async", "sparse_attn_fwd_host_workspace",
     "sparse_attn_check_device", "sparse_attn_set_debug", "sparse_attn_status_string",
     "sparse_attn_version", "sparse_attn_fwd_noalloc", "sparse_attn_fwd_heads",
     "sparse_attn_transpose_block_mask", "sparse_attn_bwd_workspace", "sparse_attn_bwd",
@@ -84,6 +84,7 @@ def _load() -> ctypes.CDLL:
     L.sparse_attn_count_pairs.argtypes = [P, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
     L.sparse_attn_fwd.argtypes = [vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp]
     L.sparse_attn_fwd_host.argtypes = [vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp]
+    L.sparse_attn_fwd_host_async.argtypes = [vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp]
     L.sparse_attn_fwd_host_workspace.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
     L.sparse_attn_fwd_noalloc.argtypes = [vp, vp, vp, M, P, S, ctypes.c_float, vp, vp, vp]
     L.sparse_attn_fwd_heads.argtypes = [vp, vp, vp, M, P, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32), S,
@@ -104,7 +105,8 @@ def _load() -> ctypes.CDLL:
     L.sparse_attn_version.argtypes = []
     L.sparse_attn_version.restype = ctypes.c_int32
     for name in ("sparse_attn_build_block_mask", "sparse_attn_count_pairs", "sparse_attn_fwd",
-                 "sparse_attn_fwd_host", "sparse_attn_fwd_host_workspace", "sparse_attn_check_device",
+                 "sparse_attn_fwd_host", "sparse_attn_fwd_host_async", "sparse_attn_fwd_host_workspace",
+                 "sparse_attn_check_device",
                  "sparse_attn_set_debug", "sparse_attn_fwd_noalloc", "sparse_attn_fwd_heads",
                  "sparse_attn_transpose_block_mask", "sparse_attn_bwd_workspace", "sparse_attn_bwd",
                  "sparse_attn_stride_plan", "sparse_attn_fwd_stride_workspace", "sparse_attn_fwd_stride",
@@ -421,11 +423,14 @@ def fwd_host_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, D: int) -> int:
 
 
 def fwd_host(q_host, k_host, v_host, mask: BlockMask, pattern: Pattern, o_host, lse_host, workspace,
-             scale: float | None = None, stream=None) -> None:
+             scale: float | None = None, stream=None, wait: bool = True) -> None:
     """Forward from host (ideally pinned) tensors: copies in, computes, copies
     out and waits, in chunks of kv heads whose copies overlap the kernels.
     ``workspace`` is a device tensor of at least ``fwd_host_workspace_bytes``
-    bytes; ``mask`` is the HOST block mask from ``build_block_mask``."""
+    bytes; ``mask`` is the HOST block mask from ``build_block_mask``.  With
+    ``wait=False`` the call only queues the work (sparse_attn_fwd_host_async):
+    ``stream`` reaches its end once O and LSE are in host memory, and successive
+    calls overlap their input and output copies."""
     if not isinstance(mask.counts, np.ndarray):
         raise TypeError("fwd_host takes the host block mask (numpy arrays), not a device copy")
     B, Hq, N, D = q_host.shape
@@ -437,11 +442,11 @@ def fwd_host(q_host, k_host, v_host, mask: BlockMask, pattern: Pattern, o_host, 
     import torch
     with torch.cuda.device(workspace.device):
         st = _stream_handle(stream, workspace.device)
-        _check(lib.sparse_attn_fwd_host(q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(),
-                                        ctypes.byref(mask._c()), ctypes.byref(pattern._c()),
-                                        ctypes.byref(shape), float(scale), o_host.data_ptr(),
-                                        lse_host.data_ptr(), workspace.data_ptr(), nbytes, st),
-               "sparse_attn_fwd_host")
+        fn = lib.sparse_attn_fwd_host if wait else lib.sparse_attn_fwd_host_async
+        _check(fn(q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(), ctypes.byref(mask._c()),
+                  ctypes.byref(pattern._c()), ctypes.byref(shape), float(scale), o_host.data_ptr(),
+                  lse_host.data_ptr(), workspace.data_ptr(), nbytes, st),
+               "sparse_attn_fwd_host" if wait else "sparse_attn_fwd_host_async")
 
 
 def fwd_noalloc(q, k, v, mask: BlockMask, pattern: Pattern, out, lse, scale: float | None = None,

@@ -4,6 +4,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include "../../include/sparse_attn.h"
@@ -484,7 +485,14 @@ HostLayout host_layout(const sa_shape& s)
 struct HostStreams {
     cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
     cudaEvent_t start = nullptr, done = nullptr;
+    cudaEvent_t comp_done = nullptr;  // the previous call's last kernel (its inputs are free after it)
     cudaEvent_t landed[kHostChunks] = {}, computed[kHostChunks] = {};
+    // Pinned staging of the block mask: a copy from pageable memory would first
+    // wait for its stream to drain, which would hold the host until the previous
+    // call's kernels are done.  Reused once the previous call's copy out of it is.
+    uint8_t* stage = nullptr;
+    size_t stage_bytes = 0;
+    cudaEvent_t staged = nullptr;
 };
 HostStreams g_host[kMaxDevices];
 std::mutex g_host_mu[kMaxDevices];
@@ -496,7 +504,9 @@ int host_streams(int dev, HostStreams** out)
         const unsigned ef = cudaEventDisableTiming;
         if (cudaStreamCreateWithFlags(&h.comp, cudaStreamNonBlocking) != cudaSuccess ||
             cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaEventCreateWithFlags(&h.start, ef) != cudaSuccess || cudaEventCreateWithFlags(&h.done, ef) != cudaSuccess)
+            cudaEventCreateWithFlags(&h.start, ef) != cudaSuccess || cudaEventCreateWithFlags(&h.done, ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&h.comp_done, ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&h.staged, ef) != cudaSuccess)
             return SA_ERR_CUDA;
         for (int c = 0; c < kHostChunks; c++)
             if (cudaEventCreateWithFlags(&h.landed[c], ef) != cudaSuccess ||
@@ -520,10 +530,10 @@ extern "C" int sparse_attn_fwd_host_workspace(const sa_shape* shape, size_t* byt
     return SA_OK;
 }
 
-extern "C" int sparse_attn_fwd_host(const void* Q_host, const void* K_host, const void* V_host,
-                                    const sa_block_mask* mask_host, const sa_pattern* pattern, const sa_shape* shape,
-                                    float scale, void* O_host, float* LSE_host, void* workspace,
-                                    size_t workspace_bytes, void* stream)
+extern "C" int sparse_attn_fwd_host_async(const void* Q_host, const void* K_host, const void* V_host,
+                                          const sa_block_mask* mask_host, const sa_pattern* pattern,
+                                          const sa_shape* shape, float scale, void* O_host, float* LSE_host,
+                                          void* workspace, size_t workspace_bytes, void* stream)
 {
     if (!shape || !mask_host || !pattern) return SA_ERR_INVALID_ARG;
     const sa_shape s = *shape;
@@ -549,20 +559,43 @@ extern "C" int sparse_attn_fwd_host(const void* Q_host, const void* K_host, cons
 
     uint8_t* w = static_cast<uint8_t*>(workspace);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // everything queued before this call on the caller's stream comes first
-    if (cudaEventRecord(hs->start, st) != cudaSuccess || cudaStreamWaitEvent(hs->in, hs->start, 0) != cudaSuccess)
+    // everything queued before this call on the caller's stream comes first; the
+    // inputs (and the mask copy) of the previous call on this device must have
+    // been read by its kernels before they are overwritten, its outputs copied
+    // back before the new kernels write theirs (its copies back may still be
+    // running while this call's inputs come in)
+    if (cudaEventRecord(hs->start, st) != cudaSuccess || cudaStreamWaitEvent(hs->in, hs->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(hs->in, hs->comp_done, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(hs->comp, hs->done, 0) != cudaSuccess)
         return SA_ERR_CUDA;
+    // the mask's three arrays, each 256-aligned, at the start of the workspace
+    // (its mask region is sized for the most tiles a shape can have)
+    const size_t idx = (size_t(T) * 4 + 255) & ~size_t(255);
+    const size_t full = idx + ((size_t(T) * T * 4 + 255) & ~size_t(255));
+    const size_t bytes = full + size_t(T) * T;
+    if (L.count + bytes > L.q) return SA_ERR_BUFFER_TOO_SMALL;  // cannot happen: T <= ceil(N / 64)
     sa_block_mask dmask = *mask_host;
     dmask.kv_count = reinterpret_cast<int32_t*>(w + L.count);
-    dmask.kv_index = reinterpret_cast<int32_t*>(w + L.index);
-    dmask.kv_full = w + L.full;
-    if (cudaMemcpyAsync(dmask.kv_count, mask_host->kv_count, size_t(T) * 4, cudaMemcpyHostToDevice, hs->in) !=
-            cudaSuccess ||
-        cudaMemcpyAsync(dmask.kv_index, mask_host->kv_index, size_t(T) * T * 4, cudaMemcpyHostToDevice, hs->in) !=
-            cudaSuccess ||
-        cudaMemcpyAsync(dmask.kv_full, mask_host->kv_full, size_t(T) * T, cudaMemcpyHostToDevice, hs->in) !=
-            cudaSuccess)
-        return SA_ERR_CUDA;
+    dmask.kv_index = reinterpret_cast<int32_t*>(w + L.count + idx);
+    dmask.kv_full = w + L.count + full;
+    {
+        // the same layout in the pinned stage, then one asynchronous copy
+        if (cudaEventSynchronize(hs->staged) != cudaSuccess) return SA_ERR_CUDA;
+        if (hs->stage_bytes < bytes) {
+            if (hs->stage && cudaFreeHost(hs->stage) != cudaSuccess) return SA_ERR_CUDA;
+            hs->stage = nullptr;
+            hs->stage_bytes = 0;
+            if (cudaHostAlloc(reinterpret_cast<void**>(&hs->stage), bytes, cudaHostAllocDefault) != cudaSuccess)
+                return SA_ERR_CUDA;
+            hs->stage_bytes = bytes;
+        }
+        std::memcpy(hs->stage, mask_host->kv_count, size_t(T) * 4);
+        std::memcpy(hs->stage + idx, mask_host->kv_index, size_t(T) * T * 4);
+        std::memcpy(hs->stage + full, mask_host->kv_full, size_t(T) * T);
+        if (cudaMemcpyAsync(w + L.count, hs->stage, bytes, cudaMemcpyHostToDevice, hs->in) != cudaSuccess ||
+            cudaEventRecord(hs->staged, hs->in) != cudaSuccess)
+            return SA_ERR_CUDA;
+    }
 
     const int64_t heads = int64_t(s.B) * s.Hkv;  // flattened kv heads
     const int64_t group = s.Hq / s.Hkv;
@@ -613,8 +646,21 @@ extern "C" int sparse_attn_fwd_host(const void* Q_host, const void* K_host, cons
             return SA_ERR_CUDA;
     }
     // the caller's stream continues after the last copy back
-    if (cudaEventRecord(hs->done, hs->out) != cudaSuccess || cudaStreamWaitEvent(st, hs->done, 0) != cudaSuccess)
+    if (cudaEventRecord(hs->comp_done, hs->comp) != cudaSuccess || cudaEventRecord(hs->done, hs->out) != cudaSuccess ||
+        cudaStreamWaitEvent(st, hs->done, 0) != cudaSuccess)
         return SA_ERR_CUDA;
+    return SA_OK;
+}
+
+extern "C" int sparse_attn_fwd_host(const void* Q_host, const void* K_host, const void* V_host,
+                                    const sa_block_mask* mask_host, const sa_pattern* pattern, const sa_shape* shape,
+                                    float scale, void* O_host, float* LSE_host, void* workspace,
+                                    size_t workspace_bytes, void* stream)
+{
+    const int rc = sparse_attn_fwd_host_async(Q_host, K_host, V_host, mask_host, pattern, shape, scale, O_host,
+                                              LSE_host, workspace, workspace_bytes, stream);
+    if (rc != SA_OK) return rc;
+    if (!shape || shape->B == 0 || shape->Hq == 0 || shape->N == 0) return SA_OK;
     return sparse_attn_check_device(stream);
 }
 

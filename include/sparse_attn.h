@@ -180,6 +180,22 @@ int sparse_attn_fwd_host(const void* Q_host, const void* K_host, const void* V_h
                          float* LSE_host, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * sparse_attn_fwd_host without the final wait: queues the same chunked copies
+ * and kernels and returns; `stream` reaches the call's end once O and LSE are
+ * in host memory.  Until then the caller must leave the host inputs, the host
+ * mask and the workspace unchanged and must not read O_host, LSE_host.  Calls
+ * on one device are ordered: a call's input copies wait only for the previous
+ * call's kernels (not for its copies back), and its kernels for the previous
+ * call's copies back, so successive steps overlap their input and output
+ * copies.  Errors in the arguments come back at once; a device timeout through
+ * sparse_attn_check_device.
+ */
+int sparse_attn_fwd_host_async(const void* Q_host, const void* K_host, const void* V_host,
+                               const sa_block_mask* mask_host, const sa_pattern* pattern, const sa_shape* shape,
+                               float scale, void* O_host, float* LSE_host, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/*
  * Forward pass with a pattern per query head ("Sparse-трансформеры" page,
  * section "Комбинация — норма, а не исключение": heads of one layer may carry
  * different patterns, some local, some strided).  Query head h attends under

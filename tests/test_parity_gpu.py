@@ -182,6 +182,30 @@ def test_host_buffer_entry_point_matches_device_entry_point(B, Hq, Hkv, N, D, bl
     compare(Oh.float().numpy(), Lh.numpy(), Oref, Lref)
 
 
+def test_host_buffer_async_calls_in_a_row():
+    """Three queued host-buffer calls on different inputs, then one wait: each
+    output equals the device call's on its inputs, bit for bit (the calls share
+    the workspace; their copies overlap, the ordering keeps them apart)."""
+    B, Hq, Hkv, N, D = 2, 8, 4, 1536, 128
+    p = sa.Pattern(window=300, sinks=4)
+    mask = sa.build_block_mask(p, N, 128)
+    ws = torch.empty(sa.fwd_host_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device="cuda")
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    runs = []
+    for i in range(3):
+        q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=40 + i)
+        Oh = torch.empty((B, Hq, N, D), dtype=torch.bfloat16).pin_memory()
+        Lh = torch.empty((B, Hq, N), dtype=torch.float32).pin_memory()
+        ins = (pin(q), pin(k), pin(v))
+        sa.fwd_host(*ins, mask, p, Oh, Lh, ws, wait=False)
+        runs.append((q, k, v, ins, Oh, Lh))
+    torch.cuda.synchronize()
+    assert sa.check_device() == sa.SA_OK
+    for q, k, v, _, Oh, Lh in runs:
+        O, LSE = run_gpu(q, k, v, p, 128, 1 / math.sqrt(D))
+        assert np.array_equal(Oh.float().numpy(), O) and np.array_equal(Lh.numpy(), LSE)
+
+
 def test_device_timeout_is_reported_and_context_survives():
     """The test hook skips the Q tile load, so the kernel's bounded waits
     expire (about 10 ms each); the status comes back as a timeout and the
