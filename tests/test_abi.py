@@ -440,3 +440,17 @@ def test_host_workspace_covers_the_mask_copy():
     T = -(-N // 64)
     need = 2 * B * Hq * N * D * 2 + 2 * B * Hkv * N * D * 2 + B * Hq * N * 4 + T * 4 + 5 * T * T
     assert need <= ws.value <= need + 8 * 256
+
+
+def test_more_tiles_than_the_kernel_takes_is_refused_without_gpu():
+    """4097 tiles per side (one past the step lists' 12-bit tile indices) is
+    SA_ERR_UNSUPPORTED before any CUDA call; 4096 passes the check (the fake
+    pointers then stop it at alignment, still before any CUDA call)."""
+    p = sa.Pattern(window=8)._c()
+    fake = 1 << 20
+    for T, want in ((4097, sa.SA_ERR_UNSUPPORTED), (4096, sa.SA_ERR_MISALIGNED)):
+        m = sa._BlockMask(T, T, 128, 1, 1, 0, fake, fake, fake)
+        shape = sa._Shape(1, 1, 1, T * 128, 128)
+        rc = sa.lib.sparse_attn_fwd(fake + 8, fake, fake, ctypes.byref(m), ctypes.byref(p), ctypes.byref(shape),
+                                    0.1, fake, fake, None)
+        assert rc == want, (T, rc)

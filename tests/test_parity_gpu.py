@@ -145,6 +145,21 @@ def test_workload_parity_sampled(name):
     compare(O[:, :, rows], LSE[:, :, rows], Oref, LSEref)
 
 
+@pytest.mark.parametrize("block,D", [(128, 128), (64, 64)])
+def test_largest_tile_count(block, D):
+    """The most tiles per side the kernel takes (4096: its step lists hold 12-bit
+    tile indices), with a ragged last tile: N = 4096 * block - 37.  Sampled
+    rows (both ends of every query tile and 64 more) against the oracle."""
+    N = 4096 * block - 37
+    B, Hq, Hkv = 1, 2, 1
+    p = sa.Pattern(window=300, sinks=4, n_global=2)
+    q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=9)
+    O, LSE = run_gpu(q, k, v, p, block, 1 / math.sqrt(D))
+    rows = sample_rows(N, extra=64)
+    Oref, LSEref = oracle.attention(q, k, v, opattern(p), 1 / math.sqrt(D), rows=rows)
+    compare(O[:, :, rows], LSE[:, :, rows], Oref, LSEref)
+
+
 def test_repeat_calls_are_deterministic():
     w = WORKLOADS["w1024_s4_n8192"]
     q, k, v = synth.qkv(1, 2, 2, 4096, 128, seed=3)
