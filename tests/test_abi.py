@@ -454,3 +454,18 @@ def test_more_tiles_than_the_kernel_takes_is_refused_without_gpu():
         rc = sa.lib.sparse_attn_fwd(fake + 8, fake, fake, ctypes.byref(m), ctypes.byref(p), ctypes.byref(shape),
                                     0.1, fake, fake, None)
         assert rc == want, (T, rc)
+
+
+def test_headline_tile_lists_are_a_diagonal_band_plus_the_sink_column():
+    """The headline pattern's picture ("Sparse Attention" glossary page, section
+    "Ein Muster in Einsparungen verwandeln"): every query tile lists kv tile 0
+    (the sinks) and the tiles from 8 before the diagonal up to it (a 1024-token
+    window is 8 tiles of 128, and q - kv <= 1024 reaches one more), nothing else;
+    only the diagonal tiles and the band's far edge are partial."""
+    m = sa.build_block_mask(sa.Pattern(window=1024, sinks=4), 8192, 128)
+    for i in range(m.T):
+        want = sorted({0} | set(range(max(0, i - 8), i + 1)))
+        assert list(m.index[i, : m.counts[i]]) == want, i
+        full = {int(j) for j, f in zip(m.index[i, : m.counts[i]], m.full[i, : m.counts[i]]) if f}
+        # full: the tiles strictly inside the band (1 <= i - j <= 7)
+        assert full == set(range(max(0, i - 7), i)), i

@@ -254,6 +254,13 @@ HEAD_CASES = [
     # no live step (its rows are O = 0, LSE = -inf) while the other runs
     (1, 4, 2, 900, 128, 128, [sa.Pattern(window=200, sinks=4), sa.Pattern(window=-1)], [0, 1, 1, 0]),
     (1, 4, 2, 700, 64, 64, [sa.Pattern(window=-1), sa.Pattern(window=90, sinks=2)], [0, 1, 1, 0]),
+    # the most patterns the table holds (8), one per head of a batch of 16 heads on 4 kv heads,
+    # causal and not, with stripes and summary columns
+    (1, 16, 4, 1100, 64, 128,
+     [sa.Pattern(window=100, sinks=4), sa.Pattern(window=40, stride=64, n_global=3), sa.Pattern(window=-1, sinks=20),
+      sa.Pattern(window=1100), sa.Pattern(window=60, causal=0), sa.Pattern(window=-1, causal=0, area=275),
+      sa.Pattern(window=-1, area=128, summary=16), sa.Pattern(window=0)],
+     [0, 1, 2, 3, 4, 5, 6, 7, 7, 6, 5, 4, 3, 2, 1, 0]),
 ]
 
 
