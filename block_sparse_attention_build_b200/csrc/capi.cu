@@ -233,6 +233,14 @@ int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* m
     p.status = status;
     p.timeout = timeout;
     p.debug_flags = debug_flags;
+    {
+        sa_block_mask_fields f{T, 0, 0};  // the longest row and the live tiles over all patterns
+        for (int i = 0; i < n_patterns; i++) {
+            f.n_live = masks[i].n_live > f.n_live ? masks[i].n_live : f.n_live;
+            f.max_per_row = masks[i].max_per_row > f.max_per_row ? masks[i].max_per_row : f.max_per_row;
+        }
+        p.snake = snake_order(f);
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int g = static_cast<int>(grid);
     HeadPatterns hp{};

@@ -170,6 +170,7 @@ extern "C" int sparse_attn_fwd_noalloc(const void* Q, const void* K, const void*
     p.status = status;
     p.timeout = wait_limit_cycles();
     p.debug_flags = debug_flags() & 1;  // the skip-Q-load test hook; work units are never split here
+    p.snake = snake_order(sa_block_mask_fields{T, mask->n_live, mask->max_per_row});
     const int grid = static_cast<int>(n_items < n_sm ? n_items : n_sm);
     int rc;
     if (s.D == 128 && bn == 128)
