@@ -483,8 +483,9 @@ def run_gpu(args, w):
         "peak_kind": f"bf16 dense, {peak_kind} ({peak} TFLOP/s burst)",
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None if stride_path else profiled_traffic(w.name),
-                     "kernel": ("stride-aware step: 3 grouping copies + 2 x fwd_kernel + merge" if stride_path
-                                else "fwd_kernel<D,BN>"),
+                     "kernel": (("stride-aware step: 2 x fwd_kernel + merge"
+                                 + ("" if (w.N // max(w.stride, 1)) % 128 == 0 and (w.N // max(w.stride, 1)) % w.block == 0
+                                    else " + 3 grouping copies")) if stride_path else "fwd_kernel<D,BN>"),
                      "mean_launch_us": mean_launch_ms * 1e3,
                      "algorithmic_flop_per_launch": executed,
                      "hbm_gbs_min_bytes": min_bytes / (mean_launch_ms * 1e-3) / 1e9},
