@@ -185,12 +185,14 @@ struct sa_block_mask_fields {
 
 // Work items (host side).  Units that fill whole rounds of the CTAs run whole.
 // When the rest would give at most half of the CTAs one more unit, those units
-// are split, two items each, so that the last round costs about half a unit.
-// `split_all` (a test switch) splits every unit.
+// are split, two items each, so that the last round costs about half a unit;
+// so are all units when there are at most half as many as CTAs (a small
+// problem: the idle CTAs then take half of every list).  `split_all` (a test
+// switch) splits every unit.
 inline void plan_items(int64_t n_units, int64_t n_ctas, bool split_all, int64_t* n_whole, int64_t* n_items)
 {
     int64_t whole = n_units;
-    if (split_all) {
+    if (split_all || 2 * n_units <= n_ctas) {
         whole = 0;
     } else if (n_units > n_ctas) {
         const int64_t r = n_units % n_ctas;

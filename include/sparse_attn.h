@@ -171,8 +171,9 @@ int sparse_attn_fwd(const void* Q, const void* K, const void* V, const sa_block_
  * too), with the first error, including a device timeout.  Pinned host memory
  * makes the copies asynchronous DMA; pageable memory works but serialises
  * them.  Each chunk is a sparse_attn_fwd call on its heads: results are those
- * of sparse_attn_fwd, bit-identical when neither call splits work units (the
- * kernel splits units only when they fill its last round of CTAs unevenly).
+ * of sparse_attn_fwd, bit-identical when both calls split work units alike
+ * (the kernel splits every unit of a problem with at most half as many units
+ * as SMs, and those of a last round that would leave most CTAs idle).
  * Calls on one device are serialised.
  */
 int sparse_attn_fwd_host(const void* Q_host, const void* K_host, const void* V_host, const sa_block_mask* mask_host,
@@ -236,8 +237,9 @@ int sparse_attn_check_device(void* stream);
  * entry point) skip the Q tile load, so the kernel's bounded waits expire and
  * it reports SA_ERR_DEVICE_TIMEOUT instead of computing.  Bit 1 makes sparse_attn_fwd
  * split every work unit (each query tile's kv list walked in two halves that
- * are merged at the end), the path the kernel otherwise takes only for the
- * last, partial round of units; results agree within rounding.  Bit 2 makes
+ * are merged at the end), the path the kernel otherwise takes only for small
+ * problems and the last, partial round of units; results agree within
+ * rounding.  Bit 2 makes
  * sparse_attn_bwd split every kv tile's list of more than 32 steps into work
  * items of at most 32 steps whose dK, dV add up in fp32 sums, the path it
  * otherwise takes only for lists longer than an SM's share of all steps.

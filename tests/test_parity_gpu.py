@@ -77,7 +77,7 @@ SMALL = [
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: f"B{c[0]}H{c[1]}/{c[2]}N{c[3]}D{c[4]}b{c[6]}-{c[5]}")
 def test_small_full_parity_split_units(case):
     """Every unit split: each query tile's kv list walked as two halves by the
-    two slots and merged at the end (the path of a partial last round)."""
+    two slots and merged at the end (the path of small problems and of a partial last round)."""
     B, Hq, Hkv, N, D, p, block = case
     q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=N + D + 1)
     scale = 1 / math.sqrt(D)
@@ -177,8 +177,9 @@ def test_repeat_calls_are_deterministic():
 ])
 def test_host_buffer_entry_point_matches_device_entry_point(B, Hq, Hkv, N, D, block, pinned):
     """The host-buffer call (chunks of kv heads, copies overlapping the kernels)
-    gives the device call's output bit for bit (neither splits work units at
-    these sizes), and both agree with the oracle."""
+    gives the device call's output bit for bit, and both agree with the oracle.
+    At these sizes the whole problem and every chunk have at most half as many
+    work units as SMs, so both calls split every unit alike."""
     p = sa.Pattern(window=200, sinks=4)
     q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=21)
     O, LSE = run_gpu(q, k, v, p, block, 1 / math.sqrt(D))
@@ -200,25 +201,33 @@ def test_host_buffer_entry_point_matches_device_entry_point(B, Hq, Hkv, N, D, bl
 def test_host_buffer_async_calls_in_a_row():
     """Three queued host-buffer calls on different inputs, then one wait: each
     output equals the device call's on its inputs, bit for bit (the calls share
-    the workspace; their copies overlap, the ordering keeps them apart)."""
+    the workspace; their copies overlap, the ordering keeps them apart).  The
+    whole problem has more units than half the SMs and its chunks fewer, so
+    the test hook splits every unit on both sides to give them one plan."""
     B, Hq, Hkv, N, D = 2, 8, 4, 1536, 128
     p = sa.Pattern(window=300, sinks=4)
     mask = sa.build_block_mask(p, N, 128)
     ws = torch.empty(sa.fwd_host_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device="cuda")
     pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
     runs = []
-    for i in range(3):
-        q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=40 + i)
-        Oh = torch.empty((B, Hq, N, D), dtype=torch.bfloat16).pin_memory()
-        Lh = torch.empty((B, Hq, N), dtype=torch.float32).pin_memory()
-        ins = (pin(q), pin(k), pin(v))
-        sa.fwd_host(*ins, mask, p, Oh, Lh, ws, wait=False)
-        runs.append((q, k, v, ins, Oh, Lh))
-    torch.cuda.synchronize()
-    assert sa.check_device() == sa.SA_OK
-    for q, k, v, _, Oh, Lh in runs:
-        O, LSE = run_gpu(q, k, v, p, 128, 1 / math.sqrt(D))
-        assert np.array_equal(Oh.float().numpy(), O) and np.array_equal(Lh.numpy(), LSE)
+    sa.set_debug(sa.DEBUG_SPLIT_ALL)
+    try:
+        for i in range(3):
+            q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=40 + i)
+            Oh = torch.empty((B, Hq, N, D), dtype=torch.bfloat16).pin_memory()
+            Lh = torch.empty((B, Hq, N), dtype=torch.float32).pin_memory()
+            ins = (pin(q), pin(k), pin(v))
+            sa.fwd_host(*ins, mask, p, Oh, Lh, ws, wait=False)
+            runs.append((q, k, v, ins, Oh, Lh))
+        torch.cuda.synchronize()
+        assert sa.check_device() == sa.SA_OK
+        for q, k, v, _, Oh, Lh in runs:
+            O, LSE = run_gpu(q, k, v, p, 128, 1 / math.sqrt(D))
+            assert np.array_equal(Oh.float().numpy(), O) and np.array_equal(Lh.numpy(), LSE)
+    finally:
+        sa.set_debug(0)
+    Oref, Lref = oracle.attention(q, k, v, oracle.Pattern(window=300, sinks=4), 1 / math.sqrt(D))
+    compare(Oh.float().numpy(), Lh.numpy(), Oref, Lref)
 
 
 def test_device_timeout_is_reported_and_context_survives():
