@@ -167,11 +167,32 @@ class BlockMask:
                           self._ptr(self.counts) if T else None, self._ptr(self.index) if T else None,
                           self._ptr(self.full) if T else None)
 
+    @property
+    def on_host(self) -> bool:
+        return isinstance(self.counts, np.ndarray)
+
     def to_device(self, device) -> "BlockMask":
         import torch
         t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
         return BlockMask(t(self.counts), t(self.index), t(self.full), self.block, self.n_live,
                          self.n_full, self.max_per_row, self.N)
+
+
+def _host_masks(where: str, *masks) -> None:
+    """The call reads the mask's arrays on the host: numpy, not a device copy
+    (whose addresses the host cannot read)."""
+    for m in masks:
+        if not m.on_host:
+            raise TypeError(f"{where} takes the host block mask (numpy arrays), not a device copy")
+
+
+def _device_masks(where: str, device, *masks) -> None:
+    """The call's kernels read the mask's arrays: a copy on the tensors' device
+    (``to_device``), not host arrays."""
+    for m in masks:
+        c = m.counts
+        if m.on_host or not getattr(c, "is_cuda", False) or c.device != device:
+            raise TypeError(f"{where} takes the block mask on the tensors' device (BlockMask.to_device)")
 
 
 def num_tiles(N: int, block: int) -> int:
@@ -198,6 +219,7 @@ def transpose_block_mask(mask: BlockMask) -> BlockMask:
     """Per-kv-tile lists of the query tiles that attend to it (host arrays);
     ``counts[c]``, ``index[c, e]`` and ``full[c, e]`` with rows and columns
     swapped relative to ``mask``.  The backward pass takes this form."""
+    _host_masks("transpose_block_mask", mask)
     T = mask.T
     counts = np.zeros(T, dtype=np.int32)
     index = np.zeros((T, T), dtype=np.int32)
@@ -261,6 +283,7 @@ def fwd(q, k, v, mask: BlockMask, pattern: Pattern, scale: float | None = None, 
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _device_masks("fwd", q.device, mask)
     shape = _Shape(B, Hq, Hkv, N, D)
     with torch.cuda.device(q.device):
         st = _stream_handle(stream, q.device)
@@ -296,6 +319,7 @@ def fwd_heads(q, k, v, masks, patterns, head_pattern, scale: float | None = None
     cmasks = (_BlockMask * max(n, 1))(*[m._c() for m in masks])
     cpats = (_Pattern * max(n, 1))(*[p_._c() for p_ in patterns])
     heads = (ctypes.c_int32 * max(len(head_pattern), 1))(*[int(h) for h in head_pattern])
+    _device_masks("fwd_heads", q.device, *masks)
     shape = _Shape(B, Hq, Hkv, N, D)
     with torch.cuda.device(q.device):
         st = _stream_handle(stream, q.device)
@@ -336,6 +360,7 @@ def bwd(q, k, v, o, lse, do, mask_t: BlockMask, pattern: Pattern, scale: float |
     need = bwd_workspace_bytes(B, Hq, Hkv, N, D)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _device_masks("bwd", q.device, mask_t)
     shape = _Shape(B, Hq, Hkv, N, D)
     with torch.cuda.device(q.device):
         st = _stream_handle(stream, q.device)
@@ -367,6 +392,7 @@ def fwd_stride(q, k, v, pass1: BlockMask, pass2: BlockMask, pattern: Pattern, sc
             raise TypeError("q, k, v must be contiguous bf16 CUDA tensors")
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _device_masks("fwd_stride", q.device, pass1, pass2)
     shape = _Shape(B, Hq, Hkv, N, D)
     n = ctypes.c_size_t(0)
     _check(lib.sparse_attn_fwd_stride_workspace(ctypes.byref(shape), ctypes.byref(n)), "sparse_attn_fwd_stride_workspace")
@@ -405,6 +431,7 @@ def bwd_heads(q, k, v, o, lse, do, masks_t, patterns, head_pattern, scale: float
     cmasks = (_BlockMask * max(n, 1))(*[m._c() for m in masks_t])
     cpats = (_Pattern * max(n, 1))(*[p_._c() for p_ in patterns])
     heads = (ctypes.c_int32 * max(len(head_pattern), 1))(*[int(h) for h in head_pattern])
+    _device_masks("bwd_heads", q.device, *masks_t)
     shape = _Shape(B, Hq, Hkv, N, D)
     with torch.cuda.device(q.device):
         st = _stream_handle(stream, q.device)
@@ -431,8 +458,7 @@ def fwd_host(q_host, k_host, v_host, mask: BlockMask, pattern: Pattern, o_host, 
     ``wait=False`` the call only queues the work (sparse_attn_fwd_host_async):
     ``stream`` reaches its end once O and LSE are in host memory, and successive
     calls overlap their input and output copies."""
-    if not isinstance(mask.counts, np.ndarray):
-        raise TypeError("fwd_host takes the host block mask (numpy arrays), not a device copy")
+    _host_masks("fwd_host", mask)
     B, Hq, N, D = q_host.shape
     Hkv = k_host.shape[1]
     if scale is None:
@@ -463,6 +489,7 @@ def fwd_noalloc(q, k, v, mask: BlockMask, pattern: Pattern, out, lse, scale: flo
     B, Hq, N, D = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    _host_masks("fwd_noalloc", mask)
     shape = _Shape(B, Hq, k.shape[1], N, D)
     with torch.cuda.device(q.device):
         st = _stream_handle(stream, q.device)

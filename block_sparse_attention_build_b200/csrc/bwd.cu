@@ -176,6 +176,8 @@ int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const f
     if (workspace_bytes < bwd_layout(s).total) return SA_ERR_BUFFER_TOO_SMALL;
     const int64_t rows = int64_t(s.B) * s.Hq * s.N;
     if (int64_t(s.B) * s.Hkv * T > INT32_MAX || (rows + 7) / 8 > INT32_MAX) return SA_ERR_UNSUPPORTED;
+    for (int i = 0; i < n_patterns; i++)  // the first CUDA call of the path
+        if (int rc = check_device_mask(&masks_t[i])) return rc;
     BwdHeads hb{};
     for (int i = 0; i < n_patterns; i++) {
         const sa_pattern& pt = patterns[i];

@@ -168,6 +168,8 @@ int fwd_impl(const void* Q, const void* K, const void* V, const sa_block_mask* m
     // LSE is written one fp32 at a time: 4-byte alignment is enough
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || (reinterpret_cast<uintptr_t>(LSE) & 3u))
         return SA_ERR_MISALIGNED;
+    for (int i = 0; i < n_patterns; i++)  // the first CUDA call of the path
+        if (int rc = check_device_mask(&masks[i])) return rc;
     const int64_t n_qtiles = (int64_t(s.N) + kBM - 1) / kBM;
     const int64_t group = s.Hq / s.Hkv;
     // work units: two 128-row query tiles that share a key/value head
@@ -305,6 +307,24 @@ int check_host_mask(const sa_block_mask* m, int64_t T)
 }
 
 int device_sm_count() { return sm_count(); }
+
+int check_device_mask(const sa_block_mask* m)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+    const void* arrays[3] = {m->kv_count, m->kv_index, m->kv_full};
+    for (const void* a : arrays) {
+        cudaPointerAttributes at;
+        if (cudaPointerGetAttributes(&at, a) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return SA_ERR_INVALID_ARG;
+        }
+        const bool ok = (at.type == cudaMemoryTypeDevice && at.device == dev) || at.type == cudaMemoryTypeManaged ||
+                        at.type == cudaMemoryTypeHost;
+        if (!ok) return SA_ERR_INVALID_ARG;
+    }
+    return SA_OK;
+}
 
 }  // namespace sa
 

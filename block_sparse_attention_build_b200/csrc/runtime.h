@@ -19,4 +19,10 @@ int device_sm_count();                  // 0 when the query fails
 // full flags 0 or 1.  SA_OK or SA_ERR_INVALID_ARG; O(T^2).
 int check_host_mask(const sa_block_mask* m, int64_t T);
 
+// The arrays of a block mask that a kernel reads are readable by the current
+// device: its own memory, managed memory or pinned host memory (pageable host
+// memory or another device's memory would fault the kernel).  SA_OK,
+// SA_ERR_INVALID_ARG, or SA_ERR_CUDA when the device query fails.
+int check_device_mask(const sa_block_mask* m);
+
 }  // namespace sa

@@ -133,7 +133,9 @@ int sparse_attn_count_pairs(const sa_pattern* pattern, int64_t N, int64_t* pairs
  * Forward pass on the GPU.  Q, K, V, O, LSE are device pointers (Q, K, V, O
  * 16-byte aligned, LSE 4-byte aligned) in the layouts above; `mask` holds DEVICE copies of the arrays
  * built by sparse_attn_build_block_mask for this pattern, N and block (its
- * scalar fields as the builder returned them).  scale > 0 multiplies q.k
+ * scalar fields as the builder returned them); arrays that the current device
+ * cannot read (pageable host memory, another device's memory) are refused with
+ * SA_ERR_INVALID_ARG before any launch.  scale > 0 multiplies q.k
  * (1/sqrt(D) in the pages' prototype).  `stream` is a cudaStream_t (NULL: the
  * legacy default stream).  Asynchronous: returns once the kernel is queued;
  * launch errors come back as SA_ERR_CUDA, a device-side timeout through
@@ -318,12 +320,14 @@ int sparse_attn_bwd_workspace(const sa_shape* shape, size_t* bytes);
  *   Q, O, dO, dQ [B, Hq, N, D] bf16;  K, V, dK, dV [B, Hkv, N, D] bf16;
  *   LSE [B, Hq, N] fp32 as written by sparse_attn_fwd (natural log).
  *   mask_t     the TRANSPOSED block mask (sparse_attn_transpose_block_mask of
- *              the pattern's mask) with its arrays in device memory; block 128
+ *              the pattern's mask) with its arrays in device memory (checked as
+ *              for sparse_attn_fwd); block 128
  *   pattern    the pattern the mask was compiled from (partial tiles are
  *              masked element by element from it)
  *   workspace  device memory of at least sparse_attn_bwd_workspace bytes,
  *              256-byte aligned; caller-owned, contents need not be preserved
- * Launches three kernels on `stream` and returns without waiting; the
+ * Launches four kernels on `stream` (work items, row sums, the main kernel,
+ * dQ conversion) and returns without waiting; the
  * workspace must not be reused until they finish.  The caller owns every
  * buffer.  Errors as sparse_attn_fwd, plus SA_ERR_UNSUPPORTED for a mask block
  * other than 128 and SA_ERR_BUFFER_TOO_SMALL for a short workspace; a bounded

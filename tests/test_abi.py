@@ -469,3 +469,21 @@ def test_headline_tile_lists_are_a_diagonal_band_plus_the_sink_column():
         full = {int(j) for j, f in zip(m.index[i, : m.counts[i]], m.full[i, : m.counts[i]]) if f}
         # full: the tiles strictly inside the band (1 <= i - j <= 7)
         assert full == set(range(max(0, i - 7), i)), i
+
+
+def test_binding_refuses_a_mask_in_the_wrong_memory():
+    """Host-side calls take numpy masks, device calls a copy on the tensors'
+    device: a mask in the other memory is a TypeError in the binding, before
+    the library could read host addresses on the device or the reverse."""
+    import torch
+    m = sa.build_block_mask(sa.Pattern(window=100, sinks=4), 1000, 128)
+    as_torch = sa.BlockMask(*(torch.from_numpy(a) for a in (m.counts, m.index, m.full)),
+                            m.block, m.n_live, m.n_full, m.max_per_row, m.N)
+    assert m.on_host and not as_torch.on_host
+    with pytest.raises(TypeError, match="host block mask"):
+        sa.transpose_block_mask(as_torch)
+    with pytest.raises(TypeError, match="host block mask"):
+        sa._host_masks("fwd_noalloc", as_torch)
+    for mask in (m, as_torch):  # numpy arrays, or torch tensors in host memory
+        with pytest.raises(TypeError, match="tensors' device"):
+            sa._device_masks("fwd", torch.device("cuda", 0), mask)

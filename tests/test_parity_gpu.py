@@ -412,3 +412,44 @@ def test_stride_aware_workload_sampled():
     # and the plain path on the same inputs agrees within the bars
     O2, LSE2 = run_gpu(q, k, v, p, w.block, w.scale)
     assert np.abs(O - O2).max() <= O_TOL and np.abs(LSE - LSE2).max() <= LSE_TOL
+
+
+def test_mask_the_device_cannot_read_is_refused():
+    """Through the C ABI: a mask in pageable host memory is refused with
+    SA_ERR_INVALID_ARG before any launch (forward and backward); one in pinned
+    host memory, which the device reads over the bus, gives the device mask's
+    output bit for bit."""
+    import ctypes
+    B, Hq, Hkv, N, D = 1, 2, 1, 600, 64
+    p = sa.Pattern(window=150, sinks=4)
+    q, k, v = synth.qkv(B, Hq, Hkv, N, D, seed=77)
+    Q, K, V = to_dev(q), to_dev(k), to_dev(v)
+    hmask = sa.build_block_mask(p, N, 128)
+    O_ref, L_ref = sa.fwd(Q, K, V, hmask.to_device("cuda"), p)
+    torch.cuda.synchronize()
+
+    def c_fwd(mask, O, L):
+        return sa.lib.sparse_attn_fwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), ctypes.byref(mask._c()),
+                                      ctypes.byref(p._c()), ctypes.byref(sa._Shape(B, Hq, Hkv, N, D)),
+                                      1 / math.sqrt(D), O.data_ptr(), L.data_ptr(), None)
+
+    O = torch.full_like(O_ref, float("nan"))
+    L = torch.full_like(L_ref, float("nan"))
+    assert c_fwd(hmask, O, L) == sa.SA_ERR_INVALID_ARG  # numpy: pageable host memory
+    torch.cuda.synchronize()
+    assert torch.isnan(O.float()).all() and torch.isnan(L).all()  # nothing ran
+    pinned = sa.BlockMask(*(torch.from_numpy(a).pin_memory() for a in (hmask.counts, hmask.index, hmask.full)),
+                          hmask.block, hmask.n_live, hmask.n_full, hmask.max_per_row, N)
+    assert c_fwd(pinned, O, L) == sa.SA_OK
+    torch.cuda.synchronize()
+    assert sa.check_device() == sa.SA_OK
+    assert torch.equal(O, O_ref) and torch.equal(L, L_ref)
+
+    ht = sa.transpose_block_mask(hmask)
+    g = [torch.empty_like(t) for t in (Q, K, V)]
+    ws = torch.empty(sa.bwd_workspace_bytes(B, Hq, Hkv, N, D), dtype=torch.uint8, device="cuda")
+    rc = sa.lib.sparse_attn_bwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O_ref.data_ptr(), L_ref.data_ptr(),
+                                Q.data_ptr(), ctypes.byref(ht._c()), ctypes.byref(p._c()),
+                                ctypes.byref(sa._Shape(B, Hq, Hkv, N, D)), 1 / math.sqrt(D), g[0].data_ptr(),
+                                g[1].data_ptr(), g[2].data_ptr(), ws.data_ptr(), ws.numel(), None)
+    assert rc == sa.SA_ERR_INVALID_ARG
