@@ -487,3 +487,27 @@ def test_binding_refuses_a_mask_in_the_wrong_memory():
     for mask in (m, as_torch):  # numpy arrays, or torch tensors in host memory
         with pytest.raises(TypeError, match="tensors' device"):
             sa._device_masks("fwd", torch.device("cuda", 0), mask)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No fallback: without the built library the binding refuses to load."""
+    monkeypatch.setattr(sa, "LIB_PATH", str(tmp_path / "libsparse_attn.so"))
+    with pytest.raises(ImportError, match="missing"):
+        sa._load()
+
+
+def test_product_and_oracle_share_no_code():
+    """The package (binding and CUDA sources) never names the oracle, and the
+    oracle never names the package, its library or its headers."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "block_sparse_attention_build_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert re.search(r"\boracle\b", text) is None, f
+    for f in os.listdir(os.path.join(root, "oracle")):
+        if f.endswith((".py", ".c", ".h")):
+            text = open(os.path.join(root, "oracle", f), encoding="utf-8").read()
+            for name in ("block_sparse_attention_build_b200", "sparse_attn.h", "libsparse_attn", "sparse_attn_"):
+                assert name not in text, (f, name)
