@@ -453,3 +453,24 @@ def test_mask_the_device_cannot_read_is_refused():
                                 ctypes.byref(sa._Shape(B, Hq, Hkv, N, D)), 1 / math.sqrt(D), g[0].data_ptr(),
                                 g[1].data_ptr(), g[2].data_ptr(), ws.data_ptr(), ws.numel(), None)
     assert rc == sa.SA_ERR_INVALID_ARG
+
+
+def test_host_buffer_entry_point_at_the_headline_size():
+    """The host-buffer path on the full headline workload (16 heads cut into
+    chunks of 8, 4, 2, 1, 1): sampled rows against the oracle, and the whole
+    output against the device call within rounding (the chunks are smaller
+    problems than the whole, so their work plans may split units differently)."""
+    w = WORKLOADS["w1024_s4_n8192"]
+    q, k, v = synth.qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=w.seed)
+    p = sa.Pattern(**w.pattern_args())
+    O, LSE = run_gpu(q, k, v, p, w.block, w.scale)
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Oh = torch.empty((w.B, w.Hq, w.N, w.D), dtype=torch.bfloat16).pin_memory()
+    Lh = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32).pin_memory()
+    ws = torch.empty(sa.fwd_host_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.D), dtype=torch.uint8, device="cuda")
+    sa.fwd_host(pin(q), pin(k), pin(v), sa.build_block_mask(p, w.N, w.block), p, Oh, Lh, ws, scale=w.scale)
+    Oh, Lh = Oh.float().numpy(), Lh.numpy()
+    assert np.abs(Oh - O).max() <= 1e-2 and np.abs(Lh - LSE).max() <= 1e-4
+    rows = sample_rows(w.N, extra=64)
+    Oref, LSEref = oracle.attention(q, k, v, opattern(p), w.scale, rows=rows)
+    compare(Oh[:, :, rows], Lh[:, :, rows], Oref, LSEref)

@@ -106,3 +106,32 @@ def test_noalloc_reports_a_device_timeout_and_recovers():
     O_ref, L_ref = sa.fwd(q, k, v, host_mask.to_device("cuda"), p, scale=1 / math.sqrt(D))
     assert sa.check_device() == sa.SA_OK
     assert torch.equal(O, O_ref) and torch.equal(L, L_ref)
+
+
+@pytest.mark.gpu
+def test_noalloc_at_the_largest_mask_its_scratch_holds():
+    """T = 457 tiles per side (N = 58 496 at block 128, ragged by 37 rows), the
+    largest mask the static scratch takes: bit for bit against sparse_attn_fwd
+    and, on sampled rows, within the parity bars against the oracle."""
+    import torch
+
+    import oracle
+
+    N, D = 457 * 128 - 37, 64
+    p = sa.Pattern(window=500, sinks=4)
+    q, k, v = synth.qkv(1, 2, 1, N, D, seed=12)
+    t = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    Q, K, V = t(q), t(k), t(v)
+    host_mask = sa.build_block_mask(p, N, 128)
+    O_ref, L_ref = sa.fwd(Q, K, V, host_mask.to_device("cuda"), p, scale=1 / math.sqrt(D))
+    O = torch.empty_like(Q)
+    L = torch.empty_like(L_ref)
+    assert _noalloc(Q, K, V, host_mask, p, 1 / math.sqrt(D), O, L) == sa.SA_OK
+    torch.cuda.synchronize()
+    assert torch.equal(O, O_ref) and torch.equal(L, L_ref)
+    rows = np.unique(np.concatenate([np.arange(0, N, 128), np.arange(127, N, 128), [N - 1],
+                                     np.random.default_rng(0).integers(0, N, 64)]))
+    Oref, Lref = oracle.attention(q, k, v, oracle.Pattern(window=500, sinks=4), 1 / math.sqrt(D), rows=rows)
+    Og = O.float().cpu().numpy()[:, :, rows]
+    Lg = L.cpu().numpy()[:, :, rows]
+    assert np.abs(Og - Oref).max() <= O_TOL and np.abs(Lg - Lref).max() <= LSE_TOL
