@@ -20,8 +20,8 @@ e2e        the same metric through the host-buffer C ABI call (pinned host
            one blocking call is reported beside it.
 cpu_baseline  the fp64 CPU oracle on a bounded row sample, host cores.
 
-With --pass bwd one step is one backward pass (three launches: prep, the
-tensor-core kernel, dQ conversion) for an upstream gradient dO, with the
+With --pass bwd one step is one backward pass (four launches: work items,
+prep, the tensor-core kernel, dQ conversion) for an upstream gradient dO, with the
 forward's O and LSE computed once before timing; value counts 10 * D useful
 FLOP per allowed pair (S, dP, dV, dK, dQ) and the roofline takes the whole
 step's device time (the launch list in profiles/ gives each kernel's share).
@@ -335,6 +335,10 @@ def run_gpu(args, w):
     p, mask_h, pairs, useful, executed, min_bytes = workload_counts(w)
     mask = mask_h.to_device(dev)
     stride_path = args.path == "stride"
+    # the stride-aware path reads pass 2 through grouped views (no copies) when the
+    # residue groups (N / stride tokens each) fill whole tiles
+    n_group = w.N // max(w.stride, 1)
+    grouped_in_place = n_group % 128 == 0 and n_group % w.block == 0
     if stride_path:
         if w.stride <= 0:
             raise SystemExit("--path stride needs a workload with a stride")
@@ -484,14 +488,14 @@ def run_gpu(args, w):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None if stride_path else profiled_traffic(w.name),
                      "kernel": (("stride-aware step: 2 x fwd_kernel + merge"
-                                 + ("" if (w.N // max(w.stride, 1)) % 128 == 0 and (w.N // max(w.stride, 1)) % w.block == 0
-                                    else " + 3 grouping copies")) if stride_path else "fwd_kernel<D,BN>"),
+                                 + ("" if grouped_in_place else " + 3 grouping copies")) if stride_path
+                                else "fwd_kernel<D,BN>"),
                      "mean_launch_us": mean_launch_ms * 1e3,
                      "algorithmic_flop_per_launch": executed,
                      "hbm_gbs_min_bytes": min_bytes / (mean_launch_ms * 1e-3) / 1e9},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * ((3 if grouped_in_place else 6) if stride_path else 1),
         "clocks": clocks.summary(),
     }
     print(json.dumps(line))
@@ -635,11 +639,11 @@ def run_gpu_bwd(args, w):
         "peak_kind": f"bf16 dense, {peak_kind} ({peak} TFLOP/s burst)",
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None,
-                     "kernel": "backward step: bwd_prep_kernel + bwd_kernel<D> + bwd_dq_kernel",
+                     "kernel": "backward step: bwd_items_kernel + bwd_prep_kernel + bwd_kernel<D> + bwd_dq_kernel",
                      "mean_step_us": step_ms * 1e3, "algorithmic_flop_per_step": executed},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 4 * args.steps,
         "clocks": clocks.summary(),
     }
     print(json.dumps(line))
